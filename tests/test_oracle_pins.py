@@ -1,0 +1,409 @@
+"""Pins of the fp64 CPU oracle against what mathematics and the pages fix.
+
+Each test ties one oracle function to something other than itself: a library
+routine (numpy complex arithmetic, torch's scaled_dot_product_attention and
+dtype casts), a closed form, an invariant, a brute-force simulation, or a
+degenerate case with a known answer. A plausible mistake (dropped term, wrong
+sign or index, transposed operand, wrong eviction) fails at least one.
+"""
+import collections
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from inputgen import spec_for, Q, K, V
+from inputgen.workloads import Workload, NORMAL, UNIFORM, ZERO, ONES
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+# tiny shapes: H=2, D=12 (bands 4/4/4), 2x3 tokens per frame
+TINY = Workload("tiny_pins", B=1, H=2, D=12, fh=2, fw=3, C=2, S=1, W=2, n_chunks=12,
+                dtype="f32", rope_dims=(4, 4, 4), refresh_period=0)
+
+
+def _cfg(w, store=O.EXACT, period=None):
+    return O.cfg_for(w, store=store, refresh_period=period)
+
+
+def _all_rows(w):
+    toks = np.repeat(np.arange(w.Lc), w.H)
+    heads = np.tile(np.arange(w.H), w.Lc)
+    return toks, heads
+
+
+# --------------------------------------------------------------------------
+# storage rounding == library casts
+# --------------------------------------------------------------------------
+def test_round_store_bf16_matches_torch_cast():
+    rng = np.random.default_rng(1)
+    x32 = (rng.standard_normal(4000) * 10.0 ** rng.integers(-6, 6, 4000)).astype(np.float32)
+    ref = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([O.round_store(O.STORE_BF16, float(v)) for v in x32])
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_round_store_bf16_ties_to_even():
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: even mantissa wins (1.0)
+    assert O.round_store(O.STORE_BF16, 1.0 + 2.0 ** -8) == 1.0
+    # 1 + 3*2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6: goes to 1 + 2^-6
+    assert O.round_store(O.STORE_BF16, 1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert O.round_store(O.STORE_BF16, -(1.0 + 3 * 2.0 ** -8)) == -(1.0 + 2.0 ** -6)
+    assert O.round_store(O.STORE_BF16, 0.0) == 0.0
+
+
+def test_round_store_f32_matches_numpy_cast():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal(2000) * 1e3
+    got = np.array([O.round_store(O.STORE_F32, float(v)) for v in x])
+    np.testing.assert_array_equal(got, x.astype(np.float32).astype(np.float64))
+    assert O.round_store(O.EXACT, 0.1) == 0.1
+
+
+# --------------------------------------------------------------------------
+# 3D RoPE == complex multiplication per pair
+# --------------------------------------------------------------------------
+def test_rope_unit_frequency_is_complex_rotation():
+    # D = 6 with bands 2/2/2: every band has a single pair with theta_0 = 1, so
+    # the pair of band b turns by exactly pos_b radians.
+    w = TINY.with_(D=6, rope_dims=(2, 2, 2))
+    cfg = _cfg(w)
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        x = rng.standard_normal(6)
+        pos = rng.uniform(-50, 50, 3)
+        got = O.rope_vec(cfg, x, *pos)
+        z = (x[0::2] + 1j * x[1::2]) * np.exp(1j * pos)
+        np.testing.assert_allclose(got[0::2], z.real, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(got[1::2], z.imag, rtol=0, atol=1e-13)
+
+
+def test_rope_frequency_ladder_values():
+    # base 10000: 10000^(-1/2) = 0.01 is pair 1 of a 4-wide band and pair 11 of
+    # the 44-wide temporal band at D = 128.
+    cfg = _cfg(TINY)
+    assert O.theta(cfg, 0, 0) == 1.0
+    assert abs(O.theta(cfg, 1, 1) - 0.01) < 1e-17
+    w128 = TINY.with_(D=128, rope_dims=(44, 42, 42))
+    assert abs(O.theta(_cfg(w128), 0, 11) - 0.01) < 1e-17
+    # the rotated pair 1 of the h band (dims 6,7 at D=12) turns by 0.01 * y
+    x = np.zeros(12)
+    x[6] = 1.0
+    y = 37.0
+    got = O.rope_vec(cfg, x, 0.0, y, 0.0)
+    z = np.exp(1j * 0.01 * y)
+    assert abs(got[6] - z.real) < 1e-15 and abs(got[7] - z.imag) < 1e-15
+    np.testing.assert_array_equal(np.delete(got, [6, 7]), 0.0)
+
+
+def test_rope_isometry_identity_group_and_relative_property():
+    w = TINY.with_(D=64, rope_dims=(24, 20, 20))
+    cfg = _cfg(w)
+    rng = np.random.default_rng(4)
+    for _ in range(20):
+        x, k = rng.standard_normal(64), rng.standard_normal(64)
+        a, b = rng.uniform(-1e3, 1e3, 3), rng.uniform(-1e3, 1e3, 3)
+        rx = O.rope_vec(cfg, x, *a)
+        assert abs(np.linalg.norm(rx) - np.linalg.norm(x)) < 1e-12
+        np.testing.assert_array_equal(O.rope_vec(cfg, x, 0.0, 0.0, 0.0), x)
+        np.testing.assert_allclose(O.rope_vec(cfg, rx, *b), O.rope_vec(cfg, x, *(a + b)),
+                                   atol=1e-10)
+        # <R(a) x, R(b) k> = <R(a - b) x, k>
+        lhs = O.rope_vec(cfg, x, *a) @ O.rope_vec(cfg, k, *b)
+        rhs = O.rope_vec(cfg, x, *(a - b)) @ k
+        assert abs(lhs - rhs) < 1e-9
+
+
+def test_rope_tband_rotates_only_temporal_band():
+    cfg = _cfg(TINY.with_(D=64, rope_dims=(24, 20, 20)))
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(64)
+    got = O.rope_tband(cfg, x, 3.5)
+    np.testing.assert_allclose(got, O.rope_vec(cfg, x, 3.5, 0.0, 0.0), atol=1e-15)
+    np.testing.assert_array_equal(got[24:], x[24:])
+
+
+# --------------------------------------------------------------------------
+# refresh schedule: "rebase t to 0 keeping relative offsets"
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("C,S,W,period", [(2, 1, 4, 3), (1, 1, 2, 4), (2, 1, 8, 5), (1, 0, 0, 2),
+                                          (3, 2, 3, 1)])
+def test_refresh_rebases_oldest_visible_frame_to_zero(C, S, W, period):
+    w = TINY.with_(C=C, S=S, W=W)
+    cfg = _cfg(w, period=period)
+    assert O.base_at(cfg, 0) == 0
+    prev = 0
+    for c in range(1, 60):
+        base = O.base_at(cfg, c)
+        if c % period == 0:
+            assert O.refresh_due(cfg, c)
+            visible_nonsink = [f for f in range((c + 1) * C) if O.visible(cfg, c, f) and f >= S]
+            assert base == min(visible_nonsink)  # oldest non-sink frame gets t = 0
+            assert base >= prev
+        else:
+            assert not O.refresh_due(cfg, c)
+            assert base == prev
+        prev = base
+    assert O.base_at(_cfg(w, period=0), 59) == 0
+
+
+# --------------------------------------------------------------------------
+# ring buffer: closed form == a plain slot-array simulation with eviction
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("C,S,W", [(1, 1, 2), (2, 1, 4), (1, 1, 6), (1, 1, 3), (2, 1, 8),
+                                   (2, 0, 0), (1, 0, 3), (3, 2, 3), (2, 2, 2), (1, 3, 2)])
+def test_ring_slots_match_simulation_and_visibility(C, S, W):
+    w = TINY.with_(C=C, S=S, W=W)
+    cfg = _cfg(w)
+    R = W + C
+    sink = [-1] * S
+    ring = [-1] * R
+    wp = 0  # next ring slot to write
+    window = collections.deque(maxlen=R)
+    for c in range(300):
+        for f in range(c * C, (c + 1) * C):
+            if f < S:
+                sink[f] = f
+            else:
+                ring[wp] = f
+                wp = (wp + 1) % R
+                window.append(f)
+            assert O.frame_slot(cfg, f) == (f if f < S else S + ring.index(f))
+        np.testing.assert_array_equal(O.slot_frames(cfg, c), np.array(sink + ring))
+        held = {f for f in sink + ring if f >= 0}
+        vis = {f for f in range((c + 1) * C) if O.visible(cfg, c, f)}
+        assert held == vis, (c, held, vis)
+        assert set(window) == {f for f in vis if f >= S}
+        assert O.n_keys(cfg, c) == len(vis) * w.F
+
+
+# --------------------------------------------------------------------------
+# T1: cache path == brute-force masked full-sequence attention
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("C,S,W,period", [(2, 1, 2, 0), (2, 1, 2, 2), (1, 1, 2, 4), (1, 0, 2, 3),
+                                          (3, 2, 3, 1), (1, 1, 0, 2)])
+def test_cache_path_equals_bruteforce(C, S, W, period):
+    w = TINY.with_(C=C, S=S, W=W)
+    cfg = _cfg(w, period=period)
+    sp = spec_for(w)
+    toks, heads = _all_rows(w)
+    for c in range(0, 9):
+        a = O.attend_rows(cfg, sp, 0, c, toks, heads)
+        b = O.bruteforce_rows(cfg, sp, 0, c, toks, heads)
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12, err_msg=f"chunk {c}")
+
+
+# --------------------------------------------------------------------------
+# T6: brute force == torch SDPA (fp64, boolean mask) on the same rotated q, k
+# --------------------------------------------------------------------------
+def test_bruteforce_matches_torch_sdpa():
+    w = TINY.with_(D=12, C=2, S=1, W=2)
+    cfg = _cfg(w)
+    sp = spec_for(w)
+    c = 5
+    F, H, D = w.F, w.H, w.D
+    nf = (c + 1) * w.C
+    kraw = np.concatenate([O.input_block(cfg, sp, 0, ch, K) for ch in range(c + 1)])
+    vraw = np.concatenate([O.input_block(cfg, sp, 0, ch, V) for ch in range(c + 1)])
+    qraw = O.input_block(cfg, sp, 0, c, Q)
+
+    def pos(frame, j):
+        return float(frame), float(j // w.fw), float(j % w.fw)
+
+    kr = np.stack([[O.rope_vec(cfg, kraw[i, h], *pos(i // F, i % F)) for h in range(H)]
+                   for i in range(nf * F)])
+    qr = np.stack([[O.rope_vec(cfg, qraw[i, h], *pos(c * w.C + i // F, i % F)) for h in range(H)]
+                   for i in range(w.Lc)])
+    # mask, written from the rule: block-causal, sink frames always, window of W
+    allowed = np.zeros((w.Lc, nf * F), dtype=bool)
+    for i in range(w.Lc):
+        fq = c * w.C + i // F
+        for j in range(nf * F):
+            fk = j // F
+            allowed[i, j] = fk < (fq // w.C + 1) * w.C and (fk < w.S or fk >= (fq // w.C) * w.C - w.W)
+    qt = torch.from_numpy(qr).permute(1, 0, 2)[None]
+    kt = torch.from_numpy(kr).permute(1, 0, 2)[None]
+    vt = torch.from_numpy(vraw).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt, vt, attn_mask=torch.from_numpy(allowed)).numpy()[0]  # [H, Lc, D]
+    toks, heads = _all_rows(w)
+    got = O.bruteforce_rows(cfg, sp, 0, c, toks, heads)
+    np.testing.assert_allclose(got, ref[heads, toks], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# T2: refresh invariance of the scores (exact arithmetic)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("period", [1, 2, 3, 5])
+def test_refresh_invariance_exact(period):
+    w = TINY.with_(C=2, S=1, W=4)
+    sp = spec_for(w)
+    toks, heads = _all_rows(w)
+    for c in range(0, 12):
+        a = O.attend_rows(_cfg(w, period=period), sp, 0, c, toks, heads)
+        b = O.attend_rows(_cfg(w, period=0), sp, 0, c, toks, heads)
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-10)
+
+
+def test_refresh_invariance_far_position():
+    # after 10,000 chunks with a refresh every 256, the sink sits near t = -2e4
+    w = TINY.with_(C=2, S=1, W=8, D=64, rope_dims=(24, 20, 20))
+    sp = spec_for(w)
+    c = 10000
+    cfg = _cfg(w, period=256)
+    assert O.base_at(cfg, c) > 19000
+    toks, heads = _all_rows(w)
+    a = O.attend_rows(cfg, sp, 0, c, toks, heads)
+    b = O.attend_rows(_cfg(w, period=0), sp, 0, c, toks, heads)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-9)
+
+
+# --------------------------------------------------------------------------
+# T3: window = 0 reduces to attention over sink + own chunk (torch SDPA)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("C,S", [(1, 1), (2, 1), (2, 2), (1, 0)])
+def test_window_zero_is_sink_plus_self(C, S):
+    w = TINY.with_(C=C, S=S, W=0)
+    cfg = _cfg(w)
+    sp = spec_for(w)
+    F, H = w.F, w.H
+    for c in (0, 1, 4):
+        frames = sorted(set(range(min(S, (c + 1) * C))) | set(range(c * C, (c + 1) * C)))
+        ks, vs = [], []
+        for f in frames:
+            blk_k = O.input_block(cfg, sp, 0, f // C, K)
+            blk_v = O.input_block(cfg, sp, 0, f // C, V)
+            for j in range(F):
+                i = (f % C) * F + j
+                ks.append([O.rope_vec(cfg, blk_k[i, h], f, j // w.fw, j % w.fw) for h in range(H)])
+                vs.append(blk_v[i])
+        qb = O.input_block(cfg, sp, 0, c, Q)
+        qs = [[O.rope_vec(cfg, qb[i, h], c * C + i // F, (i % F) // w.fw, (i % F) % w.fw)
+               for h in range(H)] for i in range(w.Lc)]
+        qt = torch.tensor(np.array(qs)).permute(1, 0, 2)[None]
+        kt = torch.tensor(np.array(ks)).permute(1, 0, 2)[None]
+        vt = torch.tensor(np.array(vs)).permute(1, 0, 2)[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).numpy()[0]
+        toks, heads = _all_rows(w)
+        got = O.attend_rows(cfg, sp, 0, c, toks, heads)
+        np.testing.assert_allclose(got, ref[heads, toks], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# T5: closed-form special cases
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("store", [O.EXACT, O.STORE_BF16])
+def test_constant_values_give_constant_output(store):
+    w = TINY.with_(dist=(NORMAL, NORMAL, ONES), dtype="bf16", refresh_period=3)
+    cfg = _cfg(w, store=store)
+    toks, heads = _all_rows(w)
+    for c in (0, 3, 7):
+        got = O.attend_rows(cfg, spec_for(w), 0, c, toks, heads)
+        np.testing.assert_allclose(got, 1.0, rtol=0, atol=1e-14)
+
+
+def test_zero_queries_give_mean_of_visible_values():
+    w = TINY.with_(dist=(ZERO, NORMAL, UNIFORM), C=2, S=1, W=2)
+    cfg = _cfg(w)
+    sp = spec_for(w)
+    F = w.F
+    toks, heads = _all_rows(w)
+    for c in (0, 1, 2, 6):
+        vis = [f for f in range((c + 1) * w.C) if f < w.S or f >= c * w.C - w.W]
+        vals = np.concatenate([O.input_block(cfg, sp, 0, f // w.C, V)[(f % w.C) * F:(f % w.C + 1) * F]
+                               for f in vis])  # [n, H, D]
+        got = O.attend_rows(cfg, sp, 0, c, toks, heads)
+        np.testing.assert_allclose(got, vals.mean(axis=0)[heads], rtol=0, atol=1e-14)
+
+
+def test_single_visible_key_returns_its_value():
+    w = TINY.with_(fh=1, fw=1, C=1, S=0, W=0)
+    cfg = _cfg(w)
+    sp = spec_for(w)
+    for c in range(5):
+        got = O.attend_rows(cfg, sp, 0, c, [0, 0], [0, 1])
+        np.testing.assert_array_equal(got, O.input_block(cfg, sp, 0, c, V)[0])
+
+
+# --------------------------------------------------------------------------
+# storage-faithful mode == exact rotation + library rounding
+# --------------------------------------------------------------------------
+def _bf16(x):
+    # orc_round_store itself is pinned to torch's cast above; here the subject
+    # is which rotations and roundings a stored key goes through.
+    return np.array([O.round_store(O.STORE_BF16, float(v)) for v in np.ravel(x)]).reshape(np.shape(x))
+
+
+def test_stored_keys_bf16_history():
+    # period 3, C=1, W=2: ring frames live 3 chunks and cross at most one refresh
+    w = TINY.with_(C=1, S=1, W=2, dtype="bf16", refresh_period=3, D=64, rope_dims=(24, 20, 20))
+    cfg_s = _cfg(w, store=O.STORE_BF16)
+    sp = spec_for(w)
+    F, H = w.F, w.H
+    for c in range(0, 10):
+        base_c = O.base_at(cfg_s, c)
+        for f in range((c + 1) * w.C):
+            if not O.visible(cfg_s, c, f):
+                continue
+            got = O.stored_key_frame(cfg_s, sp, 0, f, c)
+            raw = O.input_block(cfg_s, sp, 0, f // w.C, K)[(f % w.C) * F:(f % w.C + 1) * F]
+            for j in range(F):
+                y, x = j // w.fw, j % w.fw
+                for h in range(H):
+                    if f < w.S:
+                        # the sink is re-derived from its raw key at every refresh
+                        ref = _bf16(O.rope_vec(cfg_s, raw[j, h], f - base_c, y, x))
+                    else:
+                        cw = f // w.C
+                        ref = _bf16(O.rope_vec(cfg_s, raw[j, h], f - O.base_at(cfg_s, cw), y, x))
+                        for r in range(cw + 1, c + 1):
+                            if O.refresh_due(cfg_s, r):
+                                d = O.base_at(cfg_s, r) - O.base_at(cfg_s, r - 1)
+                                ref = _bf16(O.rope_tband(cfg_s, ref, -d))
+                    np.testing.assert_array_equal(got[j, h], ref)
+
+
+def test_storage_f32_close_to_exact():
+    w = TINY.with_(refresh_period=2)
+    sp = spec_for(w)
+    toks, heads = _all_rows(w)
+    for c in (0, 3, 8):
+        a = O.attend_rows(_cfg(w, store=O.STORE_F32), sp, 0, c, toks, heads)
+        b = O.attend_rows(_cfg(w, store=O.EXACT), sp, 0, c, toks, heads)
+        np.testing.assert_allclose(a, b, rtol=0, atol=2e-6)
+
+
+def test_cache_contents_layout():
+    w = TINY.with_(C=2, S=1, W=2, dtype="bf16", refresh_period=0)
+    cfg = _cfg(w, store=O.STORE_BF16)
+    sp = spec_for(w)
+    F = w.F
+    for c in (0, 1, 2, 5):
+        k, v, sf = O.cache_contents(cfg, sp, 0, c)
+        np.testing.assert_array_equal(sf, O.slot_frames(cfg, c))
+        for s, f in enumerate(sf):
+            rows = slice(s * F, (s + 1) * F)
+            if f < 0:
+                assert not k[:, rows].any() and not v[:, rows].any()
+                continue
+            kf = O.stored_key_frame(cfg, sp, 0, f, c)  # [F, H, D]
+            vf = O.input_block(cfg, sp, 0, f // w.C, V)[(f % w.C) * F:(f % w.C + 1) * F]
+            np.testing.assert_array_equal(k[:, rows], kf.transpose(1, 0, 2))
+            np.testing.assert_array_equal(v[:, rows], vf.transpose(1, 0, 2))
+
+
+def test_softmax_scale_default():
+    # scores are scaled by 1/sqrt(D): doubling every raw q and every raw k
+    # multiplies each score by 4; with constant V the output must not move, and
+    # with Q = 0 it is the plain mean -- both covered above; here check the
+    # explicit scale field is honoured (scale = 1/sqrt(D) gives the default).
+    w = TINY
+    sp = spec_for(w)
+    toks, heads = _all_rows(w)
+    c0 = _cfg(w)
+    c1 = _cfg(w)
+    c1.scale = 1.0 / math.sqrt(w.D)
+    np.testing.assert_array_equal(O.attend_rows(c0, sp, 0, 3, toks, heads),
+                                  O.attend_rows(c1, sp, 0, 3, toks, heads))
