@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""Benchmark of the rolling-KV-cache attention hot path on B200.
+
+One step = one whole stream of the 512p-shaped workload (B=1, H=24, D=128,
+32x32-token frames, chunk 2 frames, sink 1 frame, window 4 frames, 64 chunks,
+RoPE refresh every 32 chunks) from an empty cache: per chunk the fused
+RoPE + append kernel and the tcgen05 attention kernel, plus the refresh.
+Inputs for every chunk of the step are resident in HBM before timing (2.4 GB
+per step, larger than the 126 MB L2, so every step starts cold).
+
+Prints one JSON line (rank 0). Under torchrun each rank streams its own
+independent streams (weak scaling, no collective on the data path); the
+timed region is bracketed by a barrier and synchronisation and the time is
+the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference implementation of
+this repository) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "streamed chunks/s and attention TFLOP/s (% of B200 BF16 peak) per config"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", default="512p_32x32_h24")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), float(m["bf16_tflops_sustained"]), \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        loaded = [r[0] for r in rows if r[2] > 300.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+def gpu_id_for(dev: int) -> str:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample(w, rank_stream: int = 0, budget_rows: int = 4096):
+    """Times the fp64 oracle on one steady-state chunk: key build plus
+    `budget_rows` output rows, extrapolated linearly to a whole chunk."""
+    import numpy as np
+
+    import oracle as O
+    from inputgen import spec_for
+    cfg = O.cfg_for(w)
+    spec = spec_for(w)
+    c = min(w.n_chunks - 1, max(3, w.refresh_period + 8 if w.refresh_period else 40))
+    t0 = time.perf_counter()
+    O.attend_rows(cfg, spec, rank_stream, c, np.zeros(0, np.int32), np.zeros(0, np.int32))
+    t_fixed = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    n = min(budget_rows, w.Lc * w.H)
+    toks = rng.integers(0, w.Lc, n).astype(np.int32)
+    heads = rng.integers(0, w.H, n).astype(np.int32)
+    t0 = time.perf_counter()
+    O.attend_rows(cfg, spec, rank_stream, c, toks, heads)
+    t_rows = time.perf_counter() - t0
+    per_row = max(t_rows - t_fixed, 1e-9) / n
+    per_chunk = t_fixed + per_row * w.Lc * w.H
+    return {"value": 1.0 / per_chunk, "unit": "chunks/s", "cores": O.num_threads(),
+            "kind": "oracle",
+            "sample": f"{w.name} chunk {c}: visible-key build + {n} of {w.Lc * w.H} (token, head) "
+                      f"output rows in fp64, extrapolated linearly to the whole chunk "
+                      f"({t_fixed + t_rows:.1f} s of CPU time)"}
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    # each step is a bounded sample (fewer rows) so the whole run stays short
+    per = []
+    for i in range(warm + steps):
+        r = oracle_sample(w, budget_rows=512)
+        if i >= warm:
+            per.append(1.0 / r["value"])
+    ms_step = 1000.0 * w.n_chunks * w.B * statistics.mean(per)
+    value = w.n_chunks * w.B / (ms_step / 1000.0)
+    line = {"metric": METRIC, "value": value, "unit": "chunks/s", "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": config_json(w, world),
+            "cpu_baseline": {"value": value, "unit": "chunks/s", "cores": r["cores"],
+                             "kind": "oracle", "sample": r["sample"].replace("4096", "512")},
+            "e2e": {"value": value, "unit": "chunks/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_json(w, world):
+    return {"workload": w.name, "streams_per_gpu": w.B, "heads": w.H, "head_dim": w.D,
+            "frame": f"{w.fh}x{w.fw}", "chunk_frames": w.C, "sink_frames": w.S,
+            "window_frames": w.W, "chunks_per_stream": w.n_chunks,
+            "refresh_every": w.refresh_period, "rope_dims": list(w.dims),
+            "parallelism": f"independent streams per GPU x{world} (no collective)",
+            "l2": "inputs larger than L2 (every chunk of the step resident, "
+                  f"{3 * w.n_chunks * w.B * w.Lc * w.H * w.D * (2 if w.dtype == 'bf16' else 4) / 1e9:.1f}"
+                  " GB per step)"}
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from inputgen.workloads import BY_NAME
+    w = BY_NAME[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import inputgen as IG
+    from rolling_kv_cache_sa_b200 import SACache, attention_flops, config_for, sa_plan_chunk
+    from rolling_kv_cache_sa_b200.session import StreamSession
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    cfg = config_for(w)
+    cache = SACache(cfg)
+    sess = StreamSession(cache, w.refresh_period)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    n_steps_g = w.n_steps
+    shape = (n_steps_g, w.B, w.Lc, w.H, w.D)
+    q_all = torch.empty(shape, dtype=dt, device="cuda")
+    k_all = torch.empty_like(q_all)
+    v_all = torch.empty_like(q_all)
+    out_all = torch.empty_like(q_all)
+    st = torch.cuda.current_stream().cuda_stream
+    stream_ids = [rank * w.B + b for b in range(w.B)]  # distinct streams per rank
+    actives = []
+    for g in range(n_steps_g):
+        chunks = w.local_chunks(g)
+        actives.append([c >= 0 for c in chunks])
+        for t, buf in ((IG.Q, q_all), (IG.K, k_all), (IG.V, v_all)):
+            IG.fill_device(w, stream_ids, chunks, t, buf[g].data_ptr(), st)
+    torch.cuda.synchronize()
+
+    chunks_per_step = sum(sum(a) for a in actives)
+    # algorithmic attention FLOPs of one step: 4 * Lc * n_keys * D * H per stream-chunk
+    step_flops = 0.0
+    for c in range(w.n_chunks):
+        step_flops += w.B * attention_flops(cfg, sa_plan_chunk(cfg, c * w.C, 0).n_keys)
+    esz = 2 if w.dtype == "bf16" else 4
+    append_bytes_per_chunk = 6 * w.Lc * w.H * w.D * esz  # read q,k,v; write q',k',v
+
+    def run_step():
+        cache.reset()
+        for g in range(n_steps_g):
+            sess.step(q_all[g], k_all[g], v_all[g], out_all[g], actives[g])
+
+    for _ in range(args.warmup):
+        run_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    cache.profile_begin()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        run_step()
+    ev1.record()
+    ev1.synchronize()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    prof = cache.profile_end()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = chunks_per_step * args.steps * world / (ms / 1000.0)
+
+    hbm, pk_burst, pk_sust, pk_src = peaks()
+    att_ms, att_n = prof["attend"]
+    app_ms, app_n = prof["append"]
+    ref_ms, ref_n = prof["refresh"]
+    att_flops_per_launch = step_flops * args.steps / max(att_n, 1)
+    att_avg_s = att_ms / 1000.0 / max(att_n, 1)
+    achieved = att_flops_per_launch / att_avg_s / 1e12
+    app_avg_s = app_ms / 1000.0 / max(app_n, 1)
+    append_gbs = append_bytes_per_chunk * w.B / app_avg_s / 1e9 if app_n else None
+
+    e2e = None
+    if not args.no_e2e:
+        qh = torch.empty(q_all.shape, dtype=dt, pin_memory=True)
+        kh = torch.empty_like(qh, pin_memory=True)
+        vh = torch.empty_like(qh, pin_memory=True)
+        oh = torch.empty_like(qh, pin_memory=True)
+        qh.copy_(q_all)
+        kh.copy_(k_all)
+        vh.copy_(v_all)
+
+        def run_step_host():
+            cache.reset()
+            for g in range(n_steps_g):
+                sess.step_host(qh[g], kh[g], vh[g], oh[g], actives[g])
+
+        run_step_host()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.e2e_steps):
+            run_step_host()
+        e1.record()
+        e1.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        per_chunk_in = 3 * w.Lc * w.H * w.D * esz
+        e2e = {"value": chunks_per_step * args.e2e_steps * world / (ems / 1000.0),
+               "unit": "chunks/s", "steps": args.e2e_steps,
+               "h2d_bytes_per_step": per_chunk_in * chunks_per_step,
+               "d2h_bytes_per_step": w.Lc * w.H * w.D * esz * chunks_per_step,
+               "api": "sa_append_attend_host (pinned host buffers, copies inside the call)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(w)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        cache.close()
+        return
+    att_tflops_step = step_flops / (ms_step / 1000.0) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "chunks/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded counter generator; Irwin-Hall N(0,1) inputs)",
+        "config": config_json(w, world),
+        "ms_per_chunk": ms_step / chunks_per_step,
+        "attention_tflops_whole_step": att_tflops_step,
+        "attention_frac_of_peak_whole_step": att_tflops_step / pk_burst,
+        "append_gbs": append_gbs,
+        "append_frac_of_hbm": (append_gbs / hbm) if append_gbs else None,
+        "kernel_ms_per_step": {"attend": att_ms / args.steps, "append": app_ms / args.steps,
+                               "refresh": ref_ms / args.steps},
+        "roofline": {"bound": "tensor", "kernel": "attend_tc_kernel<128>",
+                     "achieved": achieved, "peak": pk_burst, "unit": "TFLOP/s",
+                     "frac": achieved / pk_burst, "peak_source": f"{pk_src} bf16 burst",
+                     "frac_of_sustained": achieved / pk_sust, "traffic": None},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": att_n + app_n + ref_n,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    cache.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,201 @@
+/*
+ * sa.h -- C ABI of libsa.so: per-chunk block-causal attention over a rolling
+ * (sink + sliding window) KV cache with 3D RoPE, for streaming video
+ * diffusion transformers, on NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute (the pages print no formula; the plain reading):
+ *  - StreamDiffusionV2 (technical summary, section 2.A.2): sink tokens keep
+ *    the stream anchored; RoPE offsets are reset at block boundaries so
+ *    positions stay bounded over unbounded streams -> sa_rope_refresh.
+ *  - SANA-Streaming (section "hybrid diffusion transformer"): softmax blocks
+ *    attend to a sliding local window plus a persistent sink chunk, a bounded
+ *    context with constant memory -> the cache layout of sa_cache_create and
+ *    the attention of sa_append_attend.
+ *  - StreamDiT (abstract): window attention over a moving buffer of frames.
+ *
+ * Per stream b, frames are numbered from 0 and chunk c holds frames
+ * [cC, (c+1)C). sa_append_attend appends the stream's next chunk: it rotates
+ * q and k with 3D RoPE at position (t, y, x), t = frame - pos_base, stores
+ * the rotated k and the raw v in the cache (the first S frames in a pinned
+ * sink, later frames in a ring of R = W + C frames, slot (f - S) mod R, which
+ * evicts the frame written R frames before), and lets every query of the
+ * chunk attend, with softmax scale `softmax_scale`, over
+ *     [ sink | the W frames before the chunk | the whole chunk ]
+ * (the chunk itself bidirectionally). RoPE: the head dim splits into bands
+ * (d_t | d_h | d_w); inside a band of width d, dims (2j, 2j+1) rotate by
+ * pos * base^(-2j/d) as (a, b) -> (a cos - b sin, a sin + b cos).
+ *
+ * Conventions for every call:
+ *  - Device pointers are CUDA device addresses in the current context;
+ *    `stream` is a cudaStream_t passed as void*. Calls enqueue work on that
+ *    stream and return without synchronising, except where noted.
+ *  - Validation happens before any launch: on an error nothing is enqueued
+ *    and no stream state changes. No exception crosses the ABI. The reason of
+ *    the last error of the calling thread is in sa_last_error_string().
+ *  - Inputs are borrowed only until the enqueued work completes. A handle is
+ *    not thread-safe; use it from one host thread and one CUDA stream.
+ *  - Devices other than compute capability 10.x (B200 class) are refused with
+ *    SA_ERR_UNSUPPORTED. There is no CPU fallback.
+ */
+#ifndef SA_H
+#define SA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SA_ABI_VERSION 1
+#define SA_MAX_CHUNK_FRAMES 32 /* C <= 32 */
+#define SA_MAX_SINK_FRAMES 32  /* S <= 32 */
+#define SA_MAX_STREAMS 64      /* B <= 64 */
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,    /* a pointer, size or configuration is invalid */
+  SA_ERR_UNSUPPORTED = 2,    /* no B200-class device, or a shape this build does not run */
+  SA_ERR_OOM = 3,            /* device or pinned-host allocation failed */
+  SA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
+  SA_ERR_STATE = 5,          /* call not valid in the handle's current state */
+  SA_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up on a bounded wait (see sa_get_device_status) */
+} sa_status;
+
+typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
+
+typedef void* sa_stream_t; /* a cudaStream_t */
+
+typedef struct {
+  int32_t batch;          /* B independent streams, 1..SA_MAX_STREAMS */
+  int32_t heads;          /* H */
+  int32_t head_dim;       /* D: 64 or 128 */
+  int32_t frame_h;        /* latent frame rows (fh) */
+  int32_t frame_w;        /* latent frame columns (fw); F = fh * fw tokens per frame */
+  int32_t chunk_frames;   /* C >= 1: frames appended per call */
+  int32_t sink_frames;    /* S >= 0: first frames pinned forever */
+  int32_t window_frames;  /* W >= 0: earlier frames each chunk also sees */
+  int32_t rope_dims[3];   /* (d_t, d_h, d_w): even, sum = D, d_t <= 128 */
+  float rope_base;        /* theta base (> 0), e.g. 10000 */
+  float softmax_scale;    /* 0 means 1/sqrt(D) */
+  int32_t dtype;          /* sa_dtype of q, k, v, out and the cache */
+} sa_config;
+
+typedef struct sa_cache sa_cache; /* opaque */
+
+/* Plan of one stream's next chunk (host-side bookkeeping, exposed for tests). */
+typedef struct {
+  int64_t chunk;        /* local chunk index c = frames_written / C */
+  int64_t sink_len;     /* visible sink key tokens after the append */
+  int64_t ring_len;     /* visible ring key tokens after the append */
+  int64_t n_keys;       /* sink_len + ring_len: keys are cache rows [0, n_keys) */
+  int32_t n_frames;     /* C */
+  int32_t pad_;
+  int64_t dest_row[SA_MAX_CHUNK_FRAMES]; /* cache row of each frame's first token */
+  int64_t t_pos[SA_MAX_CHUNK_FRAMES];    /* temporal RoPE position of each frame */
+  int32_t is_sink[SA_MAX_CHUNK_FRAMES];  /* 1 if the frame lands in the sink */
+} sa_chunk_plan;
+
+/*
+ * Creates a cache for cfg->batch streams on the current device and zeroes it.
+ * Device memory owned by the handle (freed by sa_cache_destroy):
+ *   K' and V cache, [B][H][(S+R)F][D] each (per (b, h): S*F sink rows, then
+ *   R*F ring rows); the raw (unrotated) sink keys, [B][H][S*F][D]; a rotated-
+ *   query workspace, [B][H][C*F][D]; the spatial cos/sin tables (fp64 on the
+ *   host, stored fp32). All streams start empty (frames_written = 0,
+ *   pos_base = 0). The zeroing runs on `stream`.
+ * Errors: SA_ERR_INVALID_ARG (cfg invalid or out == NULL), SA_ERR_UNSUPPORTED
+ * (no compute capability 10.x device), SA_ERR_OOM, SA_ERR_CUDA.
+ */
+sa_status sa_cache_create(const sa_config* cfg, sa_stream_t stream, sa_cache** out);
+
+/*
+ * The hot path: appends the next chunk of every active stream and attends.
+ *   q, k, v : device, [B][C*F][H][D] in cfg dtype, contiguous, 16-byte aligned.
+ *   out     : device, [B][C*F][H][D] in cfg dtype; rows of inactive streams
+ *             are not written.
+ *   active  : host, B bytes (nonzero = active) or NULL for all streams.
+ * Launches the fused RoPE + append kernel, then the attention kernel, on
+ * `stream`; advances frames_written of each active stream by C afterwards.
+ * Never synchronises (capturable in a CUDA graph).
+ */
+sa_status sa_append_attend(sa_cache* h, const void* q, const void* k, const void* v, void* out,
+                           const uint8_t* active, sa_stream_t stream);
+
+/*
+ * RoPE refresh of the active streams (StreamDiffusionV2, section 2.A.2):
+ * before stream b's next chunk c, every cached position is rebased by
+ *   Delta = max(S, cC - W) - pos_base,
+ * so the oldest non-sink frame that chunk c will see sits at t = 0 and all
+ * relative offsets (hence, exactly, all scores) are kept. Ring keys have
+ * their temporal band re-rotated by -Delta in place; sink keys are
+ * re-derived from their raw copy at the new position (one rounding, no drift
+ * over many refreshes). pos_base += Delta. Streams with no frames are skipped.
+ * The caller chooses when to refresh (e.g. when c > 0 and c % period == 0).
+ */
+sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream);
+
+/* Empties the selected streams (NULL = all): frames_written = pos_base = 0.
+ * Host bookkeeping only; cache contents are overwritten by later appends. */
+sa_status sa_cache_reset(sa_cache* h, const uint8_t* streams);
+
+/* Synchronises the stream given at create, frees all memory of the handle. */
+sa_status sa_cache_destroy(sa_cache* h);
+
+/*
+ * Host-buffer variant of sa_append_attend: q, k, v are HOST pointers
+ * ([B][C*F][H][D]); they are copied to device staging buffers owned by the
+ * handle, the chunk is processed, and the result is copied back to the host
+ * pointer `out` before the call returns (the call synchronises `stream`).
+ * Page-locked host memory gives asynchronous copies. The staging buffers are
+ * allocated by the first call on a handle.
+ */
+sa_status sa_append_attend_host(sa_cache* h, const void* q, const void* k, const void* v,
+                                void* out, const uint8_t* active, sa_stream_t stream);
+
+/* ---- introspection (tests, benchmarks) ---- */
+
+/* frames_written and pos_base of stream b (host bookkeeping; no sync). */
+sa_status sa_stream_state(const sa_cache* h, int32_t b, int64_t* frames_written,
+                          int64_t* pos_base);
+
+/* Copies stream b's cache to host: host_k and host_v receive [H][(S+R)F][D]
+ * each in cfg dtype (rows of never-written slots are zero). Synchronous. */
+sa_status sa_cache_copy_out(const sa_cache* h, int32_t b, void* host_k, void* host_v,
+                            sa_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the device error word. Returns
+ * SA_ERR_DEVICE_TIMEOUT if a kernel abandoned a bounded wait since the last
+ * call, else SA_OK. */
+sa_status sa_get_device_status(sa_cache* h, sa_stream_t stream);
+
+/* Plan of the next chunk of a stream in state (frames_written, pos_base);
+ * pure host computation, needs no device. frames_written must be a multiple
+ * of C. */
+sa_status sa_plan_chunk(const sa_config* cfg, int64_t frames_written, int64_t pos_base,
+                        sa_chunk_plan* plan);
+
+/* Refresh offset Delta for a stream in state (frames_written, pos_base);
+ * pure host computation. */
+sa_status sa_refresh_delta(const sa_config* cfg, int64_t frames_written, int64_t pos_base,
+                           int64_t* delta);
+
+/* Kernel timing with CUDA events recorded around each launch on the launch
+ * stream. sa_profile_begin clears the counters and starts recording (up to
+ * 8192 launches); sa_profile_end synchronises and returns the summed device
+ * times in milliseconds and the launch counts, then stops recording. Any
+ * output pointer may be NULL. */
+sa_status sa_profile_begin(sa_cache* h);
+sa_status sa_profile_end(sa_cache* h, double* append_ms, int32_t* n_append, double* attend_ms,
+                         int32_t* n_attend, double* refresh_ms, int32_t* n_refresh);
+
+/* Thread-local text of the last error; never NULL. */
+const char* sa_last_error_string(void);
+
+int32_t sa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H */

@@ -1,0 +1,97 @@
+"""ctypes declarations of libsa.so (include/sa.h). Argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsa.so")
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_OOM, SA_ERR_CUDA, SA_ERR_STATE, \
+    SA_ERR_DEVICE_TIMEOUT = range(7)
+STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_OOM",
+                4: "SA_ERR_CUDA", 5: "SA_ERR_STATE", 6: "SA_ERR_DEVICE_TIMEOUT"}
+SA_F32, SA_BF16 = 0, 1
+SA_MAX_CHUNK_FRAMES = 32
+
+# every symbol include/sa.h declares
+EXPORTED = (
+    "sa_cache_create", "sa_append_attend", "sa_rope_refresh", "sa_cache_reset",
+    "sa_cache_destroy", "sa_append_attend_host", "sa_stream_state", "sa_cache_copy_out",
+    "sa_get_device_status", "sa_plan_chunk", "sa_refresh_delta", "sa_profile_begin",
+    "sa_profile_end", "sa_last_error_string", "sa_abi_version",
+)
+
+
+class sa_config(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("frame_h", ctypes.c_int32), ("frame_w", ctypes.c_int32),
+        ("chunk_frames", ctypes.c_int32), ("sink_frames", ctypes.c_int32),
+        ("window_frames", ctypes.c_int32), ("rope_dims", ctypes.c_int32 * 3),
+        ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class sa_chunk_plan(ctypes.Structure):
+    _fields_ = [
+        ("chunk", ctypes.c_int64), ("sink_len", ctypes.c_int64), ("ring_len", ctypes.c_int64),
+        ("n_keys", ctypes.c_int64), ("n_frames", ctypes.c_int32), ("pad_", ctypes.c_int32),
+        ("dest_row", ctypes.c_int64 * SA_MAX_CHUNK_FRAMES),
+        ("t_pos", ctypes.c_int64 * SA_MAX_CHUNK_FRAMES),
+        ("is_sink", ctypes.c_int32 * SA_MAX_CHUNK_FRAMES),
+    ]
+
+
+class SAError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libsa.so; raises if it is missing (there is no fallback path)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: the CUDA library must be built "
+                           "(__graft_entry__.build()); there is no fallback path")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    P = ctypes.POINTER
+    sig = {
+        "sa_cache_create": [P(sa_config), vp, P(vp)],
+        "sa_append_attend": [vp, vp, vp, vp, vp, vp, vp],
+        "sa_rope_refresh": [vp, vp, vp],
+        "sa_cache_reset": [vp, vp],
+        "sa_cache_destroy": [vp],
+        "sa_append_attend_host": [vp, vp, vp, vp, vp, vp, vp],
+        "sa_stream_state": [vp, i32, P(i64), P(i64)],
+        "sa_cache_copy_out": [vp, i32, vp, vp, vp],
+        "sa_get_device_status": [vp, vp],
+        "sa_plan_chunk": [P(sa_config), i64, i64, P(sa_chunk_plan)],
+        "sa_refresh_delta": [P(sa_config), i64, i64, P(i64)],
+        "sa_profile_begin": [vp],
+        "sa_profile_end": [vp, P(ctypes.c_double), P(i32), P(ctypes.c_double), P(i32),
+                           P(ctypes.c_double), P(i32)],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.sa_last_error_string.argtypes = []
+    L.sa_last_error_string.restype = ctypes.c_char_p
+    L.sa_abi_version.argtypes = []
+    L.sa_abi_version.restype = ctypes.c_int32
+    _LIB = L
+    return L
+
+
+def check(status: int, where: str) -> None:
+    if status != SA_OK:
+        raise SAError(status, where, lib().sa_last_error_string().decode())

@@ -1,0 +1,46 @@
+"""Builds rolling_kv_cache_sa_b200/libsa.so (sm_100a) from csrc/*.cu with nvcc."""
+import glob
+import os
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+LIB = os.path.join(HERE, "libsa.so")
+
+NVCC_FLAGS = ["-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+              "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+              "-Xptxas", "-v", "--expt-relaxed-constexpr"]
+
+
+def sources():
+    return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
+
+
+def deps():
+    return sources() + sorted(glob.glob(os.path.join(HERE, "csrc", "*.h"))) + \
+        sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + \
+        [os.path.join(ROOT, "include", "sa.h")]
+
+
+def is_stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    return any(os.path.getmtime(s) > t for s in deps())
+
+
+def build(verbose: bool = False) -> str:
+    cmd = ["nvcc", *NVCC_FLAGS, *sources(), "-o", LIB, "-lcuda"]
+    if verbose:
+        print(" ".join(cmd))
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    log = os.path.join(HERE, "build.log")
+    with open(log, "w") as f:
+        f.write(r.stdout + r.stderr)
+    if r.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + r.stderr[-6000:])
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(verbose=True))

@@ -1,0 +1,215 @@
+"""Python binding of libsa.so: the C-ABI calls under the same names, plus a
+small handle class. Argument marshalling only -- every step of the path runs
+in the library's CUDA kernels; PyTorch supplies device memory and streams."""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from ._lib import SA_BF16, SA_F32, check, lib, sa_chunk_plan, sa_config
+
+
+def make_config(batch: int, heads: int, head_dim: int, frame_h: int, frame_w: int,
+                chunk_frames: int, sink_frames: int, window_frames: int,
+                rope_dims: Sequence[int], rope_base: float = 10000.0,
+                softmax_scale: float = 0.0, dtype: str = "bf16") -> sa_config:
+    c = sa_config()
+    c.batch, c.heads, c.head_dim = batch, heads, head_dim
+    c.frame_h, c.frame_w = frame_h, frame_w
+    c.chunk_frames, c.sink_frames, c.window_frames = chunk_frames, sink_frames, window_frames
+    for i in range(3):
+        c.rope_dims[i] = int(rope_dims[i])
+    c.rope_base = rope_base
+    c.softmax_scale = softmax_scale
+    c.dtype = SA_BF16 if dtype == "bf16" else SA_F32
+    return c
+
+
+def config_for(w) -> sa_config:
+    """sa_config of a workload description (inputgen.workloads.Workload)."""
+    return make_config(w.B, w.H, w.D, w.fh, w.fw, w.C, w.S, w.W, w.dims, w.rope_base, 0.0, w.dtype)
+
+
+def _mask(active, n: int):
+    if active is None:
+        return None
+    a = (ctypes.c_uint8 * n)(*[1 if x else 0 for x in active])
+    return a
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+# ---- the C-ABI calls, same names -------------------------------------------------
+def sa_cache_create(cfg: sa_config, stream: Optional[torch.cuda.Stream] = None) -> int:
+    h = ctypes.c_void_p()
+    check(lib().sa_cache_create(ctypes.byref(cfg), ctypes.c_void_p(_stream_ptr(stream)),
+                                ctypes.byref(h)), "sa_cache_create")
+    return h.value
+
+
+def sa_append_attend(h: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                     active=None, stream: Optional[torch.cuda.Stream] = None, batch: int = 0):
+    check(lib().sa_append_attend(h, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 _mask(active, batch or q.shape[0]), _stream_ptr(stream)),
+          "sa_append_attend")
+
+
+def sa_rope_refresh(h: int, active=None, batch: int = 0,
+                    stream: Optional[torch.cuda.Stream] = None):
+    check(lib().sa_rope_refresh(h, _mask(active, batch), _stream_ptr(stream)), "sa_rope_refresh")
+
+
+def sa_cache_reset(h: int, streams=None, batch: int = 0):
+    check(lib().sa_cache_reset(h, _mask(streams, batch)), "sa_cache_reset")
+
+
+def sa_cache_destroy(h: int):
+    check(lib().sa_cache_destroy(h), "sa_cache_destroy")
+
+
+def sa_append_attend_host(h: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          out: torch.Tensor, active=None,
+                          stream: Optional[torch.cuda.Stream] = None):
+    for t in (q, k, v, out):
+        assert t.device.type == "cpu" and t.is_contiguous()
+    check(lib().sa_append_attend_host(h, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      _mask(active, q.shape[0]), _stream_ptr(stream)),
+          "sa_append_attend_host")
+
+
+def sa_stream_state(h: int, b: int):
+    fw, base = ctypes.c_int64(), ctypes.c_int64()
+    check(lib().sa_stream_state(h, b, ctypes.byref(fw), ctypes.byref(base)), "sa_stream_state")
+    return fw.value, base.value
+
+
+def sa_cache_copy_out(h: int, b: int, k_host: np.ndarray, v_host: np.ndarray,
+                      stream: Optional[torch.cuda.Stream] = None):
+    check(lib().sa_cache_copy_out(h, b, k_host.ctypes.data, v_host.ctypes.data,
+                                  _stream_ptr(stream)), "sa_cache_copy_out")
+
+
+def sa_get_device_status(h: int, stream: Optional[torch.cuda.Stream] = None) -> int:
+    return lib().sa_get_device_status(h, _stream_ptr(stream))
+
+
+def sa_plan_chunk(cfg: sa_config, frames_written: int, pos_base: int) -> sa_chunk_plan:
+    plan = sa_chunk_plan()
+    check(lib().sa_plan_chunk(ctypes.byref(cfg), frames_written, pos_base, ctypes.byref(plan)),
+          "sa_plan_chunk")
+    return plan
+
+
+def sa_refresh_delta(cfg: sa_config, frames_written: int, pos_base: int) -> int:
+    d = ctypes.c_int64()
+    check(lib().sa_refresh_delta(ctypes.byref(cfg), frames_written, pos_base, ctypes.byref(d)),
+          "sa_refresh_delta")
+    return d.value
+
+
+def sa_profile_begin(h: int):
+    check(lib().sa_profile_begin(h), "sa_profile_begin")
+
+
+def sa_profile_end(h: int):
+    ms = [ctypes.c_double() for _ in range(3)]
+    n = [ctypes.c_int32() for _ in range(3)]
+    check(lib().sa_profile_end(h, ctypes.byref(ms[0]), ctypes.byref(n[0]), ctypes.byref(ms[1]),
+                               ctypes.byref(n[1]), ctypes.byref(ms[2]), ctypes.byref(n[2])),
+          "sa_profile_end")
+    return {"append": (ms[0].value, n[0].value), "attend": (ms[1].value, n[1].value),
+            "refresh": (ms[2].value, n[2].value)}
+
+
+def sa_abi_version() -> int:
+    return lib().sa_abi_version()
+
+
+# ---- handle class -----------------------------------------------------------------
+class SACache:
+    """Owns one libsa cache handle on the current CUDA device."""
+
+    def __init__(self, cfg: sa_config, stream: Optional[torch.cuda.Stream] = None):
+        self.cfg = cfg
+        self.B, self.H, self.D = cfg.batch, cfg.heads, cfg.head_dim
+        self.F = cfg.frame_h * cfg.frame_w
+        self.Lc = cfg.chunk_frames * self.F
+        self.R = cfg.window_frames + cfg.chunk_frames
+        self.ntok = (cfg.sink_frames + self.R) * self.F
+        self.dtype = torch.bfloat16 if cfg.dtype == SA_BF16 else torch.float32
+        self.device = torch.device("cuda", torch.cuda.current_device())
+        self.h = sa_cache_create(cfg, stream)
+
+    def _check_tensor(self, t: torch.Tensor, name: str):
+        if t.device != self.device or t.dtype != self.dtype or not t.is_contiguous() or \
+                tuple(t.shape) != (self.B, self.Lc, self.H, self.D):
+            raise ValueError(f"{name} must be a contiguous {self.dtype} tensor of shape "
+                             f"{(self.B, self.Lc, self.H, self.D)} on {self.device}")
+
+    def append_attend(self, q, k, v, out, active=None, stream=None):
+        for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+            self._check_tensor(t, n)
+        sa_append_attend(self.h, q, k, v, out, active, stream, self.B)
+
+    def append_attend_host(self, q, k, v, out, active=None, stream=None):
+        sa_append_attend_host(self.h, q, k, v, out, active, stream)
+
+    def rope_refresh(self, active=None, stream=None):
+        sa_rope_refresh(self.h, active, self.B, stream)
+
+    def reset(self, streams=None):
+        sa_cache_reset(self.h, streams, self.B)
+
+    def state(self, b: int):
+        return sa_stream_state(self.h, b)
+
+    def copy_out(self, b: int):
+        """(K', V) of stream b as float32 numpy arrays [H, (S+R)F, D]."""
+        shape = (self.H, self.ntok, self.D)
+        if self.cfg.dtype == SA_BF16:
+            kb = np.empty(shape, np.uint16)
+            vb = np.empty(shape, np.uint16)
+            sa_cache_copy_out(self.h, b, kb, vb)
+            f = lambda x: (x.astype(np.uint32) << 16).view(np.float32)  # noqa: E731
+            return f(kb), f(vb)
+        kf = np.empty(shape, np.float32)
+        vf = np.empty(shape, np.float32)
+        sa_cache_copy_out(self.h, b, kf, vf)
+        return kf, vf
+
+    def device_status(self, stream=None) -> int:
+        return sa_get_device_status(self.h, stream)
+
+    def profile_begin(self):
+        sa_profile_begin(self.h)
+
+    def profile_end(self):
+        return sa_profile_end(self.h)
+
+    def close(self):
+        if self.h:
+            sa_cache_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def attention_flops(cfg: sa_config, n_keys: int) -> float:
+    """Algorithmic FLOPs of one (stream, chunk): 4 * Lc * n_keys * D * H (QK^T and PV)."""
+    Lc = cfg.chunk_frames * cfg.frame_h * cfg.frame_w
+    return 4.0 * Lc * n_keys * cfg.head_dim * cfg.heads
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,84 @@
+// internal.h -- launch parameter blocks and kernel entry points of libsa.so.
+// Every parameter block is passed by value (__grid_constant__), so a launch
+// needs no host->device copy and can be captured in a CUDA graph.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sa.h"
+
+namespace sa {
+
+constexpr int kMaxEntries = 32;   // (stream, frame) entries per append launch
+constexpr int kMaxRefresh = 16;   // streams, and (stream, sink frame) entries, per refresh launch
+constexpr int kMaxDt2 = 64;       // d_t / 2 <= 64
+constexpr int kMaxAttnStreams = SA_MAX_STREAMS;
+constexpr int kDeviceErrTimeout = 1;
+
+// Fused 3D-RoPE + append (one launch covers up to kMaxEntries (stream, frame)
+// entries; entry e = a*C + i is frame i of the a-th stream of the launch).
+struct AppendParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* q_ws;        // [B][H][Lc][D]
+  void* k_cache;     // [B][H][ntok][D]
+  void* v_cache;     // [B][H][ntok][D]
+  void* k_raw;       // [B][H][S*F][D]
+  const float2* htab;  // [fh][d_h/2] (cos, sin)
+  const float2* wtab;  // [fw][d_w/2]
+  int32_t H, D, fw, F, C, Lc;
+  int64_t ntok, sf;    // cache rows per (b, h); sink rows per (b, h)
+  int32_t dt2, dh2, dw2;
+  int32_t n_streams;   // streams in this launch
+  int32_t stream_of[kMaxEntries];
+  int64_t dest_row[kMaxEntries];   // cache row of the frame's first token
+  int64_t raw_row[kMaxEntries];    // raw-sink row of the frame, or -1
+  float2 tcs[kMaxEntries][kMaxDt2];  // temporal band (cos, sin) per entry
+};
+
+// RoPE refresh: ring keys' temporal band rotated by -Delta in place; sink keys
+// re-derived from raw keys at their new positions.
+struct RefreshParams {
+  void* k_cache;
+  const void* k_raw;
+  const float2* htab;
+  const float2* wtab;
+  int32_t H, D, fw, F, S;
+  int64_t ntok, sf;
+  int32_t dt2, dh2, dw2;
+  int32_t n_streams;
+  int32_t stream_of[kMaxRefresh];
+  int64_t ring_rows[kMaxRefresh];    // valid ring rows of the stream
+  int64_t sink_rows[kMaxRefresh];    // valid sink rows of the stream
+  float2 dcs[kMaxRefresh][kMaxDt2];  // (cos, sin) of -Delta * theta_j, per stream
+  float2 scs[kMaxRefresh][kMaxDt2];  // (cos, sin) of t * theta_j per sink entry a*S + s
+};
+
+// Attention over the contiguous key prefix [0, n_keys) of each (b, h).
+struct AttnParams {
+  int32_t H, Lc;
+  int64_t ntok;
+  int32_t n_q_tiles;   // ceil(Lc / 128)
+  int32_t n_streams;
+  float scale_log2;    // softmax_scale * log2(e)
+  int32_t pad_;
+  void* out;           // [B][Lc][H][D]
+  const void* q_ws;    // [B][H][Lc][D] (SIMT path)
+  const void* k_cache; // (SIMT path)
+  const void* v_cache; // (SIMT path)
+  int* status;
+  int32_t stream_of[kMaxAttnStreams];
+  int32_t n_keys[kMaxAttnStreams];
+};
+
+cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStream_t st);
+cudaError_t launch_refresh(const RefreshParams& p, int dtype, int num_sms, cudaStream_t st);
+cudaError_t launch_attend_simt_f32(const AttnParams& p, int D, cudaStream_t st);
+cudaError_t launch_attend_tc_bf16(const AttnParams& p, int D, const CUtensorMap* tm_q,
+                                  const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                  cudaStream_t st);
+
+}  // namespace sa

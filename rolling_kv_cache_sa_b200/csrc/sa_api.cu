@@ -1,0 +1,591 @@
+// sa_api.cu -- host side of libsa.so: the C ABI declared in include/sa.h.
+//
+// Host planner (per active stream, per call): local chunk index, cache row of
+// each appended frame (sink slot f, or ring slot S + (f - S) mod R), temporal
+// RoPE position t = f - pos_base with its (cos, sin) values computed in fp64,
+// and the visible key count. Because sink frames fill the first S*F rows and
+// later frames fill the ring from its first slot, the keys a chunk sees are
+// always the contiguous row prefix [0, n_keys) of its (stream, head) cache:
+// while the sink is not full no frame has reached the ring; once it is full,
+// the sink rows are followed by the occupied ring rows. The attention kernel
+// therefore needs one number per stream. Everything is passed by value in
+// launch parameters: no host->device copy, no synchronisation on the hot path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error = "no error";
+
+sa_status fail(sa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+sa_status cuda_fail(cudaError_t e, const char* what) {
+  if (e == cudaErrorMemoryAllocation)
+    return fail(SA_ERR_OOM, "%s: %s", what, cudaGetErrorString(e));
+  return fail(SA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- config
+sa_status validate_config(const sa_config* c) {
+  if (!c) return fail(SA_ERR_INVALID_ARG, "config is NULL");
+  if (c->batch < 1 || c->batch > SA_MAX_STREAMS)
+    return fail(SA_ERR_INVALID_ARG, "batch must be in [1, %d], got %d", SA_MAX_STREAMS, c->batch);
+  if (c->heads < 1) return fail(SA_ERR_INVALID_ARG, "heads must be >= 1");
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return fail(SA_ERR_INVALID_ARG, "head_dim must be 64 or 128, got %d", c->head_dim);
+  if (c->frame_h < 1 || c->frame_w < 1) return fail(SA_ERR_INVALID_ARG, "frame_h, frame_w >= 1");
+  if (c->chunk_frames < 1 || c->chunk_frames > SA_MAX_CHUNK_FRAMES)
+    return fail(SA_ERR_INVALID_ARG, "chunk_frames must be in [1, %d]", SA_MAX_CHUNK_FRAMES);
+  if (c->sink_frames < 0 || c->sink_frames > SA_MAX_SINK_FRAMES)
+    return fail(SA_ERR_INVALID_ARG, "sink_frames must be in [0, %d]", SA_MAX_SINK_FRAMES);
+  if (c->window_frames < 0) return fail(SA_ERR_INVALID_ARG, "window_frames must be >= 0");
+  int sum = 0;
+  for (int i = 0; i < 3; ++i) {
+    if (c->rope_dims[i] < 0 || (c->rope_dims[i] & 1))
+      return fail(SA_ERR_INVALID_ARG, "rope_dims must be even and >= 0");
+    sum += c->rope_dims[i];
+  }
+  if (sum != c->head_dim) return fail(SA_ERR_INVALID_ARG, "rope_dims must sum to head_dim");
+  if (c->rope_dims[0] / 2 > sa::kMaxDt2) return fail(SA_ERR_INVALID_ARG, "d_t must be <= 128");
+  if (!(c->rope_base > 0.f)) return fail(SA_ERR_INVALID_ARG, "rope_base must be > 0");
+  if (c->softmax_scale < 0.f || !isfinite(c->softmax_scale))
+    return fail(SA_ERR_INVALID_ARG, "softmax_scale must be >= 0 (0 = 1/sqrt(D))");
+  if (c->dtype != SA_F32 && c->dtype != SA_BF16)
+    return fail(SA_ERR_INVALID_ARG, "dtype must be SA_F32 or SA_BF16");
+  const int64_t F = (int64_t)c->frame_h * c->frame_w;
+  const int64_t Lc = F * c->chunk_frames;
+  const int64_t ntok = F * ((int64_t)c->sink_frames + c->window_frames + c->chunk_frames);
+  if (Lc * c->heads * (int64_t)c->head_dim * c->batch > ((int64_t)1 << 31) / 2)
+    return fail(SA_ERR_UNSUPPORTED, "B*C*F*H*D too large for one call");
+  if (ntok > ((int64_t)1 << 30)) return fail(SA_ERR_UNSUPPORTED, "cache rows per head too large");
+  if ((int64_t)c->batch * c->heads > ((int64_t)1 << 30))
+    return fail(SA_ERR_UNSUPPORTED, "batch*heads too large");
+  return SA_OK;
+}
+
+double theta(const sa_config* c, int band, int j) {
+  return pow((double)c->rope_base, -2.0 * (double)j / (double)c->rope_dims[band]);
+}
+
+sa_status plan_chunk(const sa_config* c, int64_t fw_, int64_t base, sa_chunk_plan* pl) {
+  const int64_t C = c->chunk_frames, S = c->sink_frames, R = (int64_t)c->window_frames + C;
+  const int64_t F = (int64_t)c->frame_h * c->frame_w;
+  if (fw_ < 0 || fw_ % C != 0)
+    return fail(SA_ERR_STATE, "frames_written (%lld) is not a multiple of the chunk size",
+                (long long)fw_);
+  memset(pl, 0, sizeof(*pl));
+  pl->chunk = fw_ / C;
+  pl->n_frames = (int32_t)C;
+  for (int64_t i = 0; i < C; ++i) {
+    const int64_t f = fw_ + i;
+    pl->is_sink[i] = f < S;
+    pl->dest_row[i] = (f < S ? f : S + (f - S) % R) * F;
+    pl->t_pos[i] = f - base;
+  }
+  const int64_t after = fw_ + C;
+  pl->sink_len = std::min(S, after) * F;
+  pl->ring_len = std::min(std::max<int64_t>(0, after - S), R) * F;
+  pl->n_keys = pl->sink_len + pl->ring_len;
+  return SA_OK;
+}
+
+int64_t refresh_delta(const sa_config* c, int64_t fw_, int64_t base) {
+  const int64_t C = c->chunk_frames;
+  const int64_t next = fw_ / C;
+  const int64_t first = std::max<int64_t>(c->sink_frames, next * C - c->window_frames);
+  return first - base;
+}
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3D bf16 map over [planes][rows][D] with 64 x 128 x 1 boxes, 128-byte swizzle.
+// Rows past `rows` of a plane read as zeros.
+bool make_map(CUtensorMap* m, void* base, int64_t D, int64_t rows, int64_t planes) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
+  cuuint64_t strides[2] = {(cuuint64_t)(D * 2), (cuuint64_t)(rows * D * 2)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+enum { KIND_APPEND = 0, KIND_ATTEND = 1, KIND_REFRESH = 2 };
+
+}  // namespace
+
+struct sa_cache {
+  sa_config cfg;
+  int dev = 0;
+  int num_sms = 148;
+  cudaStream_t create_stream = nullptr;
+  int64_t F = 0, Lc = 0, R = 0, ntok = 0, sf = 0;
+  size_t esz = 2;
+  float scale = 0.f;
+  void* k_cache = nullptr;
+  void* v_cache = nullptr;
+  void* k_raw = nullptr;
+  void* q_ws = nullptr;
+  float2* htab = nullptr;
+  float2* wtab = nullptr;
+  int* d_status = nullptr;
+  std::vector<int64_t> frames_written, pos_base;
+  CUtensorMap tm_q, tm_k, tm_v;
+  // host-buffer staging (allocated by the first sa_append_attend_host)
+  void* stage[4] = {nullptr, nullptr, nullptr, nullptr};
+  // profiling
+  bool profiling = false;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> ev_kind;
+  size_t ev_used = 0;
+};
+
+namespace {
+
+void prof_before(sa_cache* h, cudaStream_t st, int kind) {
+  if (!h->profiling || h->ev_used + 2 > h->ev.size()) return;
+  cudaEventRecord(h->ev[h->ev_used], st);
+  h->ev_kind[h->ev_used / 2] = kind;
+}
+
+void prof_after(sa_cache* h, cudaStream_t st) {
+  if (!h->profiling || h->ev_used + 2 > h->ev.size()) return;
+  cudaEventRecord(h->ev[h->ev_used + 1], st);
+  h->ev_used += 2;
+}
+
+void free_all(sa_cache* h) {
+  void* ptrs[] = {h->k_cache, h->v_cache, h->k_raw, h->q_ws, h->htab, h->wtab, h->d_status,
+                  h->stage[0], h->stage[1], h->stage[2], h->stage[3]};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+}
+
+sa_status active_list(const sa_cache* h, const uint8_t* active, std::vector<int>& out) {
+  out.clear();
+  for (int b = 0; b < h->cfg.batch; ++b)
+    if (!active || active[b]) out.push_back(b);
+  return SA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t sa_abi_version(void) { return SA_ABI_VERSION; }
+
+const char* sa_last_error_string(void) { return g_last_error.c_str(); }
+
+sa_status sa_plan_chunk(const sa_config* cfg, int64_t frames_written, int64_t pos_base,
+                        sa_chunk_plan* plan) {
+  sa_status st = validate_config(cfg);
+  if (st != SA_OK) return st;
+  if (!plan) return fail(SA_ERR_INVALID_ARG, "plan is NULL");
+  return plan_chunk(cfg, frames_written, pos_base, plan);
+}
+
+sa_status sa_refresh_delta(const sa_config* cfg, int64_t frames_written, int64_t pos_base,
+                           int64_t* delta) {
+  sa_status st = validate_config(cfg);
+  if (st != SA_OK) return st;
+  if (!delta) return fail(SA_ERR_INVALID_ARG, "delta is NULL");
+  if (frames_written < 0 || frames_written % cfg->chunk_frames != 0)
+    return fail(SA_ERR_STATE, "frames_written is not a multiple of the chunk size");
+  *delta = refresh_delta(cfg, frames_written, pos_base);
+  return SA_OK;
+}
+
+sa_status sa_cache_create(const sa_config* cfg, sa_stream_t stream, sa_cache** out) {
+  if (!out) return fail(SA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  sa_status st = validate_config(cfg);
+  if (st != SA_OK) return st;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SA_ERR_UNSUPPORTED, "no CUDA device: %s", cudaGetErrorString(e));
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10)
+    return fail(SA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100a (B200)",
+                dev, prop.major, prop.minor);
+
+  sa_cache* h = new sa_cache();
+  h->cfg = *cfg;
+  h->dev = dev;
+  h->num_sms = prop.multiProcessorCount;
+  h->create_stream = static_cast<cudaStream_t>(stream);
+  h->F = (int64_t)cfg->frame_h * cfg->frame_w;
+  h->Lc = h->F * cfg->chunk_frames;
+  h->R = (int64_t)cfg->window_frames + cfg->chunk_frames;
+  h->sf = h->F * cfg->sink_frames;
+  h->ntok = h->sf + h->R * h->F;
+  h->esz = cfg->dtype == SA_BF16 ? 2 : 4;
+  h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : (float)(1.0 / sqrt((double)cfg->head_dim));
+  h->frames_written.assign(cfg->batch, 0);
+  h->pos_base.assign(cfg->batch, 0);
+  const int64_t B = cfg->batch, H = cfg->heads, D = cfg->head_dim;
+  const size_t cache_bytes = (size_t)(B * H * h->ntok * D) * h->esz;
+  const size_t raw_bytes = (size_t)(B * H * std::max<int64_t>(h->sf, 1) * D) * h->esz;
+  const size_t ws_bytes = (size_t)(B * H * h->Lc * D) * h->esz;
+  const int dh2 = cfg->rope_dims[1] / 2, dw2 = cfg->rope_dims[2] / 2;
+  cudaStream_t cs = h->create_stream;
+  struct Alloc { void** p; size_t n; } allocs[] = {
+      {&h->k_cache, cache_bytes}, {&h->v_cache, cache_bytes}, {&h->k_raw, raw_bytes},
+      {&h->q_ws, ws_bytes},
+      {reinterpret_cast<void**>(&h->htab), sizeof(float2) * (size_t)std::max(1, cfg->frame_h * dh2)},
+      {reinterpret_cast<void**>(&h->wtab), sizeof(float2) * (size_t)std::max(1, cfg->frame_w * dw2)},
+      {reinterpret_cast<void**>(&h->d_status), 256}};
+  for (auto& a : allocs) {
+    e = cudaMalloc(a.p, a.n);
+    if (e != cudaSuccess) {
+      free_all(h);
+      delete h;
+      return cuda_fail(e, "cudaMalloc");
+    }
+    e = cudaMemsetAsync(*a.p, 0, a.n, cs);
+    if (e != cudaSuccess) {
+      free_all(h);
+      delete h;
+      return cuda_fail(e, "cudaMemsetAsync");
+    }
+  }
+  // spatial RoPE tables: fp64 on the host, stored fp32
+  std::vector<float2> ht((size_t)std::max(1, cfg->frame_h * dh2)), wt((size_t)std::max(1, cfg->frame_w * dw2));
+  for (int y = 0; y < cfg->frame_h; ++y)
+    for (int j = 0; j < dh2; ++j) {
+      const double ang = (double)y * theta(cfg, 1, j);
+      ht[(size_t)y * dh2 + j] = make_float2((float)cos(ang), (float)sin(ang));
+    }
+  for (int x = 0; x < cfg->frame_w; ++x)
+    for (int j = 0; j < dw2; ++j) {
+      const double ang = (double)x * theta(cfg, 2, j);
+      wt[(size_t)x * dw2 + j] = make_float2((float)cos(ang), (float)sin(ang));
+    }
+  e = cudaMemcpyAsync(h->htab, ht.data(), sizeof(float2) * ht.size(), cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(h->wtab, wt.data(), sizeof(float2) * wt.size(), cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);  // the host tables go out of scope
+  if (e != cudaSuccess) {
+    free_all(h);
+    delete h;
+    return cuda_fail(e, "table upload");
+  }
+  if (cfg->dtype == SA_BF16) {
+    if (!make_map(&h->tm_q, h->q_ws, D, h->Lc, B * H) ||
+        !make_map(&h->tm_k, h->k_cache, D, h->ntok, B * H) ||
+        !make_map(&h->tm_v, h->v_cache, D, h->ntok, B * H)) {
+      free_all(h);
+      delete h;
+      return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    }
+  }
+  *out = h;
+  return SA_OK;
+}
+
+sa_status sa_cache_destroy(sa_cache* h) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  cudaStreamSynchronize(h->create_stream);
+  free_all(h);
+  delete h;
+  return SA_OK;
+}
+
+sa_status sa_cache_reset(sa_cache* h, const uint8_t* streams) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  for (int b = 0; b < h->cfg.batch; ++b)
+    if (!streams || streams[b]) {
+      h->frames_written[b] = 0;
+      h->pos_base[b] = 0;
+    }
+  return SA_OK;
+}
+
+sa_status sa_append_attend(sa_cache* h, const void* q, const void* k, const void* v, void* out,
+                           const uint8_t* active, sa_stream_t stream) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (!q || !k || !v || !out) return fail(SA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SA_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+  const sa_config& c = h->cfg;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<int> act;
+  active_list(h, active, act);
+  if (act.empty()) return SA_OK;
+
+  // plans for every active stream (validated before anything is launched)
+  std::vector<sa_chunk_plan> plans(act.size());
+  for (size_t i = 0; i < act.size(); ++i) {
+    sa_status s = plan_chunk(&c, h->frames_written[act[i]], h->pos_base[act[i]], &plans[i]);
+    if (s != SA_OK) return s;
+  }
+  const int C = c.chunk_frames, dt2 = c.rope_dims[0] / 2;
+  // ---- K1: fused RoPE + append, up to kMaxEntries (stream, frame) entries per launch
+  const int per_launch = std::max(1, sa::kMaxEntries / C);
+  for (size_t s0 = 0; s0 < act.size(); s0 += per_launch) {
+    sa::AppendParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v;
+    p.q_ws = h->q_ws; p.k_cache = h->k_cache; p.v_cache = h->v_cache; p.k_raw = h->k_raw;
+    p.htab = h->htab; p.wtab = h->wtab;
+    p.H = c.heads; p.D = c.head_dim; p.fw = c.frame_w; p.F = (int32_t)h->F; p.C = C;
+    p.Lc = (int32_t)h->Lc; p.ntok = h->ntok; p.sf = h->sf;
+    p.dt2 = dt2; p.dh2 = c.rope_dims[1] / 2; p.dw2 = c.rope_dims[2] / 2;
+    const size_t n = std::min(act.size() - s0, (size_t)per_launch);
+    p.n_streams = (int32_t)n;
+    for (size_t a = 0; a < n; ++a) {
+      const sa_chunk_plan& pl = plans[s0 + a];
+      p.stream_of[a] = act[s0 + a];
+      for (int i = 0; i < C; ++i) {
+        const int e = (int)a * C + i;
+        p.dest_row[e] = pl.dest_row[i];
+        p.raw_row[e] = pl.is_sink[i] ? pl.dest_row[i] : -1;
+        for (int j = 0; j < dt2; ++j) {
+          const double ang = (double)pl.t_pos[i] * theta(&c, 0, j);
+          p.tcs[e][j] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+      }
+    }
+    prof_before(h, st, KIND_APPEND);
+    cudaError_t e = sa::launch_append(p, c.dtype, h->num_sms, st);
+    prof_after(h, st);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  }
+  // ---- K2: attention, streams ordered by decreasing key count
+  std::vector<int> order(act.size());
+  for (size_t i = 0; i < act.size(); ++i) order[i] = (int)i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int x, int y) { return plans[x].n_keys > plans[y].n_keys; });
+  sa::AttnParams ap;
+  memset(&ap, 0, sizeof(ap));
+  ap.H = c.heads; ap.Lc = (int32_t)h->Lc; ap.ntok = h->ntok;
+  ap.n_q_tiles = (int32_t)((h->Lc + 127) / 128);
+  ap.n_streams = (int32_t)act.size();
+  ap.scale_log2 = (float)((double)h->scale * 1.4426950408889634);
+  ap.out = out; ap.q_ws = h->q_ws; ap.k_cache = h->k_cache; ap.v_cache = h->v_cache;
+  ap.status = h->d_status;
+  for (size_t i = 0; i < act.size(); ++i) {
+    ap.stream_of[i] = act[order[i]];
+    ap.n_keys[i] = (int32_t)plans[order[i]].n_keys;
+  }
+  prof_before(h, st, KIND_ATTEND);
+  cudaError_t e = c.dtype == SA_BF16
+                      ? sa::launch_attend_tc_bf16(ap, c.head_dim, &h->tm_q, &h->tm_k, &h->tm_v, st)
+                      : sa::launch_attend_simt_f32(ap, c.head_dim, st);
+  prof_after(h, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  for (int b : act) h->frames_written[b] += C;
+  return SA_OK;
+}
+
+sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  const sa_config& c = h->cfg;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<int> act, todo;
+  active_list(h, active, act);
+  for (int b : act)
+    if (h->frames_written[b] > 0) todo.push_back(b);
+  if (todo.empty()) return SA_OK;
+  const int S = c.sink_frames, dt2 = c.rope_dims[0] / 2;
+  int per_launch = sa::kMaxRefresh;
+  if (S > 0) per_launch = std::max(1, std::min(per_launch, sa::kMaxRefresh / S));
+  if (S > sa::kMaxRefresh)
+    return fail(SA_ERR_UNSUPPORTED, "refresh supports at most %d sink frames", sa::kMaxRefresh);
+  std::vector<int64_t> deltas(todo.size());
+  for (size_t i = 0; i < todo.size(); ++i)
+    deltas[i] = refresh_delta(&c, h->frames_written[todo[i]], h->pos_base[todo[i]]);
+  for (size_t s0 = 0; s0 < todo.size(); s0 += per_launch) {
+    sa::RefreshParams p;
+    memset(&p, 0, sizeof(p));
+    p.k_cache = h->k_cache; p.k_raw = h->k_raw; p.htab = h->htab; p.wtab = h->wtab;
+    p.H = c.heads; p.D = c.head_dim; p.fw = c.frame_w; p.F = (int32_t)h->F; p.S = S;
+    p.ntok = h->ntok; p.sf = h->sf;
+    p.dt2 = dt2; p.dh2 = c.rope_dims[1] / 2; p.dw2 = c.rope_dims[2] / 2;
+    const size_t n = std::min(todo.size() - s0, (size_t)per_launch);
+    p.n_streams = (int32_t)n;
+    for (size_t a = 0; a < n; ++a) {
+      const int b = todo[s0 + a];
+      const int64_t fw_ = h->frames_written[b];
+      const int64_t new_base = h->pos_base[b] + deltas[s0 + a];
+      p.stream_of[a] = b;
+      p.sink_rows[a] = std::min<int64_t>(S, fw_) * h->F;
+      p.ring_rows[a] = std::min<int64_t>(std::max<int64_t>(0, fw_ - S), h->R) * h->F;
+      for (int j = 0; j < dt2; ++j) {
+        const double ang = -(double)deltas[s0 + a] * theta(&c, 0, j);
+        p.dcs[a][j] = make_float2((float)cos(ang), (float)sin(ang));
+      }
+      for (int s = 0; s < S; ++s)
+        for (int j = 0; j < dt2; ++j) {
+          const double ang = (double)(s - new_base) * theta(&c, 0, j);
+          p.scs[a * S + s][j] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+    }
+    prof_before(h, st, KIND_REFRESH);
+    cudaError_t e = sa::launch_refresh(p, c.dtype, h->num_sms, st);
+    prof_after(h, st);
+    if (e != cudaSuccess) return cuda_fail(e, "refresh launch");
+  }
+  for (size_t i = 0; i < todo.size(); ++i) h->pos_base[todo[i]] += deltas[i];
+  return SA_OK;
+}
+
+sa_status sa_append_attend_host(sa_cache* h, const void* q, const void* k, const void* v,
+                                void* out, const uint8_t* active, sa_stream_t stream) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (!q || !k || !v || !out) return fail(SA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t per = (size_t)(h->Lc * h->cfg.heads * h->cfg.head_dim) * h->esz;
+  const size_t total = per * (size_t)h->cfg.batch;
+  for (int i = 0; i < 4; ++i) {
+    if (!h->stage[i]) {
+      cudaError_t e = cudaMalloc(&h->stage[i], total);
+      if (e != cudaSuccess) return cuda_fail(e, "staging cudaMalloc");
+    }
+  }
+  std::vector<int> act;
+  active_list(h, active, act);
+  const void* src[3] = {q, k, v};
+  for (int t = 0; t < 3; ++t)
+    for (int b : act) {
+      cudaError_t e = cudaMemcpyAsync(static_cast<char*>(h->stage[t]) + per * b,
+                                      static_cast<const char*>(src[t]) + per * b, per,
+                                      cudaMemcpyHostToDevice, st);
+      if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    }
+  sa_status s = sa_append_attend(h, h->stage[0], h->stage[1], h->stage[2], h->stage[3], active, stream);
+  if (s != SA_OK) return s;
+  for (int b : act) {
+    cudaError_t e = cudaMemcpyAsync(static_cast<char*>(out) + per * b,
+                                    static_cast<const char*>(h->stage[3]) + per * b, per,
+                                    cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  }
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  return SA_OK;
+}
+
+sa_status sa_stream_state(const sa_cache* h, int32_t b, int64_t* frames_written,
+                          int64_t* pos_base) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (b < 0 || b >= h->cfg.batch) return fail(SA_ERR_INVALID_ARG, "stream index out of range");
+  if (frames_written) *frames_written = h->frames_written[b];
+  if (pos_base) *pos_base = h->pos_base[b];
+  return SA_OK;
+}
+
+sa_status sa_cache_copy_out(const sa_cache* h, int32_t b, void* host_k, void* host_v,
+                            sa_stream_t stream) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (b < 0 || b >= h->cfg.batch) return fail(SA_ERR_INVALID_ARG, "stream index out of range");
+  if (!host_k || !host_v) return fail(SA_ERR_INVALID_ARG, "host buffers must be non-NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = (size_t)(h->cfg.heads * h->ntok * h->cfg.head_dim) * h->esz;
+  cudaError_t e = cudaMemcpyAsync(host_k, static_cast<const char*>(h->k_cache) + n * b, n,
+                                  cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(host_v, static_cast<const char*>(h->v_cache) + n * b, n,
+                        cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cache copy-out");
+  return SA_OK;
+}
+
+sa_status sa_get_device_status(sa_cache* h, sa_stream_t stream) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, h->d_status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->d_status, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "device status read");
+  if (word & sa::kDeviceErrTimeout)
+    return fail(SA_ERR_DEVICE_TIMEOUT, "a kernel abandoned a bounded wait");
+  return SA_OK;
+}
+
+sa_status sa_profile_begin(sa_cache* h) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (h->ev.empty()) {
+    h->ev.resize(2 * 8192);
+    h->ev_kind.resize(8192);
+    for (auto& e : h->ev) {
+      cudaError_t r = cudaEventCreate(&e);
+      if (r != cudaSuccess) return cuda_fail(r, "cudaEventCreate");
+    }
+  }
+  h->ev_used = 0;
+  h->profiling = true;
+  return SA_OK;
+}
+
+sa_status sa_profile_end(sa_cache* h, double* append_ms, int32_t* n_append, double* attend_ms,
+                         int32_t* n_attend, double* refresh_ms, int32_t* n_refresh) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  double ms[3] = {0, 0, 0};
+  int32_t cnt[3] = {0, 0, 0};
+  for (size_t i = 0; i + 1 < h->ev_used + 1 && i < h->ev_used; i += 2) {
+    cudaError_t e = cudaEventSynchronize(h->ev[i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    float t = 0.f;
+    cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]);
+    const int kind = h->ev_kind[i / 2];
+    ms[kind] += t;
+    cnt[kind] += 1;
+  }
+  h->profiling = false;
+  h->ev_used = 0;
+  if (append_ms) *append_ms = ms[KIND_APPEND];
+  if (n_append) *n_append = cnt[KIND_APPEND];
+  if (attend_ms) *attend_ms = ms[KIND_ATTEND];
+  if (n_attend) *n_attend = cnt[KIND_ATTEND];
+  if (refresh_ms) *refresh_ms = ms[KIND_REFRESH];
+  if (n_refresh) *n_refresh = cnt[KIND_REFRESH];
+  return SA_OK;
+}
+
+}  // extern "C"

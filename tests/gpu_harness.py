@@ -1,0 +1,119 @@
+"""Drives a workload through the CUDA path and compares sampled outputs with
+the fp64 oracle. Test infrastructure (imports the oracle)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import inputgen as IG
+import oracle as O
+from inputgen import spec_for
+from rolling_kv_cache_sa_b200 import SACache, config_for
+from rolling_kv_cache_sa_b200.session import StreamSession
+
+BF16_MAX_ABS = 2e-2
+BF16_MEAN_ABS = 2e-3
+F32_MAX_ABS = 1e-4
+
+
+def torch_dtype(w):
+    return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+class Runner:
+    """Holds a cache, a session and device input buffers for one workload."""
+
+    def __init__(self, w):
+        self.w = w
+        self.cache = SACache(config_for(w))
+        self.sess = StreamSession(self.cache, w.refresh_period)
+        shape = (w.B, w.Lc, w.H, w.D)
+        dt = torch_dtype(w)
+        self.q = torch.empty(shape, dtype=dt, device="cuda")
+        self.k = torch.empty_like(self.q)
+        self.v = torch.empty_like(self.q)
+        self.out = torch.zeros_like(self.q)
+
+    def fill(self, chunks):
+        st = torch.cuda.current_stream().cuda_stream
+        for t, buf in ((IG.Q, self.q), (IG.K, self.k), (IG.V, self.v)):
+            IG.fill_device(self.w, list(range(self.w.B)), chunks, t, buf.data_ptr(), st)
+
+    def step(self, g):
+        chunks = self.w.local_chunks(g)
+        active = [c >= 0 for c in chunks]
+        if not any(active):
+            return chunks, active
+        self.fill(chunks)
+        self.sess.step(self.q, self.k, self.v, self.out, active)
+        return chunks, active
+
+    def device_status(self):
+        return self.cache.device_status()
+
+    def close(self):
+        self.cache.close()
+
+
+def sample_tokens(w, n_random=12, seed=0):
+    Lc = w.Lc
+    fixed = {0, 1, 31, 32, 127, 128, 129, Lc // 2, Lc - 129, Lc - 128, Lc - 2, Lc - 1,
+             w.F - 1, w.F, min(Lc - 1, w.F + w.fw)}
+    rng = np.random.default_rng(seed)
+    rand = set(rng.integers(0, Lc, n_random).tolist())
+    return sorted(t for t in fixed | rand if 0 <= t < Lc)
+
+
+def compare_rows(w, b, c, out_b, toks, heads=None, store=None):
+    """Max and mean abs error of GPU rows vs the storage-faithful oracle."""
+    heads = list(range(w.H)) if heads is None else heads
+    tt = np.repeat(np.asarray(toks), len(heads))
+    hh = np.tile(np.asarray(heads), len(toks))
+    cfg = O.cfg_for(w, store=store)
+    ref = O.attend_rows(cfg, spec_for(w), b, c, tt, hh)
+    got = out_b[torch.as_tensor(tt), torch.as_tensor(hh)].double().numpy()
+    err = np.abs(got - ref)
+    return float(err.max()), float(err.mean()), ref, got
+
+
+def assert_rows(w, b, c, out_b, toks, heads=None):
+    mx, mean, ref, got = compare_rows(w, b, c, out_b, toks, heads)
+    if w.dtype == "bf16":
+        assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, (b, c, mx, mean)
+    else:
+        assert mx <= F32_MAX_ABS, (b, c, mx, mean)
+    assert np.isfinite(got).all()
+    return mx, mean
+
+
+def bf16_ulp(x):
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, 2.0 ** (e - 7), 2.0 ** -133)
+
+
+def assert_cache(w, runner, b, c):
+    """GPU cache of stream b after chunk c vs the oracle's storage model:
+    V bit-exact, K' within one storage ulp, metadata exact."""
+    cfg = O.cfg_for(w)
+    k_ref, v_ref, slot_frame = O.cache_contents(cfg, spec_for(w), b, c)
+    k_got, v_got = runner.cache.copy_out(b)
+    fw, base = runner.cache.state(b)
+    assert fw == (c + 1) * w.C
+    assert base == O.base_at(cfg, c)
+    rows = np.concatenate([np.arange(s * w.F, (s + 1) * w.F) for s, f in enumerate(slot_frame)
+                           if f >= 0]).astype(np.int64)
+    np.testing.assert_array_equal(v_got[:, rows], v_ref[:, rows])
+    kr = k_ref[:, rows]
+    kd = np.abs(k_got[:, rows].astype(np.float64) - kr)
+    # the GPU rotates in fp32 (rounding error ~2^-22 of the row's scale, which
+    # can exceed a storage ulp of a small element), then rounds to storage;
+    # a key re-rotated by a refresh goes through that twice
+    rowmax = np.abs(kr).max(axis=-1, keepdims=True)
+    if w.dtype == "bf16":
+        tol = 2.0 * bf16_ulp(kr) + rowmax * 2.0 ** -21
+    else:
+        tol = np.abs(kr) * 2.0 ** -22 + rowmax * 2.0 ** -21 + 1e-9
+    bad = kd > tol
+    assert not bad.any(), (b, c, int(bad.sum()), float(kd.max()))
+    return float(kd.max())

@@ -1,0 +1,107 @@
+"""The C ABI on the host (no GPU needed): exports, validation, host planner.
+
+The planner's slot map, visible-key count, positions and refresh offset are
+compared bit for bit with the oracle's independent closed forms."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import oracle as O
+import rolling_kv_cache_sa_b200 as S
+from rolling_kv_cache_sa_b200 import _lib
+from inputgen.workloads import ALL, Workload
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "sa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib.lib()
+    declared = _declared_symbols()
+    assert len(declared) >= 15
+    for name in declared:
+        assert hasattr(L, name), name
+    assert sorted(_lib.EXPORTED) == declared
+    assert S.sa_abi_version() == 1
+
+
+def test_invalid_configs_are_rejected():
+    base = S.config_for(ALL[1])
+    bad = []
+    for field, val in [("batch", 0), ("batch", 65), ("heads", 0), ("head_dim", 96),
+                       ("frame_h", 0), ("chunk_frames", 0), ("chunk_frames", 33),
+                       ("sink_frames", -1), ("window_frames", -1), ("rope_base", 0.0),
+                       ("softmax_scale", -1.0), ("dtype", 7)]:
+        c = S.config_for(ALL[1])
+        setattr(c, field, val)
+        bad.append(c)
+    c = S.config_for(ALL[1]); c.rope_dims[0] = 43; c.rope_dims[1] = 43; bad.append(c)  # odd
+    c = S.config_for(ALL[1]); c.rope_dims[0] = 40; bad.append(c)  # sum != D
+    for c in bad:
+        with pytest.raises(S.SAError) as e:
+            S.sa_plan_chunk(c, 0, 0)
+        assert e.value.status == _lib.SA_ERR_INVALID_ARG
+        h = ctypes.c_void_p()
+        assert _lib.lib().sa_cache_create(ctypes.byref(c), None, ctypes.byref(h)) == \
+            _lib.SA_ERR_INVALID_ARG
+        assert h.value is None
+    S.sa_plan_chunk(base, 0, 0)
+
+
+def test_state_errors():
+    c = S.config_for(ALL[1])  # C = 2
+    with pytest.raises(S.SAError) as e:
+        S.sa_plan_chunk(c, 3, 0)
+    assert e.value.status == _lib.SA_ERR_STATE
+    with pytest.raises(S.SAError):
+        S.sa_refresh_delta(c, 5, 0)
+    assert _lib.lib().sa_append_attend(None, None, None, None, None, None, None) == \
+        _lib.SA_ERR_INVALID_ARG
+    assert b"NULL" in _lib.lib().sa_last_error_string()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device refusal")
+def test_create_without_device_is_refused():
+    h = ctypes.c_void_p()
+    c = S.config_for(ALL[1])
+    assert _lib.lib().sa_cache_create(ctypes.byref(c), None, ctypes.byref(h)) == \
+        _lib.SA_ERR_UNSUPPORTED
+    assert h.value is None
+
+
+@pytest.mark.parametrize("C,Sn,W", [(1, 1, 2), (2, 1, 4), (1, 1, 6), (1, 1, 3), (2, 1, 8),
+                                    (2, 0, 0), (3, 2, 3), (1, 3, 2), (2, 2, 2)])
+def test_planner_matches_oracle(C, Sn, W):
+    w = Workload("p", B=1, H=2, D=64, fh=3, fw=5, C=C, S=Sn, W=W, n_chunks=1, dtype="bf16",
+                 refresh_period=7)
+    cfg = S.config_for(w)
+    ocfg = O.cfg_for(w)
+    base = 0
+    for c in range(0, 120):
+        if c > 0 and c % 7 == 0:
+            d = S.sa_refresh_delta(cfg, c * C, base)
+            assert d == O.refresh_delta(ocfg, c, base)
+            base += d
+        assert base == O.base_at(ocfg, c)
+        pl = S.sa_plan_chunk(cfg, c * C, base)
+        assert pl.chunk == c and pl.n_frames == C
+        assert pl.n_keys == O.n_keys(ocfg, c)
+        assert pl.sink_len + pl.ring_len == pl.n_keys
+        for i in range(C):
+            f = c * C + i
+            assert pl.dest_row[i] == O.frame_slot(ocfg, f) * w.F
+            assert pl.t_pos[i] == f - base
+            assert pl.is_sink[i] == (f < Sn)
+        # keys are the row prefix [0, n_keys): the occupied slots are exactly
+        # the first n_keys / F slots after this chunk's append
+        sf = O.slot_frames(ocfg, c)
+        occupied = [s for s, f in enumerate(sf) if f >= 0]
+        assert occupied == list(range(pl.n_keys // w.F))
