@@ -36,13 +36,15 @@ METRIC = "streamed chunks/s and attention TFLOP/s (% of B200 BF16 peak) per conf
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="512p_32x32_h24")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--chunks", type=int, default=0,
+                    help="stream only this many chunks per stream (small profiling cases)")
     return ap.parse_args()
 
 
@@ -190,6 +192,8 @@ def main():
 
     from inputgen.workloads import BY_NAME
     w = BY_NAME[args.workload]
+    if args.chunks:
+        w = w.with_(n_chunks=args.chunks)
 
     if args.impl == "reference":
         run_reference(args, w, rank, world)
