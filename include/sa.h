@@ -189,6 +189,40 @@ sa_status sa_profile_begin(sa_cache* h);
 sa_status sa_profile_end(sa_cache* h, double* append_ms, int32_t* n_append, double* attend_ms,
                          int32_t* n_attend, double* refresh_ms, int32_t* n_refresh);
 
+/*
+ * Allocation-free form of sa_append_attend. The pages have no counterpart:
+ * this entry exists for callers that must not call the CUDA allocator at all
+ * -- engines and plugin hosts that own every byte of device memory through
+ * their own pool and do not let a library allocate, and real-time frame
+ * loops that cannot afford cudaMalloc/cudaFree, which may synchronise the
+ * whole device and stall the loop past its per-frame deadline. Such callers
+ * cannot create a cache handle (sa_cache_create allocates); here they pass
+ * the cache memory themselves.
+ *   cfg            : as for sa_cache_create.
+ *   k_cache, v_cache, k_raw : caller-owned device buffers with the layouts
+ *                    sa_cache_create documents ([B][H][(S+R)F][D] and
+ *                    [B][H][S*F][D]); zero them before a stream's first
+ *                    chunk. k_raw may be NULL when S = 0.
+ *   frames_written : host array [B], read and advanced by C per active stream.
+ *   pos_base       : host array [B], the streams' RoPE position bases (read).
+ *   q, k, v, out, active, stream : as for sa_append_attend.
+ * Scratch: a file-scope static device array of 16 MiB (rotated queries
+ * B*H*C*F*D elements, the spatial RoPE tables and a status word), present on
+ * every GPU that loads the library until the process exits. Configurations
+ * that need more return SA_ERR_UNSUPPORTED with the sizes in the error text.
+ * The first call on a device looks up the scratch address on that device;
+ * make that first call before any stream capture. Every call shares the one
+ * scratch array, which keeps the last call's contents: calls whose work
+ * overlaps on the GPU (other streams, other host threads) race and must be
+ * serialised by the caller. Enqueues work on `stream` and never synchronises;
+ * calls no allocator. A bounded-wait expiry is recorded in the scratch status
+ * word only (not reported).
+ */
+sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cache, void* v_cache,
+                                   void* k_raw, int64_t* frames_written, const int64_t* pos_base,
+                                   const void* q, const void* k, const void* v, void* out,
+                                   const uint8_t* active, sa_stream_t stream);
+
 /* Thread-local text of the last error; never NULL. */
 const char* sa_last_error_string(void);
 

@@ -128,6 +128,20 @@ def sa_profile_end(h: int):
             "refresh": (ms[2].value, n[2].value)}
 
 
+def sa_append_attend_noalloc(cfg: sa_config, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                             k_raw: Optional[torch.Tensor], frames_written, pos_base,
+                             q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                             active=None, stream: Optional[torch.cuda.Stream] = None):
+    """Allocation-free append + attention over caller-owned cache buffers.
+    frames_written / pos_base: ctypes int64 arrays of length B (host);
+    frames_written is advanced in place."""
+    check(lib().sa_append_attend_noalloc(
+        ctypes.byref(cfg), k_cache.data_ptr(), v_cache.data_ptr(),
+        k_raw.data_ptr() if k_raw is not None else None, frames_written, pos_base,
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _mask(active, cfg.batch),
+        _stream_ptr(stream)), "sa_append_attend_noalloc")
+
+
 def sa_abi_version() -> int:
     return lib().sa_abi_version()
 

@@ -589,3 +589,195 @@ sa_status sa_profile_end(sa_cache* h, double* append_ms, int32_t* n_append, doub
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of sa_append_attend.
+//
+// For callers that may not call the CUDA allocator at all: engines and plugin
+// hosts that own every byte of device memory through their own pool, and
+// real-time frame loops that cannot afford cudaMalloc/cudaFree (they may
+// synchronise the whole device). The caller passes the cache buffers and the
+// stream state; the one scratch buffer the path needs (the rotated-query
+// workspace, the spatial RoPE tables and a device status word) lives in the
+// static array below, 16 MiB, which every GPU that loads this library holds
+// until the process exits. The first call on a device looks its address up
+// (cudaGetSymbolAddress with that device current), so that first call should
+// come before any stream capture. All calls share the array and it keeps the
+// last call's contents: the status word is cleared by each call, and calls
+// whose work overlaps on the GPU race.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+#define SA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+static __device__ __align__(256) unsigned char g_sa_noalloc_scratch[SA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Device address of the static scratch on the current device. Looked up once
+// per device (with that device current) and remembered.
+sa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoallocMaxDevices)
+    return fail(SA_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kNoallocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_sa_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SA_OK;
+}
+
+// Spatial RoPE tables, (cos, sin) of y * base^(-2j/d_h) and x * base^(-2j/d_w),
+// evaluated in fp64 and stored as fp32.
+__global__ void noalloc_tables_kernel(float2* htab, float2* wtab, int fh, int fw, int dh2,
+                                      int dw2, int dh, int dw, double base) {
+  const int nh = fh * dh2, nw = fw * dw2;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nh + nw; i += gridDim.x * blockDim.x) {
+    if (i < nh) {
+      const int y = i / dh2, j = i % dh2;
+      const double ang = (double)y * pow(base, -2.0 * (double)j / (double)dh);
+      htab[i] = make_float2((float)cos(ang), (float)sin(ang));
+    } else {
+      const int k = i - nh, x = k / dw2, j = k % dw2;
+      const double ang = (double)x * pow(base, -2.0 * (double)j / (double)dw);
+      wtab[k] = make_float2((float)cos(ang), (float)sin(ang));
+    }
+  }
+}
+
+}  // namespace
+
+extern "C" sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cache, void* v_cache,
+                                              void* k_raw, int64_t* frames_written,
+                                              const int64_t* pos_base, const void* q,
+                                              const void* k, const void* v, void* out,
+                                              const uint8_t* active, sa_stream_t stream) {
+  sa_status st = validate_config(cfg);
+  if (st != SA_OK) return st;
+  if (!k_cache || !v_cache || !frames_written || !pos_base || !q || !k || !v || !out)
+    return fail(SA_ERR_INVALID_ARG, "cache buffers, stream state, q, k, v and out must be non-NULL");
+  if (cfg->sink_frames > 0 && !k_raw)
+    return fail(SA_ERR_INVALID_ARG, "k_raw must be non-NULL when sink_frames > 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || (k_raw && !aligned16(k_raw)))
+    return fail(SA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  const sa_config& c = *cfg;
+  const int64_t B = c.batch, H = c.heads, D = c.head_dim;
+  const int64_t F = (int64_t)c.frame_h * c.frame_w, Lc = F * c.chunk_frames;
+  const int64_t R = (int64_t)c.window_frames + c.chunk_frames, sf = F * c.sink_frames;
+  const int64_t ntok = sf + R * F;
+  const size_t esz = c.dtype == SA_BF16 ? 2 : 4;
+  const int dt2 = c.rope_dims[0] / 2, dh2 = c.rope_dims[1] / 2, dw2 = c.rope_dims[2] / 2;
+  // scratch layout: [0,256) status word | tables | (1024-aligned) Q' workspace
+  const size_t tab_bytes = sizeof(float2) * (size_t)(c.frame_h * dh2 + c.frame_w * dw2);
+  const size_t q_off = (256 + tab_bytes + 1023) & ~(size_t)1023;
+  const size_t q_bytes = (size_t)(B * H * Lc * D) * esz;
+  if (q_off + q_bytes > SA_NOALLOC_SCRATCH_BYTES)
+    return fail(SA_ERR_UNSUPPORTED,
+                "sa_append_attend_noalloc: needs %zu bytes of scratch (rotated queries "
+                "B*H*C*F*D plus RoPE tables) but the static scratch holds %u bytes",
+                q_off + q_bytes, (unsigned)SA_NOALLOC_SCRATCH_BYTES);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SA_ERR_UNSUPPORTED, "no CUDA device: %s", cudaGetErrorString(e));
+  int major = 0, nsm = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (major != 10)
+    return fail(SA_ERR_UNSUPPORTED, "device %d is not compute capability 10.x (B200)", dev);
+  std::vector<int> act;
+  for (int b = 0; b < c.batch; ++b)
+    if (!active || active[b]) act.push_back(b);
+  if (act.empty()) return SA_OK;
+  std::vector<sa_chunk_plan> plans(act.size());
+  for (size_t i = 0; i < act.size(); ++i) {
+    st = plan_chunk(&c, frames_written[act[i]], pos_base[act[i]], &plans[i]);
+    if (st != SA_OK) return st;
+  }
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != SA_OK) return st;
+  char* sbase = static_cast<char*>(scratch);
+  int* d_status = reinterpret_cast<int*>(sbase);
+  float2* htab = reinterpret_cast<float2*>(sbase + 256);
+  float2* wtab = htab + c.frame_h * dh2;
+  void* q_ws = sbase + q_off;
+  CUtensorMap tm_q, tm_k, tm_v;
+  if (c.dtype == SA_BF16) {
+    if (!make_map(&tm_q, q_ws, D, Lc, B * H) || !make_map(&tm_k, k_cache, D, ntok, B * H) ||
+        !make_map(&tm_v, v_cache, D, ntok, B * H))
+      return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // every call shares the scratch: the status word must start at zero
+  e = cudaMemsetAsync(d_status, 0, sizeof(int), s);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  if (c.frame_h * dh2 + c.frame_w * dw2 > 0) {
+    noalloc_tables_kernel<<<std::max(1, nsm), 256, 0, s>>>(
+        htab, wtab, c.frame_h, c.frame_w, dh2, dw2, c.rope_dims[1], c.rope_dims[2],
+        (double)c.rope_base);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "RoPE table launch");
+  }
+  const int C = c.chunk_frames;
+  const int per_launch = std::max(1, sa::kMaxEntries / C);
+  for (size_t s0 = 0; s0 < act.size(); s0 += per_launch) {
+    sa::AppendParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v;
+    p.q_ws = q_ws; p.k_cache = k_cache; p.v_cache = v_cache; p.k_raw = k_raw;
+    p.htab = htab; p.wtab = wtab;
+    p.H = c.heads; p.D = c.head_dim; p.fw = c.frame_w; p.F = (int32_t)F; p.C = C;
+    p.Lc = (int32_t)Lc; p.ntok = ntok; p.sf = sf;
+    p.dt2 = dt2; p.dh2 = dh2; p.dw2 = dw2;
+    const size_t n = std::min(act.size() - s0, (size_t)per_launch);
+    p.n_streams = (int32_t)n;
+    for (size_t a = 0; a < n; ++a) {
+      const sa_chunk_plan& pl = plans[s0 + a];
+      p.stream_of[a] = act[s0 + a];
+      for (int i = 0; i < C; ++i) {
+        const int en = (int)a * C + i;
+        p.dest_row[en] = pl.dest_row[i];
+        p.raw_row[en] = pl.is_sink[i] ? pl.dest_row[i] : -1;
+        for (int j = 0; j < dt2; ++j) {
+          const double ang = (double)pl.t_pos[i] * theta(&c, 0, j);
+          p.tcs[en][j] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+      }
+    }
+    e = sa::launch_append(p, c.dtype, nsm, s);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  }
+  std::vector<int> order(act.size());
+  for (size_t i = 0; i < act.size(); ++i) order[i] = (int)i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int x, int y) { return plans[x].n_keys > plans[y].n_keys; });
+  sa::AttnParams ap;
+  memset(&ap, 0, sizeof(ap));
+  ap.H = c.heads; ap.Lc = (int32_t)Lc; ap.ntok = ntok;
+  ap.n_q_tiles = (int32_t)((Lc + 127) / 128);
+  ap.n_streams = (int32_t)act.size();
+  const double scale = c.softmax_scale > 0.f ? (double)c.softmax_scale : 1.0 / sqrt((double)D);
+  ap.scale_log2 = (float)((double)(float)scale * 1.4426950408889634);
+  ap.out = out; ap.q_ws = q_ws; ap.k_cache = k_cache; ap.v_cache = v_cache;
+  ap.status = d_status;
+  for (size_t i = 0; i < act.size(); ++i) {
+    ap.stream_of[i] = act[order[i]];
+    ap.n_keys[i] = (int32_t)plans[order[i]].n_keys;
+  }
+  e = c.dtype == SA_BF16 ? sa::launch_attend_tc_bf16(ap, c.head_dim, &tm_q, &tm_k, &tm_v, s)
+                         : sa::launch_attend_simt_f32(ap, c.head_dim, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  for (int b : act) frames_written[b] += C;
+  return SA_OK;
+}
