@@ -281,6 +281,7 @@ def main():
     ev1.synchronize()
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1)
+    launches = cache.profile_launches()
     prof = cache.profile_end()
     clocks = sampler.stop() if sampler else None
     if world > 1:
@@ -370,7 +371,7 @@ def main():
                                      "(7168 keys); algorithmic minimum 113 MB"},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": att_n + app_n + ref_n,
+        "gpu_launches": launches,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -223,6 +223,9 @@ sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cache, void* v_
                                    const void* q, const void* k, const void* v, void* out,
                                    const uint8_t* active, sa_stream_t stream);
 
+/* Number of kernels the handle launched since sa_profile_begin (host count). */
+sa_status sa_profile_launches(const sa_cache* h, int64_t* launches);
+
 /* Thread-local text of the last error; never NULL. */
 const char* sa_last_error_string(void);
 

@@ -20,6 +20,7 @@ EXPORTED = (
     "sa_cache_destroy", "sa_append_attend_host", "sa_stream_state", "sa_cache_copy_out",
     "sa_get_device_status", "sa_plan_chunk", "sa_refresh_delta", "sa_profile_begin",
     "sa_profile_end", "sa_last_error_string", "sa_abi_version", "sa_append_attend_noalloc",
+    "sa_profile_launches",
 )
 
 
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
         "sa_plan_chunk": [P(sa_config), i64, i64, P(sa_chunk_plan)],
         "sa_refresh_delta": [P(sa_config), i64, i64, P(i64)],
         "sa_profile_begin": [vp],
+        "sa_profile_launches": [vp, P(i64)],
         "sa_append_attend_noalloc": [P(sa_config), vp, vp, vp, P(i64), P(i64), vp, vp, vp, vp,
                                      vp, vp],
         "sa_profile_end": [vp, P(ctypes.c_double), P(i32), P(ctypes.c_double), P(i32),

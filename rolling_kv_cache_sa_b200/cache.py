@@ -128,6 +128,12 @@ def sa_profile_end(h: int):
             "refresh": (ms[2].value, n[2].value)}
 
 
+def sa_profile_launches(h: int) -> int:
+    n = ctypes.c_int64()
+    check(lib().sa_profile_launches(h, ctypes.byref(n)), "sa_profile_launches")
+    return n.value
+
+
 def sa_append_attend_noalloc(cfg: sa_config, k_cache: torch.Tensor, v_cache: torch.Tensor,
                              k_raw: Optional[torch.Tensor], frames_written, pos_base,
                              q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
@@ -206,6 +212,9 @@ class SACache:
 
     def profile_end(self):
         return sa_profile_end(self.h)
+
+    def profile_launches(self) -> int:
+        return sa_profile_launches(self.h)
 
     def close(self):
         if self.h:

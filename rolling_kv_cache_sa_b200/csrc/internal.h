@@ -74,11 +74,20 @@ struct AttnParams {
   int32_t n_keys[kMaxAttnStreams];
 };
 
+// Workspace the bf16 attention may use for split work units: per slot (two
+// per CTA) the unnormalised fp32 O of two 128-row tiles and their (m, l).
+size_t attend_partials_bytes(int D, int num_sms);
+
 cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_refresh(const RefreshParams& p, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_attend_simt_f32(const AttnParams& p, int D, cudaStream_t st);
+// bf16 tensor-core attention. `partials` (attend_partials_bytes) lets the
+// persistent kernel split work units at equal-work boundaries (a combine
+// kernel then merges the pieces); with partials == nullptr every CTA takes
+// whole units. *n_kernels (if non-null) receives the kernels launched.
 cudaError_t launch_attend_tc_bf16(const AttnParams& p, int D, const CUtensorMap* tm_q,
                                   const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                  cudaStream_t st);
+                                  void* partials, size_t partials_bytes, int num_sms,
+                                  cudaStream_t st, int* n_kernels);
 
 }  // namespace sa

@@ -167,6 +167,8 @@ struct sa_cache {
   float2* htab = nullptr;
   float2* wtab = nullptr;
   int* d_status = nullptr;
+  void* partials = nullptr;  // split-unit workspace of the bf16 attention
+  size_t partials_bytes = 0;
   std::vector<int64_t> frames_written, pos_base;
   CUtensorMap tm_q, tm_k, tm_v;
   // host-buffer staging (allocated by the first sa_append_attend_host)
@@ -176,6 +178,7 @@ struct sa_cache {
   std::vector<cudaEvent_t> ev;
   std::vector<int> ev_kind;
   size_t ev_used = 0;
+  int64_t kernels = 0;  // kernel launches since sa_profile_begin
 };
 
 namespace {
@@ -194,7 +197,7 @@ void prof_after(sa_cache* h, cudaStream_t st) {
 
 void free_all(sa_cache* h) {
   void* ptrs[] = {h->k_cache, h->v_cache, h->k_raw, h->q_ws, h->htab, h->wtab, h->d_status,
-                  h->stage[0], h->stage[1], h->stage[2], h->stage[3]};
+                  h->partials, h->stage[0], h->stage[1], h->stage[2], h->stage[3]};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
@@ -313,6 +316,14 @@ sa_status sa_cache_create(const sa_config* cfg, sa_stream_t stream, sa_cache** o
     return cuda_fail(e, "table upload");
   }
   if (cfg->dtype == SA_BF16) {
+    h->partials_bytes = sa::attend_partials_bytes((int)D, h->num_sms);
+    e = cudaMalloc(&h->partials, h->partials_bytes);
+    if (e != cudaSuccess) {
+      h->partials = nullptr;
+      free_all(h);
+      delete h;
+      return cuda_fail(e, "cudaMalloc(partials)");
+    }
     if (!make_map(&h->tm_q, h->q_ws, D, h->Lc, B * H) ||
         !make_map(&h->tm_k, h->k_cache, D, h->ntok, B * H) ||
         !make_map(&h->tm_v, h->v_cache, D, h->ntok, B * H)) {
@@ -392,6 +403,7 @@ sa_status sa_append_attend(sa_cache* h, const void* q, const void* k, const void
     cudaError_t e = sa::launch_append(p, c.dtype, h->num_sms, st);
     prof_after(h, st);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    h->kernels += 1;
   }
   // ---- K2: attention, streams ordered by decreasing key count
   std::vector<int> order(act.size());
@@ -411,11 +423,15 @@ sa_status sa_append_attend(sa_cache* h, const void* q, const void* k, const void
     ap.n_keys[i] = (int32_t)plans[order[i]].n_keys;
   }
   prof_before(h, st, KIND_ATTEND);
+  int n_att = 1;
   cudaError_t e = c.dtype == SA_BF16
-                      ? sa::launch_attend_tc_bf16(ap, c.head_dim, &h->tm_q, &h->tm_k, &h->tm_v, st)
+                      ? sa::launch_attend_tc_bf16(ap, c.head_dim, &h->tm_q, &h->tm_k, &h->tm_v,
+                                                  h->partials, h->partials_bytes, h->num_sms, st,
+                                                  &n_att)
                       : sa::launch_attend_simt_f32(ap, c.head_dim, st);
   prof_after(h, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  h->kernels += n_att;
   for (int b : act) h->frames_written[b] += C;
   return SA_OK;
 }
@@ -467,6 +483,7 @@ sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream
     cudaError_t e = sa::launch_refresh(p, c.dtype, h->num_sms, st);
     prof_after(h, st);
     if (e != cudaSuccess) return cuda_fail(e, "refresh launch");
+    h->kernels += 1;
   }
   for (size_t i = 0; i < todo.size(); ++i) h->pos_base[todo[i]] += deltas[i];
   return SA_OK;
@@ -559,7 +576,14 @@ sa_status sa_profile_begin(sa_cache* h) {
     }
   }
   h->ev_used = 0;
+  h->kernels = 0;
   h->profiling = true;
+  return SA_OK;
+}
+
+sa_status sa_profile_launches(const sa_cache* h, int64_t* launches) {
+  if (!h || !launches) return fail(SA_ERR_INVALID_ARG, "handle and launches must be non-NULL");
+  *launches = h->kernels;
   return SA_OK;
 }
 
@@ -775,7 +799,8 @@ extern "C" sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cach
     ap.stream_of[i] = act[order[i]];
     ap.n_keys[i] = (int32_t)plans[order[i]].n_keys;
   }
-  e = c.dtype == SA_BF16 ? sa::launch_attend_tc_bf16(ap, c.head_dim, &tm_q, &tm_k, &tm_v, s)
+  e = c.dtype == SA_BF16 ? sa::launch_attend_tc_bf16(ap, c.head_dim, &tm_q, &tm_k, &tm_v, nullptr,
+                                                     0, nsm, s, nullptr)
                          : sa::launch_attend_simt_f32(ap, c.head_dim, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   for (int b : act) frames_written[b] += C;
