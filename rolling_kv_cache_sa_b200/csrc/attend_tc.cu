@@ -9,12 +9,13 @@
 // row sum) of its pieces. Without a partials buffer, ranges snap to whole
 // units instead.
 //
-// CTA of 12 warps, per work unit:
-//   warp 0      : TMA producer: Q tiles of the unit, then K and V tiles
-//                 (kStages each, separate barriers so QK^T starts before V lands)
-//   warp 1      : TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 4..7  : softmax + epilogue of query tile 0 (one thread per row)
-//   warps 8..11 : softmax + epilogue of query tile 1
+// CTA of 10 warps, per work unit:
+//   warp 0     : TMA producer: Q tiles of the unit, then K and V tiles
+//                (kStages each, separate barriers so QK^T starts before V lands)
+//   warp 1     : TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2..5 : softmax + epilogue of query tile 0 (one thread per row; a
+//                warp reads TMEM lanes 32*(warp % 4) .. +31)
+//   warps 6..9 : softmax + epilogue of query tile 1
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 after O0.
 // P_i (bf16 pairs) overwrites the first 64 columns of S_i once S_i is in
 // registers and feeds the PV MMA from TMEM (A operand), V being an MN-major
@@ -23,9 +24,8 @@
 // so each tile's softmax runs while the tensor core works on the other tile;
 // tcgen05.mma ops issued by one thread execute in order, so QK_i(j+1) cannot
 // overwrite P_i(j) before PV_i(j) has read it.
-// Online softmax: running max in the log2 domain; O is rescaled in TMEM only
-// when the max grows by more than 8 (factor 256); exact division by the row
-// sum at the end.
+// Online softmax in the log2 domain; O is rescaled in TMEM only when the
+// running max grows by more than 8; exact division by the row sum at the end.
 // Every wait is bounded (about 1 s); on expiry the CTA records a device error,
 // drains its outstanding copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -44,8 +44,7 @@ constexpr int BM = 128;                  // query rows per tile
 constexpr int BN = 128;                  // keys per tile
 constexpr uint32_t PANEL = 128u * 128u;  // one 128-row x 128-byte swizzled panel
 constexpr uint64_t kTimeoutNs = 1000000000ull;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kThreads = 384;
+constexpr int kThreads = 320;
 constexpr int kMaxCtas = 256;
 
 struct TcParams {
@@ -135,6 +134,63 @@ struct Layout {
   static constexpr uint32_t bytes = misc + 16;
   static_assert(bytes <= 232448, "exceeds 227 KB of shared memory per CTA");
 };
+
+// Softmax numerator of one query row for one key tile. The 128 scores are
+// loaded from TMEM once (extra TMEM reads are expensive while the tensor core
+// runs), so the max, the exponentials and the packing run from registers with
+// no control flow between elements. Running max m in the log2 domain: it only
+// moves when the tile's max exceeds it by more than 8 (alpha < 1 is then the
+// factor for O), so P stays below 2^8. P (bf16 pairs) overwrites S columns
+// [0, 64). Returns the fp32 row sum of P.
+__device__ __forceinline__ float row_softmax(uint32_t sbuf, int valid, bool first, float& m,
+                                            float sl2, float& alpha) {
+  uint32_t sv[BN];
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) ptx::tmem_ld32u(sbuf + (uint32_t)c * 32u, sv + c * 32);
+  ptx::tmem_wait_ld_dep(sv);
+  ptx::tmem_wait_ld_dep(sv + 32);
+  ptx::tmem_wait_ld_dep(sv + 64);
+  ptx::tmem_wait_ld_dep(sv + 96);
+  if (valid < BN) {
+#pragma unroll
+    for (int i = 0; i < BN; ++i)
+      if (i >= valid) sv[i] = __float_as_uint(-INFINITY);
+  }
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sv[i]);
+#pragma unroll
+  for (int i = 8; i < BN; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[i]));
+#pragma unroll
+  for (int w2 = 4; w2 > 0; w2 >>= 1)
+#pragma unroll
+    for (int i = 0; i < w2; ++i) mx[i] = fmaxf(mx[i], mx[i + w2]);
+  const float tmax = mx[0] * sl2;
+  alpha = 1.f;
+  if (first) {
+    m = tmax;
+  } else if (tmax > m + 8.0f) {
+    alpha = ptx::ex2(m - tmax);
+    m = tmax;
+  }
+  float ls[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ls[i] = 0.f;
+#pragma unroll
+  for (int q = 0; q < BN / 32; ++q) {
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float p0 = ptx::ex2(fmaf(__uint_as_float(sv[q * 32 + 2 * e]), sl2, -m));
+      const float p1 = ptx::ex2(fmaf(__uint_as_float(sv[q * 32 + 2 * e + 1]), sl2, -m));
+      ls[(e & 3) * 2] += p0;
+      ls[(e & 3) * 2 + 1] += p1;
+      w[e] = ptx::pack_bf16x2(p0, p1);
+    }
+    ptx::tmem_st16u(sbuf + (uint32_t)(q * 16), w);
+  }
+  return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -340,10 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::umma_commit(bar(L::B_DR));
       ptx::mbar_wait(bar(L::B_DR), 0, no_abort, kTimeoutNs);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int ti = (warp - 4) >> 2;  // query tile of this warpgroup
-    const int quad = warp & 3;
+    const int ti = (warp - 2) >> 2;  // query tile: warps 2..5 -> 0, warps 6..9 -> 1
+    const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t sbuf = t_lane + (uint32_t)ti * 128u;
@@ -367,73 +423,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        float sv[BN];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) ptx::tmem_ld32(sbuf + c * 32, sv + c * 32);
-        ptx::tmem_wait_ld();
         const int valid = n_keys - kv * BN;
-        if (valid < BN) {
-#pragma unroll
-          for (int i = 0; i < BN; ++i)
-            if (i >= valid) sv[i] = -INFINITY;
-        }
-        float mx8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
-#pragma unroll
-        for (int i = 8; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-#pragma unroll
-        for (int w2 = 4; w2 > 0; w2 >>= 1)
-#pragma unroll
-          for (int i = 0; i < w2; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + w2]);
-        const float m_tile = mx8[0] * sl2;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (kv == sg.lo) {
-          m_used = m_tile;
-        } else if (m_tile > m_used + kRescaleThreshold) {
-          alpha = ptx::ex2(m_used - m_tile);
-          m_used = m_tile;
-          rescale = true;
-        }
-        float ls8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ls8[i] = 0.f;
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ptx::ex2(fmaf(sv[c * 32 + 2 * e], sl2, -m_used));
-            const float p1 = ptx::ex2(fmaf(sv[c * 32 + 2 * e + 1], sl2, -m_used));
-            ls8[e & 7] += p0 + p1;
-            w[e] = ptx::pack_bf16x2(p0, p1);
-          }
-          ptx::tmem_st16u(sbuf + (uint32_t)c * 16u, w);
-        }
-#pragma unroll
-        for (int w2 = 4; w2 > 0; w2 >>= 1)
-#pragma unroll
-          for (int i = 0; i < w2; ++i) ls8[i] += ls8[i + w2];
-        l = l * alpha + ls8[0];
-        if (kv > sg.lo) {
-          // O_i must hold PV_i of the previous key tile before it is rescaled
+        // the first tile of a piece sets the running max exactly; later tiles
+        // use it as is and only take the slow path (exact max, rescale,
+        // recompute) when the row sum shows a value above 2^16 (or not finite)
+        float alpha;
+        const float lsum = row_softmax(sbuf, valid, kv == sg.lo, m_used, sl2, alpha);
+        const bool rescale = alpha < 1.f;
+        l = l * alpha + lsum;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O_i holds PV_i of the previous key tile: MMAs complete in issue
+          // order and QK_i of this tile (issued after that PV) has completed
           if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_OD + ti), (uint32_t)(gi - 1) & 1,
                                                       abort_flag, kTimeoutNs))) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
-              float ov[32];
-              ptx::tmem_ld32(obuf + c * 32, ov);
-              ptx::tmem_wait_ld();
+          for (int c = 0; c < HD / 32; ++c) {
+            float ov[32];
+            ptx::tmem_ld32(obuf + c * 32, ov);
+            ptx::tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-              ptx::tmem_st32(obuf + c * 32, ov);
-            }
+            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            ptx::tmem_st32(obuf + c * 32, ov);
           }
         }
         ptx::tmem_wait_st();
