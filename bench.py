@@ -57,6 +57,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--eager", action="store_true", help="time eager launches, no CUDA graph")
     ap.add_argument("--chunks", type=int, default=0,
                     help="stream only this many chunks per stream (small profiling cases)")
     return ap.parse_args()
@@ -265,29 +266,58 @@ def main():
     if world > 1:
         dist.barrier()
 
+    def timed(fn, steps):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        e1.synchronize()
+        torch.cuda.synchronize()
+        t_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([t_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            t_ms = float(t.item())
+        return t_ms
+
+    # eager: every library call issued from Python, one launch at a time; the
+    # library's per-launch CUDA events (on the launch stream) time each kernel
     sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
     if sampler:
         sampler.start()
         time.sleep(0.3)
+    eager_steps = args.steps if args.eager else max(1, min(args.steps, 20))
     cache.profile_begin()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record()
-    for _ in range(args.steps):
-        run_step()
-    ev1.record()
-    ev1.synchronize()
-    torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    launches = cache.profile_launches()
+    ms_eager = timed(run_step, eager_steps)
+    launches_per_step = cache.profile_launches() / eager_steps
     prof = cache.profile_end()
+    prof_steps = eager_steps
+
+    # graph: one whole step captured once (every hot call of the library is
+    # capturable: no synchronisation, parameters by value) and replayed with
+    # profiling off, so the graph holds kernel nodes only
+    graph = None
+    if args.eager:
+        ms = ms_eager
+    else:
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            run_step()
+        torch.cuda.synchronize()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        ms = timed(graph.replay, args.steps)
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    launches = int(round(launches_per_step * args.steps))
+    ms_eager /= eager_steps
+    cache.reset()
     ms_step = ms / args.steps
     value = chunks_per_step * args.steps * world / (ms / 1000.0)
 
@@ -295,7 +325,7 @@ def main():
     att_ms, att_n = prof["attend"]
     app_ms, app_n = prof["append"]
     ref_ms, ref_n = prof["refresh"]
-    att_flops_per_launch = step_flops * args.steps / max(att_n, 1)
+    att_flops_per_launch = step_flops * prof_steps / max(att_n, 1)
     att_avg_s = att_ms / 1000.0 / max(att_n, 1)
     achieved = att_flops_per_launch / att_avg_s / 1e12
     app_avg_s = app_ms / 1000.0 / max(app_n, 1)
@@ -360,12 +390,17 @@ def main():
         "attention_frac_of_peak_whole_step": att_tflops_step / pk_burst,
         "append_gbs": append_gbs,
         "append_frac_of_hbm": (append_gbs / hbm) if append_gbs else None,
-        "kernel_ms_per_step": {"attend": att_ms / args.steps, "append": app_ms / args.steps,
-                               "refresh": ref_ms / args.steps},
+        "kernel_ms_per_step": {"attend": att_ms / prof_steps, "append": app_ms / prof_steps,
+                               "refresh": ref_ms / prof_steps},
+        "launch_mode": "cuda graph of one step, replayed" if graph is not None else "eager",
+        "eager_chunks_per_s": chunks_per_step * world / (ms_eager / 1000.0),
+        "eager_ms_per_step": ms_eager,
         "roofline": {"bound": "tensor", "kernel": "attend_tc_kernel<128>",
                      "achieved": achieved, "peak": pk_burst, "unit": "TFLOP/s",
                      "frac": achieved / pk_burst, "peak_source": f"{pk_src} bf16 burst",
                      "frac_of_sustained": achieved / pk_sust,
+                     "duration": "mean of the library's CUDA events around each launch, on "
+                                 "its launch stream, over the eager timed pass",
                      "traffic": PROFILED_TRAFFIC.get(attend_source_hash()),
                      "traffic_note": "ncu dram read+write bytes of one steady-state launch "
                                      "(7168 keys); algorithmic minimum 113 MB"},

@@ -181,10 +181,12 @@ sa_status sa_refresh_delta(const sa_config* cfg, int64_t frames_written, int64_t
                            int64_t* delta);
 
 /* Kernel timing with CUDA events recorded around each launch on the launch
- * stream. sa_profile_begin clears the counters and starts recording (up to
- * 8192 launches); sa_profile_end synchronises and returns the summed device
- * times in milliseconds and the launch counts, then stops recording. Any
- * output pointer may be NULL. */
+ * stream (as external records, so launches captured into a CUDA graph keep
+ * their timing: the events then hold the last replay's times).
+ * sa_profile_begin clears the counters and starts recording (up to 8192
+ * launches); sa_profile_end synchronises and returns the summed device times
+ * in milliseconds and the launch counts, then stops recording. Any output
+ * pointer may be NULL. */
 sa_status sa_profile_begin(sa_cache* h);
 sa_status sa_profile_end(sa_cache* h, double* append_ms, int32_t* n_append, double* attend_ms,
                          int32_t* n_attend, double* refresh_ms, int32_t* n_refresh);

@@ -183,15 +183,26 @@ struct sa_cache {
 
 namespace {
 
+// A record into a capturing stream is made an external event node, so the event
+// still carries a time after each replay; the external flag is refused outside
+// capture, where a plain record does the same.
+void prof_record(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, st);
+}
+
 void prof_before(sa_cache* h, cudaStream_t st, int kind) {
   if (!h->profiling || h->ev_used + 2 > h->ev.size()) return;
-  cudaEventRecord(h->ev[h->ev_used], st);
+  prof_record(h->ev[h->ev_used], st);
   h->ev_kind[h->ev_used / 2] = kind;
 }
 
 void prof_after(sa_cache* h, cudaStream_t st) {
   if (!h->profiling || h->ev_used + 2 > h->ev.size()) return;
-  cudaEventRecord(h->ev[h->ev_used + 1], st);
+  prof_record(h->ev[h->ev_used + 1], st);
   h->ev_used += 2;
 }
 
