@@ -4,10 +4,12 @@
 // Work unit = one (stream, head) and a pair of 128-row query tiles. The key
 // tiles of all units are laid end to end; a persistent grid of one CTA per SM
 // takes equal contiguous ranges of that sequence (stream-K), so no SM idles
-// in a last partial wave. A unit cut by a range boundary is finished by the
-// combine kernel from fp32 partial results (unnormalised O, running max,
-// row sum) of its pieces. Without a partials buffer, ranges snap to whole
-// units instead.
+// in a last partial wave. A unit cut by range boundaries is finished inside
+// the same launch: every piece stores its fp32 partial result (unnormalised
+// O, running max, row sum) and counts itself in on a per-row counter; the
+// thread that arrives last for a row merges all pieces of that row and
+// writes it (no waiting on other CTAs). Without a partials buffer, ranges
+// snap to whole units instead.
 //
 // CTA of 10 warps, per work unit:
 //   warp 0     : TMA producer: Q tiles of the unit, then K and V tiles
@@ -54,8 +56,9 @@ struct TcParams {
   int32_t pad_;
   int64_t total;      // key tiles over all units
   void* out;          // [B][Lc][H][D] bf16
-  float* part_o;      // [slots][2][128][D] fp32
-  float* part_ml;     // [slots][2][128][2] fp32 (m in log2 units, l)
+  float4* part_o;     // [slots][2][D/4][128] fp32 (row-contiguous per column quad)
+  float2* part_ml;    // [slots][2][128] (m in log2 units, l)
+  int* counters;      // [units][2][128] pieces counted in; back to 0 after the merge
   int* status;
   int32_t stream_of[kMaxAttnStreams];
   int32_t n_keys[kMaxAttnStreams];
@@ -110,6 +113,71 @@ __host__ __device__ inline Seg make_seg(const TcParams& p, int64_t t, int64_t r1
   return s;
 }
 
+// CTA whose range holds key tile t (split mode)
+__device__ inline int cta_of(const TcParams& p, int64_t t) {
+  int c = (int)(t * p.grid / p.total);
+  while (c + 1 < p.grid && p.total * (c + 1) / p.grid <= t) ++c;
+  while (c > 0 && p.total * c / p.grid > t) --c;
+  return c;
+}
+
+// Partial slot of the piece that CTA c holds of the unit starting at tile us:
+// slot 2c for a CTA's first segment, 2c + 1 for a later one.
+__device__ inline int piece_slot(const TcParams& p, int c, int c_first, int64_t us) {
+  return 2 * c + ((c == c_first && p.total * c / p.grid != us) ? 1 : 0);
+}
+
+// Merge of one query row of a split unit from the partial results of its
+// pieces (CTAs c0..c1): O = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,
+// stored as bf16 to dst (nullptr: a padding row past Lc, nothing stored).
+// Kept out of line so the softmax loop's register allocation does not see it.
+template <int HD>
+__device__ __noinline__ void merge_row(const TcParams& p, int ti, int row, int c0, int c1,
+                                       int64_t us, __nv_bfloat16* dst) {
+  float M = -INFINITY;
+  for (int c = c0; c <= c1; ++c) {
+    const int sl = piece_slot(p, c, c0, us);
+    M = fmaxf(M, __ldcg(p.part_ml + ((int64_t)sl * 2 + ti) * BM + row).x);
+  }
+  float Ls = 0.f;
+  for (int c = c0; c <= c1; ++c) {
+    const int sl = piece_slot(p, c, c0, us);
+    const float2 ml = __ldcg(p.part_ml + ((int64_t)sl * 2 + ti) * BM + row);
+    Ls += ptx::ex2(ml.x - M) * ml.y;
+  }
+  const float inv = 1.f / Ls;
+  if (!dst) return;
+#pragma unroll 1
+  for (int cc = 0; cc < HD / 32; ++cc) {
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    for (int c = c0; c <= c1; ++c) {
+      const int sl = piece_slot(p, c, c0, us);
+      const float2 ml = __ldcg(p.part_ml + ((int64_t)sl * 2 + ti) * BM + row);
+      const float w = ptx::ex2(ml.x - M);
+      const float4* src = p.part_o + (((int64_t)sl * 2 + ti) * (HD / 4) + cc * 8) * BM + row;
+#pragma unroll
+      for (int g4 = 0; g4 < 8; ++g4) {
+        const float4 v = __ldcg(src + g4 * BM);
+        acc[g4 * 4 + 0] = fmaf(w, v.x, acc[g4 * 4 + 0]);
+        acc[g4 * 4 + 1] = fmaf(w, v.y, acc[g4 * 4 + 1]);
+        acc[g4 * 4 + 2] = fmaf(w, v.z, acc[g4 * 4 + 2]);
+        acc[g4 * 4 + 3] = fmaf(w, v.w, acc[g4 * 4 + 3]);
+      }
+    }
+#pragma unroll
+    for (int g8 = 0; g8 < 4; ++g8) {
+      uint4 v;
+      v.x = ptx::pack_bf16x2(acc[g8 * 8 + 0] * inv, acc[g8 * 8 + 1] * inv);
+      v.y = ptx::pack_bf16x2(acc[g8 * 8 + 2] * inv, acc[g8 * 8 + 3] * inv);
+      v.z = ptx::pack_bf16x2(acc[g8 * 8 + 4] * inv, acc[g8 * 8 + 5] * inv);
+      v.w = ptx::pack_bf16x2(acc[g8 * 8 + 6] * inv, acc[g8 * 8 + 7] * inv);
+      *reinterpret_cast<uint4*>(dst + cc * 32 + g8 * 8) = v;
+    }
+  }
+}
+
 template <int HD>
 struct Layout {
   static constexpr int kStages = HD == 128 ? 2 : 4;
@@ -125,8 +193,9 @@ struct Layout {
   static constexpr int B_VF = B_KE + kStages;
   static constexpr int B_VE = B_VF + kStages;
   static constexpr int B_SF = B_VE + kStages;  // [2] S_i written by QK_i
-  static constexpr int B_PF = B_SF + 2;        // [2] P_i written by softmax i
-  static constexpr int B_OD = B_PF + 2;        // [2] PV_i done
+  static constexpr int B_PF = B_SF + 2;        // [2] P_i keys [0, 64) written by softmax i
+  static constexpr int B_PB = B_PF + 2;        // [2] P_i keys [64, 128) written
+  static constexpr int B_OD = B_PB + 2;        // [2] PV_i done
   static constexpr int B_OF = B_OD + 2;        // [2] O_i read by the epilogue
   static constexpr int B_DR = B_OF + 2;        // drain
   static constexpr int kNumBars = B_DR + 1;
@@ -135,15 +204,37 @@ struct Layout {
   static_assert(bytes <= 232448, "exceeds 227 KB of shared memory per CTA");
 };
 
+// O row *= alpha in TMEM (rare; out of line so that the softmax keeps its
+// scores in registers without spilling around it)
+template <int HD>
+__device__ __noinline__ void rescale_o(uint32_t obuf, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < HD / 32; ++c) {
+    float ov[32];
+    ptx::tmem_ld32(obuf + c * 32, ov);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+    ptx::tmem_st32(obuf + c * 32, ov);
+  }
+}
+
 // Softmax numerator of one query row for one key tile. The 128 scores are
 // loaded from TMEM once (extra TMEM reads are expensive while the tensor core
 // runs), so the max, the exponentials and the packing run from registers with
 // no control flow between elements. Running max m in the log2 domain: it only
 // moves when the tile's max exceeds it by more than 8 (alpha < 1 is then the
-// factor for O), so P stays below 2^8. P (bf16 pairs) overwrites S columns
-// [0, 64). Returns the fp32 row sum of P.
-__device__ __forceinline__ float row_softmax(uint32_t sbuf, int valid, bool first, float& m,
-                                            float sl2, float& alpha) {
+// factor for O), so P stays below 2^8. A rescale of O (rare) is done before
+// any P is published (PV accumulates onto it); it only needs PV of the
+// previous key tile complete (bar_od). P (bf16 pairs) overwrites S columns [0, 64) and is published in
+// two halves, keys [0, 64) on bar_pa and [64, 128) on bar_pb, so the PV MMA
+// of the first half runs while the second half is computed. Adds the row sum
+// of P to l (after scaling l by alpha). Returns false if a wait gave up.
+template <int HD>
+__device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int valid, bool first,
+                                            float& m, float& l, float sl2, uint32_t bar_od,
+                                            uint32_t od_parity, uint32_t bar_pa, uint32_t bar_pb,
+                                            volatile int* abort_flag) {
   uint32_t sv[BN];
 #pragma unroll
   for (int c = 0; c < BN / 32; ++c) ptx::tmem_ld32u(sbuf + (uint32_t)c * 32u, sv + c * 32);
@@ -158,15 +249,16 @@ __device__ __forceinline__ float row_softmax(uint32_t sbuf, int valid, bool firs
   }
   float mx[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sv[i]);
+  for (int i = 0; i < 8; ++i) mx[i] = fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[i + 8]));
 #pragma unroll
-  for (int i = 8; i < BN; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[i]));
+  for (int i = 16; i < BN; i += 16)
 #pragma unroll
-  for (int w2 = 4; w2 > 0; w2 >>= 1)
-#pragma unroll
-    for (int i = 0; i < w2; ++i) mx[i] = fmaxf(mx[i], mx[i + w2]);
-  const float tmax = mx[0] * sl2;
-  alpha = 1.f;
+    for (int k = 0; k < 8; ++k)
+      mx[k] = ptx::fmax3(mx[k], __uint_as_float(sv[i + k]), __uint_as_float(sv[i + 8 + k]));
+  const float tmax =
+      ptx::fmax3(ptx::fmax3(mx[0], mx[1], mx[2]), ptx::fmax3(mx[3], mx[4], mx[5]),
+                 fmaxf(mx[6], mx[7])) * sl2;
+  float alpha = 1.f;
   if (first) {
     m = tmax;
   } else if (tmax > m + 8.0f) {
@@ -188,8 +280,22 @@ __device__ __forceinline__ float row_softmax(uint32_t sbuf, int valid, bool firs
       w[e] = ptx::pack_bf16x2(p0, p1);
     }
     ptx::tmem_st16u(sbuf + (uint32_t)(q * 16), w);
+    if (q == 1 && __any_sync(0xffffffffu, alpha < 1.f)) {
+      // O holds PV of the previous key tile: MMAs complete in issue order and
+      // QK of this tile (issued after that PV) has completed
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_od, od_parity, abort_flag, kTimeoutNs)))
+        return false;
+      ptx::tc_fence_after();
+      rescale_o<HD>(obuf, alpha);
+    }
+    if (q == 1 || q == 3) {
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(q == 1 ? bar_pa : bar_pb);
+    }
   }
-  return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+  l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
+  return true;
 }
 
 template <int HD>
@@ -225,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(bar(L::B_SF + i), 1);
       ptx::mbar_init(bar(L::B_PF + i), 128);
+      ptx::mbar_init(bar(L::B_PB + i), 128);
       ptx::mbar_init(bar(L::B_OD + i), 1);
       ptx::mbar_init(bar(L::B_OF + i), 128);
     }
@@ -316,16 +423,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pend_first && pend_nseg1 > 0 &&
             !ptx::mbar_wait(bar(L::B_OF + 1), (uint32_t)(pend_nseg1 - 1) & 1, abort_flag, kTimeoutNs))
           return false;
-        if (!ptx::mbar_wait(bar(L::B_PF + 1), (uint32_t)pend_g1 & 1, abort_flag, kTimeoutNs))
-          return false;
-        ptx::tc_fence_after();
         const int s = pend_g % ST;
         const uint32_t vb = base + L::v0 + s * L::kTile;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          if (!ptx::mbar_wait(bar((h2 == 0 ? L::B_PF : L::B_PB) + 1), (uint32_t)pend_g1 & 1,
+                              abort_flag, kTimeoutNs))
+            return false;
+          ptx::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          ptx::umma_ts(o1, tmem + 128u + (uint32_t)kk * 8u,
-                       ptx::sdesc_sw128(vb + (uint32_t)kk * 2048u, PANEL, 1024), idesc_pv,
-                       (!pend_first || kk > 0) ? 1u : 0u);
+          for (int k2 = 0; k2 < BN / 32; ++k2) {
+            const int kk = h2 * (BN / 32) + k2;
+            ptx::umma_ts(o1, tmem + 128u + (uint32_t)kk * 8u,
+                         ptx::sdesc_sw128(vb + (uint32_t)kk * 2048u, PANEL, 1024), idesc_pv,
+                         (!pend_first || kk > 0) ? 1u : 0u);
+          }
+        }
         ptx::umma_commit(bar(L::B_OD + 1));
         ptx::umma_commit(bar(L::B_VE + s));
         pend = false;
@@ -367,14 +479,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (!ptx::mbar_wait(bar(L::B_PF + 0), (uint32_t)g & 1, abort_flag, kTimeoutNs)) { ok = false; break; }
-          ptx::tc_fence_after();
           const uint32_t vb = base + L::v0 + s * L::kTile;
+          for (int h2 = 0; h2 < 2 && ok; ++h2) {
+            if (!ptx::mbar_wait(bar((h2 == 0 ? L::B_PF : L::B_PB) + 0), (uint32_t)g & 1, abort_flag,
+                                kTimeoutNs)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            ptx::umma_ts(o0, tmem + (uint32_t)kk * 8u,
-                         ptx::sdesc_sw128(vb + (uint32_t)kk * 2048u, PANEL, 1024), idesc_pv,
-                         (kv > sg.lo || kk > 0) ? 1u : 0u);
+            for (int k2 = 0; k2 < BN / 32; ++k2) {
+              const int kk = h2 * (BN / 32) + k2;
+              ptx::umma_ts(o0, tmem + (uint32_t)kk * 8u,
+                           ptx::sdesc_sw128(vb + (uint32_t)kk * 2048u, PANEL, 1024), idesc_pv,
+                           (kv > sg.lo || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
           ptx::umma_commit(bar(L::B_OD + 0));
           if (sg.two) {
             pend = true;
@@ -424,35 +545,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         const int valid = n_keys - kv * BN;
-        // the first tile of a piece sets the running max exactly; later tiles
-        // use it as is and only take the slow path (exact max, rescale,
-        // recompute) when the row sum shows a value above 2^16 (or not finite)
-        float alpha;
-        const float lsum = row_softmax(sbuf, valid, kv == sg.lo, m_used, sl2, alpha);
-        const bool rescale = alpha < 1.f;
-        l = l * alpha + lsum;
-        if (__any_sync(0xffffffffu, rescale)) {
-          // O_i holds PV_i of the previous key tile: MMAs complete in issue
-          // order and QK_i of this tile (issued after that PV) has completed
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_OD + ti), (uint32_t)(gi - 1) & 1,
-                                                      abort_flag, kTimeoutNs))) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
-            float ov[32];
-            ptx::tmem_ld32(obuf + c * 32, ov);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-            ptx::tmem_st32(obuf + c * 32, ov);
-          }
+        if (!row_softmax<HD>(sbuf, obuf, valid, kv == sg.lo, m_used, l, sl2, bar(L::B_OD + ti),
+                             (uint32_t)(gi - 1) & 1, bar(L::B_PF + ti), bar(L::B_PB + ti),
+                             abort_flag)) {
+          ok = false;
+          break;
         }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(L::B_PF + ti));
       }
       if (!ok) break;
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_OD + ti), (uint32_t)(gi - 1) & 1,
@@ -486,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const int slot = 2 * (int)blockIdx.x + (seg_first ? 0 : 1);
-        float* po = p.part_o + (((int64_t)slot * 2 + ti) * BM + row) * HD;
+        float4* po = p.part_o + ((int64_t)slot * 2 + ti) * (HD / 4) * BM + row;
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           float ov[32];
@@ -494,14 +592,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_wait_ld();
 #pragma unroll
           for (int g4 = 0; g4 < 8; ++g4)
-            *reinterpret_cast<float4*>(po + c * 32 + g4 * 4) =
+            po[(c * 8 + g4) * BM] =
                 make_float4(ov[g4 * 4], ov[g4 * 4 + 1], ov[g4 * 4 + 2], ov[g4 * 4 + 3]);
         }
-        *reinterpret_cast<float2*>(p.part_ml + (((int64_t)slot * 2 + ti) * BM + row) * 2) =
-            make_float2(m_used, l);
+        p.part_ml[((int64_t)slot * 2 + ti) * BM + row] = make_float2(m_used, l);
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(L::B_OF + ti));
+      ptx::mbar_arrive(bar(L::B_OF + ti));  // O_i is free for the next unit
+      if (sg.partial) {
+        // count this piece in for the row; the last one merges all pieces
+        const int64_t us = sg.t_end - (sg.hi - sg.lo) - sg.lo;
+        const int c0 = cta_of(p, us), c1 = cta_of(p, us + sg.nkv - 1);
+        const int64_t u = (int64_t)sg.a * p.units_per_stream + (int64_t)sg.h * p.n_pairs + sg.qp;
+        int* ctr = p.counters + (u * 2 + ti) * BM + row;
+        __threadfence();
+        if (atomicAdd(ctr, 1) == c1 - c0) {
+          atomicExch(ctr, 0);
+          __threadfence();
+          merge_row<HD>(p, ti, row, c0, c1, us,
+                        tok < p.Lc ? static_cast<__nv_bfloat16*>(p.out) +
+                                         (((int64_t)sg.b * p.Lc + tok) * p.H + sg.h) * HD
+                                   : nullptr);
+        }
+      }
     }
     if (!ok) fail();
   }
@@ -510,57 +623,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == 1) ptx::tmem_dealloc(tmem, 512);
-}
-
-// ---------------------------------------------------------------- combine
-constexpr int kMaxCombine = kMaxCtas;
-
-struct CombineParams {
-  int32_t H, Lc, n_q_tiles, n_units;
-  const float* part_o;
-  const float* part_ml;
-  void* out;
-  int32_t unit_b[kMaxCombine];
-  int32_t unit_h[kMaxCombine];
-  int32_t unit_qp[kMaxCombine];
-  int32_t slot_begin[kMaxCombine + 1];
-  int32_t slots[2 * kMaxCtas];
-};
-
-// One warp per output row: O = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k.
-template <int HD>
-__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ CombineParams p) {
-  constexpr int PER = HD / 32;
-  const int u = blockIdx.x, ti = blockIdx.y;
-  const int row = blockIdx.z * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const int qt = 2 * p.unit_qp[u] + ti;
-  if (qt >= p.n_q_tiles) return;
-  const int tok = qt * BM + row;
-  if (tok >= p.Lc) return;
-  const int k0 = p.slot_begin[u], k1 = p.slot_begin[u + 1];
-  float M = -INFINITY;
-  for (int k = k0; k < k1; ++k)
-    M = fmaxf(M, p.part_ml[(((int64_t)p.slots[k] * 2 + ti) * BM + row) * 2]);
-  float acc[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  float Lsum = 0.f;
-  for (int k = k0; k < k1; ++k) {
-    const int64_t r = ((int64_t)p.slots[k] * 2 + ti) * BM + row;
-    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + r * 2);
-    const float w = exp2f(ml.x - M);
-    Lsum += w * ml.y;
-    const float* src = p.part_o + r * HD + lane * PER;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] += w * src[e];
-  }
-  const float inv = 1.f / Lsum;
-  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
-                       (((int64_t)p.unit_b[u] * p.Lc + tok) * p.H + p.unit_h[u]) * HD + lane * PER;
-#pragma unroll
-  for (int e = 0; e < PER; e += 2)
-    *reinterpret_cast<uint32_t*>(dst + e) = ptx::pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
 }
 
 template <int HD>
@@ -600,74 +662,31 @@ cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtenso
   p.total = total;
   const int64_t units = (int64_t)ap.n_streams * p.units_per_stream;
   int G = std::min(num_sms, kMaxCtas);
-  const size_t need = attend_partials_bytes(HD, G);
+  const size_t need = attend_partials_bytes(HD, G, units);
   p.split = partials != nullptr && partials_bytes >= need && total >= G;
   if (!p.split) G = (int)std::min<int64_t>(G, units);
   p.grid = G;
-  p.part_o = static_cast<float*>(partials);
-  p.part_ml = p.part_o ? p.part_o + (size_t)2 * G * 2 * BM * HD : nullptr;
+  if (p.split) {
+    char* w = static_cast<char*>(partials);
+    p.part_o = reinterpret_cast<float4*>(w);
+    w += (size_t)2 * G * 2 * BM * HD * sizeof(float);
+    p.part_ml = reinterpret_cast<float2*>(w);
+    w += (size_t)2 * G * 2 * BM * sizeof(float2);
+    p.counters = reinterpret_cast<int*>(w);
+  }
   attend_tc_kernel<HD><<<G, kThreads, L::bytes, st>>>(*tq, *tk, *tv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  int launched = 1;
-  if (p.split) {
-    // the units cut by CTA range boundaries, with the partial slot of each piece in key order
-    CombineParams cp;
-    memset(&cp, 0, sizeof(cp));
-    cp.H = p.H;
-    cp.Lc = p.Lc;
-    cp.n_q_tiles = p.n_q_tiles;
-    cp.part_o = p.part_o;
-    cp.part_ml = p.part_ml;
-    cp.out = p.out;
-    struct Piece { int64_t unit_start; int lo; int slot; int b, h, qp; };
-    std::vector<Piece> pieces;
-    for (int c = 0; c < G; ++c) {
-      int64_t r0, r1;
-      cta_range(p, c, r0, r1);
-      bool first = true;
-      for (int64_t t = r0; t < r1;) {
-        const Seg sg = make_seg(p, t, r1);
-        if (sg.partial)
-          pieces.push_back({t - sg.lo, sg.lo, 2 * c + (first ? 0 : 1), sg.b, sg.h, sg.qp});
-        first = false;
-        t = sg.t_end;
-      }
-    }
-    std::stable_sort(pieces.begin(), pieces.end(), [](const Piece& x, const Piece& y) {
-      return x.unit_start != y.unit_start ? x.unit_start < y.unit_start : x.lo < y.lo;
-    });
-    int nu = 0, ns = 0;
-    for (size_t i = 0; i < pieces.size(); ++i) {
-      if (i == 0 || pieces[i].unit_start != pieces[i - 1].unit_start) {
-        if (nu >= kMaxCombine) return cudaErrorInvalidValue;
-        cp.unit_b[nu] = pieces[i].b;
-        cp.unit_h[nu] = pieces[i].h;
-        cp.unit_qp[nu] = pieces[i].qp;
-        cp.slot_begin[nu] = ns;
-        ++nu;
-      }
-      if (ns >= 2 * kMaxCtas) return cudaErrorInvalidValue;
-      cp.slots[ns++] = pieces[i].slot;
-    }
-    cp.slot_begin[nu] = ns;
-    cp.n_units = nu;
-    if (nu > 0) {
-      combine_kernel<HD><<<dim3(nu, 2, BM / 8), 256, 0, st>>>(cp);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-      ++launched;
-    }
-  }
+  const int launched = 1;
   if (n_kernels) *n_kernels = launched;
   return cudaSuccess;
 }
 
 }  // namespace
 
-size_t attend_partials_bytes(int D, int num_sms) {
+size_t attend_partials_bytes(int D, int num_sms, int64_t max_units) {
   const size_t G = (size_t)std::min(num_sms, kMaxCtas);
-  return 2 * G * 2 * BM * ((size_t)D * 4 + 8);
+  return 2 * G * 2 * BM * ((size_t)D * 4 + 8) + (size_t)max_units * 2 * BM * sizeof(int);
 }
 
 cudaError_t launch_attend_tc_bf16(const AttnParams& p, int D, const CUtensorMap* tm_q,

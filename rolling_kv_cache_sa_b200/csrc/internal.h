@@ -75,16 +75,21 @@ struct AttnParams {
 };
 
 // Workspace the bf16 attention may use for split work units: per slot (two
-// per CTA) the unnormalised fp32 O of two 128-row tiles and their (m, l).
-size_t attend_partials_bytes(int D, int num_sms);
+// per CTA) the unnormalised fp32 O of two 128-row tiles and their (m, l),
+// then one arrival counter per (unit, tile, row) for max_units units (a unit
+// is a stream, a head and a pair of 128-row query tiles). The counters must
+// be zero before the first launch; every launch that completes leaves them
+// zero again.
+size_t attend_partials_bytes(int D, int num_sms, int64_t max_units);
 
 cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_refresh(const RefreshParams& p, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_attend_simt_f32(const AttnParams& p, int D, cudaStream_t st);
 // bf16 tensor-core attention. `partials` (attend_partials_bytes) lets the
-// persistent kernel split work units at equal-work boundaries (a combine
-// kernel then merges the pieces); with partials == nullptr every CTA takes
-// whole units. *n_kernels (if non-null) receives the kernels launched.
+// persistent kernel split work units at equal-work boundaries (the last
+// piece of each row to finish merges the pieces); with partials == nullptr
+// every CTA takes whole units. *n_kernels (if non-null) receives the kernels
+// launched.
 cudaError_t launch_attend_tc_bf16(const AttnParams& p, int D, const CUtensorMap* tm_q,
                                   const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                   void* partials, size_t partials_bytes, int num_sms,

@@ -269,6 +269,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// max of three floats in one instruction (sm_100 three-input max.f32)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   // cvt.rn.bf16x2.f32 d, a, b puts a in the upper half and b in the lower half

@@ -327,8 +327,20 @@ sa_status sa_cache_create(const sa_config* cfg, sa_stream_t stream, sa_cache** o
     return cuda_fail(e, "table upload");
   }
   if (cfg->dtype == SA_BF16) {
-    h->partials_bytes = sa::attend_partials_bytes((int)D, h->num_sms);
+    const int64_t max_units = B * H * ((h->Lc + 255) / 256);
+    h->partials_bytes = sa::attend_partials_bytes((int)D, h->num_sms, max_units);
     e = cudaMalloc(&h->partials, h->partials_bytes);
+    if (e == cudaSuccess) {  // the split-unit arrival counters start at zero
+      e = cudaMemsetAsync(h->partials, 0, h->partials_bytes, cs);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+      if (e != cudaSuccess) {
+        cudaFree(h->partials);
+        h->partials = nullptr;
+        free_all(h);
+        delete h;
+        return cuda_fail(e, "partials init");
+      }
+    }
     if (e != cudaSuccess) {
       h->partials = nullptr;
       free_all(h);
