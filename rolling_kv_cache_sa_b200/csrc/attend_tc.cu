@@ -228,7 +228,11 @@ __device__ __noinline__ void rescale_o(uint32_t obuf, float alpha) {
 // any P is published (PV accumulates onto it); it only needs PV of the
 // previous key tile complete (bar_od). P (bf16 pairs) overwrites S columns [0, 64) and is published in
 // two halves, keys [0, 64) on bar_pa and [64, 128) on bar_pb, so the PV MMA
-// of the first half runs while the second half is computed. Adds the row sum
+// of the first half runs while the second half is computed. The scale and
+// subtract and the row sums use packed two-float FMA/add: the phase is bound
+// by instruction count and latency rather than by the exponential unit's
+// rate (moving a share of the exponentials to a polynomial on the FMA pipe
+// made it slower). Adds the row sum
 // of P to l (after scaling l by alpha). Returns false if a wait gave up.
 template <int HD>
 __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int valid, bool first,
@@ -265,19 +269,21 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
     alpha = ptx::ex2(m - tmax);
     m = tmax;
   }
-  float ls[8];
+  const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(-m, -m);
+  float2 ls[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) ls[i] = 0.f;
+  for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int q = 0; q < BN / 32; ++q) {
     uint32_t w[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float p0 = ptx::ex2(fmaf(__uint_as_float(sv[q * 32 + 2 * e]), sl2, -m));
-      const float p1 = ptx::ex2(fmaf(__uint_as_float(sv[q * 32 + 2 * e + 1]), sl2, -m));
-      ls[(e & 3) * 2] += p0;
-      ls[(e & 3) * 2 + 1] += p1;
-      w[e] = ptx::pack_bf16x2(p0, p1);
+      const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[q * 32 + 2 * e]),
+                                              __uint_as_float(sv[q * 32 + 2 * e + 1])),
+                                  sl2v, nmv);
+      const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+      ls[e & 3] = __fadd2_rn(ls[e & 3], pe);
+      w[e] = ptx::pack_bf16x2(pe.x, pe.y);
     }
     ptx::tmem_st16u(sbuf + (uint32_t)(q * 16), w);
     if (q == 1 && __any_sync(0xffffffffu, alpha < 1.f)) {
@@ -294,7 +300,8 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
       ptx::mbar_arrive(q == 1 ? bar_pa : bar_pb);
     }
   }
-  l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
+  const float2 l2 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+  l = l * alpha + (l2.x + l2.y);
   return true;
 }
 
