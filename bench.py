@@ -35,7 +35,7 @@ METRIC = "streamed chunks/s and attention TFLOP/s (% of B200 BF16 peak) per conf
 # DRAM bytes (read + write) per launch of the attention kernel, from the ncu
 # capture summarised in profiles/ (512p, steady chunk with 7168 keys), keyed by
 # a hash of the kernel sources it was taken on: a changed kernel reports null.
-PROFILED_TRAFFIC = {"f993361fc77cc7f0": 106.1e6}
+PROFILED_TRAFFIC = {"fff8e35f79fc94b1": 183.66e6}
 
 
 def attend_source_hash() -> str:
@@ -403,7 +403,9 @@ def main():
                                  "its launch stream, over the eager timed pass",
                      "traffic": PROFILED_TRAFFIC.get(attend_source_hash()),
                      "traffic_note": "ncu dram read+write bytes of one steady-state launch "
-                                     "(7168 keys); algorithmic minimum 113 MB"},
+                                     "(7168 keys, cold L2); algorithmic minimum 113 MB; the "
+                                     "excess is split-unit fp32 partials written and read "
+                                     "back (~39 MB) and K/V re-reads past L2"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
