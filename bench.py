@@ -219,6 +219,7 @@ def main():
 
     import inputgen as IG
     from rolling_kv_cache_sa_b200 import SACache, attention_flops, config_for, sa_plan_chunk
+    from rolling_kv_cache_sa_b200.dist import aggregate_rate, max_over_ranks, rank_stream_ids
     from rolling_kv_cache_sa_b200.session import StreamSession
 
     torch.cuda.set_device(local)
@@ -238,7 +239,7 @@ def main():
     v_all = torch.empty_like(q_all)
     out_all = torch.empty_like(q_all)
     st = torch.cuda.current_stream().cuda_stream
-    stream_ids = [rank * w.B + b for b in range(w.B)]  # distinct streams per rank
+    stream_ids = rank_stream_ids(rank, w.B)  # distinct streams per rank
     actives = []
     for g in range(n_steps_g):
         chunks = w.local_chunks(g)
@@ -277,12 +278,7 @@ def main():
         e1.record()
         e1.synchronize()
         torch.cuda.synchronize()
-        t_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([t_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t_ms = float(t.item())
-        return t_ms
+        return max_over_ranks(e0.elapsed_time(e1), "cuda")
 
     # eager: every library call issued from Python, one launch at a time; the
     # library's per-launch CUDA events (on the launch stream) time each kernel
@@ -316,10 +312,30 @@ def main():
         ms = timed(graph.replay, args.steps)
     clocks = sampler.stop() if sampler else None
     launches = int(round(launches_per_step * args.steps))
+
+    # per-call latency: two eager steps, CUDA events around each call (device
+    # time of the call's kernels on the launch stream, refresh included when due)
+    lat = []
+    for _ in range(2):
+        cache.reset()
+        evs = []
+        for g in range(n_steps_g):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sess.step(q_all[g], k_all[g], v_all[g], out_all[g], actives[g])
+            e1.record()
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        lat += [a.elapsed_time(b) for a, b in evs]
+    import numpy as np
+    call_latency = {"p50_ms": float(np.percentile(lat, 50)), "p99_ms": float(np.percentile(lat, 99)),
+                    "calls": len(lat),
+                    "what": "device time per step call (append + attention, refresh when due), "
+                            "eager, CUDA events on the launch stream"}
     ms_eager /= eager_steps
     cache.reset()
     ms_step = ms / args.steps
-    value = chunks_per_step * args.steps * world / (ms / 1000.0)
+    value = aggregate_rate(chunks_per_step * args.steps, world, ms)
 
     hbm, pk_burst, pk_sust, pk_src = peaks()
     att_ms, att_n = prof["attend"]
@@ -356,13 +372,9 @@ def main():
             run_step_host()
         e1.record()
         e1.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), "cuda")
         per_chunk_in = 3 * w.Lc * w.H * w.D * esz
-        e2e = {"value": chunks_per_step * args.e2e_steps * world / (ems / 1000.0),
+        e2e = {"value": aggregate_rate(chunks_per_step * args.e2e_steps, world, ems),
                "unit": "chunks/s", "steps": args.e2e_steps,
                "h2d_bytes_per_step": per_chunk_in * chunks_per_step,
                "d2h_bytes_per_step": w.Lc * w.H * w.D * esz * chunks_per_step,
@@ -392,6 +404,7 @@ def main():
         "append_frac_of_hbm": (append_gbs / hbm) if append_gbs else None,
         "kernel_ms_per_step": {"attend": att_ms / prof_steps, "append": app_ms / prof_steps,
                                "refresh": ref_ms / prof_steps},
+        "call_latency": call_latency,
         "launch_mode": "cuda graph of one step, replayed" if graph is not None else "eager",
         "eager_chunks_per_s": chunks_per_step * world / (ms_eager / 1000.0),
         "eager_ms_per_step": ms_eager,

@@ -123,6 +123,23 @@ sa_status sa_append_attend(sa_cache* h, const void* q, const void* k, const void
                            const uint8_t* active, sa_stream_t stream);
 
 /*
+ * Attention of the next chunk without committing it (StreamDiffusionV2,
+ * section 2.B.2 "Stream-Batch": a chunk is denoised over several steps, and
+ * each step is a forward pass over the same cached context with that step's
+ * latents; section 3 reports 1-step and 4-step runs). Same arguments, layouts
+ * and output as sa_append_attend: the chunk's queries attend to the cached
+ * context plus the chunk's own keys and values. The chunk's rotated keys and
+ * values are written into the cache rows the chunk will occupy -- ring rows
+ * whose frames no chunk from this one on can see (or empty sink rows) -- but
+ * frames_written and pos_base do not advance, so the next sa_attend or
+ * sa_append_attend on the handle processes the same chunk again, overwriting
+ * those rows; the final step of a chunk calls sa_append_attend, which commits.
+ * Never synchronises (capturable in a CUDA graph). Errors as sa_append_attend.
+ */
+sa_status sa_attend(sa_cache* h, const void* q, const void* k, const void* v, void* out,
+                    const uint8_t* active, sa_stream_t stream);
+
+/*
  * RoPE refresh of the active streams (StreamDiffusionV2, section 2.A.2):
  * before stream b's next chunk c, every cached position is rebased by
  *   Delta = max(S, cC - W) - pos_base,
@@ -152,6 +169,28 @@ sa_status sa_cache_destroy(sa_cache* h);
  */
 sa_status sa_append_attend_host(sa_cache* h, const void* q, const void* k, const void* v,
                                 void* out, const uint8_t* active, sa_stream_t stream);
+
+/*
+ * Pipelined host-buffer variant: the same work as sa_append_attend_host, but
+ * the call returns once the work is queued, so consecutive calls overlap the
+ * host-to-device copies of one chunk, the computation of another and the
+ * device-to-host copy of a third. The handle owns three staging slots (q, k,
+ * v, out; allocated by the first call) and two copy streams; events order
+ * copy-in -> compute (on `stream`) -> copy-out per slot, and a slot is reused
+ * only after its previous chunk's computation and copy-out completed.
+ * Ownership: q, k, v are read until their copies complete; `out` is written
+ * when the copy-out completes. Call sa_host_wait before reading `out` or
+ * reusing the input buffers. Page-locked host memory is needed for copies to
+ * overlap (pageable memory works but serialises). Refreshes on `stream` are
+ * ordered with the computations. Errors as sa_append_attend (validated before
+ * any copy is queued), SA_ERR_CUDA on a copy or setup failure.
+ */
+sa_status sa_append_attend_host_async(sa_cache* h, const void* q, const void* k, const void* v,
+                                      void* out, const uint8_t* active, sa_stream_t stream);
+
+/* Blocks until every copy queued by sa_append_attend_host_async on the handle
+ * has completed (and with them the computations they follow). */
+sa_status sa_host_wait(sa_cache* h);
 
 /* ---- introspection (tests, benchmarks) ---- */
 
@@ -227,6 +266,60 @@ sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cache, void* v_
 
 /* Number of kernels the handle launched since sa_profile_begin (host count). */
 sa_status sa_profile_launches(const sa_cache* h, int64_t* launches);
+
+/* Sink position modes (sa_cache_set_sink_mode). */
+#define SA_SINK_SHIFT 0 /* a refresh rebases the sink with every other position: scores invariant */
+#define SA_SINK_REPIN 1 /* after a refresh the sink sits right before the oldest window frame */
+
+/*
+ * How the sink's temporal positions follow a RoPE refresh (StreamDiffusionV2,
+ * section 2.A.2: RoPE offsets are reset at block boundaries; sink tokens
+ * anchor the stream). SA_SINK_SHIFT (the default): sink frame f is at
+ * t = f - pos_base, like every other key, so a refresh leaves every score
+ * unchanged. SA_SINK_REPIN: sink frame f is at t = f - min(pos_base, S): a
+ * refresh (which sets pos_base >= S and puts the oldest visible window frame
+ * at t = 0) places the sink immediately before the window, instead of ever
+ * farther in the past; scores involving the sink change at each refresh.
+ * Takes effect at the next sa_rope_refresh or sa_sink_update (stored keys are
+ * not touched by this call). Host only; never fails for a valid handle and
+ * mode (SA_ERR_INVALID_ARG otherwise). sa_append_attend_noalloc always shifts.
+ */
+sa_status sa_cache_set_sink_mode(sa_cache* h, int32_t mode);
+
+/*
+ * Adaptive sink update (StreamDiffusionV2, section 2.A.2: sink tokens are
+ * updated dynamically from the prompt's semantics and the recent visual
+ * context). For every active stream, the sink's raw (unrotated) keys and its
+ * values become (1 - alpha) * old + alpha * new, computed in fp32 and rounded
+ * to the cache dtype; the stored sink keys are then re-derived from the new
+ * raw keys at the sink's current positions (sa_cache_set_sink_mode).
+ *   k_new, v_new : device, [B][S*F][H][D] in cfg dtype (the sink frames'
+ *                  tokens in frame, row, column order), contiguous, 16-byte
+ *                  aligned; rows of inactive streams are not read. Borrowed
+ *                  until the stream-ordered work completes.
+ *   alpha        : in [0, 1]; 1 replaces the sink, 0 leaves it unchanged.
+ *   active       : host, B bytes or NULL for all streams.
+ * One kernel on `stream`; never synchronises. Errors: SA_ERR_INVALID_ARG
+ * (no sink, NULL or unaligned buffers, alpha outside [0, 1]), SA_ERR_STATE
+ * (an active stream's sink frames are not all written yet), SA_ERR_UNSUPPORTED
+ * (more than 16 sink frames), SA_ERR_CUDA; nothing is launched on error.
+ */
+sa_status sa_sink_update(sa_cache* h, const void* k_new, const void* v_new, float alpha,
+                         const uint8_t* active, sa_stream_t stream);
+
+/* Check of the bounded device waits that every kernel of the library relies
+ * on (no reference passage: robustness of this implementation). Launches one
+ * CTA on `stream` whose two warps wait on a shared-memory barrier that
+ * nothing completes: warp 0 gives up after limit_ns nanoseconds, raises the
+ * CTA's abort flag and records SA_ERR_DEVICE_TIMEOUT in a device status
+ * word; warp 1 waits with a 20x longer limit but leaves as soon as it sees
+ * the abort flag. Synchronises `stream`, then stores the two warps' waiting
+ * times (ns) to waited_ns[0..1] (host array, may be NULL) and returns
+ * SA_ERR_DEVICE_TIMEOUT when the wait expired as designed (the CUDA context
+ * stays usable), SA_OK if the barrier completed, SA_ERR_INVALID_ARG for
+ * limit_ns outside [1e5, 1e10] (0.1 ms .. 10 s), SA_ERR_CUDA on a CUDA
+ * error. No fault, trap or unbounded wait is involved. */
+sa_status sa_wait_probe(uint64_t limit_ns, int64_t* waited_ns, sa_stream_t stream);
 
 /* Thread-local text of the last error; never NULL. */
 const char* sa_last_error_string(void);

@@ -17,6 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
 Q, K, V = 0, 1, 2
+SINK_UPDATE_CHUNK0 = 1 << 40  # chunk coordinate base of sink-update blocks (sa_inputgen.h)
 F32, BF16 = 0, 1
 
 
@@ -88,13 +89,21 @@ def fill_host_f32(w: Workload, stream: int, chunk: int, tensor: int, **kw) -> np
     return bf16_bits_to_f32(a) if a.dtype == np.uint16 else a
 
 
-def fill_device(w: Workload, stream_ids, chunks, tensor: int, out_ptr: int, cuda_stream: int):
-    """Fill a device buffer [len(chunks), Lc, H, D]; chunks[i] < 0 skips slot i."""
+def sink_update_chunk(u: int) -> int:
+    """Chunk coordinate of the sink-update block applied before chunk u."""
+    return SINK_UPDATE_CHUNK0 + u
+
+
+def fill_device(w: Workload, stream_ids, chunks, tensor: int, out_ptr: int, cuda_stream: int,
+                n_tok: int | None = None):
+    """Fill a device buffer [len(chunks), n_tok, H, D] (n_tok defaults to Lc);
+    chunks[i] < 0 skips slot i."""
     n = len(chunks)
     sids = (ctypes.c_int64 * n)(*stream_ids)
     chs = (ctypes.c_int64 * n)(*chunks)
     sp = spec_for(w)
-    rc = lib().ig_fill_device(ctypes.byref(sp), n, sids, chs, tensor, w.Lc, w.H, w.D,
+    rc = lib().ig_fill_device(ctypes.byref(sp), n, sids, chs, tensor,
+                              w.Lc if n_tok is None else n_tok, w.H, w.D,
                               dtype_code(w), ctypes.c_void_p(out_ptr), ctypes.c_void_p(cuda_stream))
     if rc != 0:
         raise RuntimeError(f"ig_fill_device failed ({rc})")

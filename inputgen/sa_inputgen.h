@@ -53,6 +53,11 @@ typedef struct {
 
 #define IG_GOLDEN 0x9E3779B97F4A7C15ULL
 
+/* Chunk coordinate of the sink-update blocks: the [S*F][H][D] keys (IG_K) and
+ * values (IG_V) of the sink update applied before chunk u are drawn at chunk
+ * coordinate IG_SINK_UPDATE_CHUNK0 + u, far from every real chunk index. */
+#define IG_SINK_UPDATE_CHUNK0 (1LL << 40)
+
 IG_FN uint64_t ig_mix64(uint64_t z) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
   z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;

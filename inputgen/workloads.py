@@ -46,6 +46,9 @@ class Workload:
     rope_base: float = 10000.0
     refresh_period: int = 0  # chunks; 0 = never
     starts: Tuple[int, ...] = field(default_factory=tuple)  # global start step per stream
+    sink_repin: bool = False  # after a refresh the sink sits right before the window
+    sink_update_period: int = 0  # sink update before chunk u (u > 0, u % period == 0); 0 = never
+    sink_alpha: float = 1.0  # weight of the new sink data (1 = replace)
 
     @property
     def F(self) -> int:

@@ -27,7 +27,8 @@ class Cfg(ctypes.Structure):
         ("W", ctypes.c_int32), ("rope_dims", ctypes.c_int32 * 3),
         ("rope_base", ctypes.c_double), ("scale", ctypes.c_double),
         ("refresh_period", ctypes.c_int64), ("store", ctypes.c_int32),
-        ("in_dtype", ctypes.c_int32),
+        ("in_dtype", ctypes.c_int32), ("sink_repin", ctypes.c_int32), ("pad_", ctypes.c_int32),
+        ("sink_update_period", ctypes.c_int64), ("sink_alpha", ctypes.c_double),
     ]
 
 
@@ -62,6 +63,9 @@ def lib():
             "orc_cache_contents": ([C, S, i64, i64, _D, _D, _D], i32),
             "orc_attend_rows": ([C, S, i64, i64, i32, _D, _D, _D], i32),
             "orc_bruteforce_rows": ([C, S, i64, i64, i32, _D, _D, _D], i32),
+            "orc_attend_rows_uncommitted": ([C, S, S, i64, i64, i32, _D, _D, _D], i32),
+            "orc_sink_pos": ([C, i64, i64], ctypes.c_double),
+            "orc_sink_raw": ([C, S, i64, i64, i64, i32, _D], i32),
             "orc_num_threads": ([], i32),
         }
         for name, (args, res) in sig.items():
@@ -86,6 +90,9 @@ def cfg_for(w: Workload, store: int | None = None, refresh_period: int | None = 
         store = STORE_BF16 if w.dtype == "bf16" else STORE_F32
     c.store = store
     c.in_dtype = 1 if w.dtype == "bf16" else 0
+    c.sink_repin = 1 if w.sink_repin else 0
+    c.sink_update_period = w.sink_update_period
+    c.sink_alpha = w.sink_alpha
     return c
 
 
@@ -196,6 +203,34 @@ def _rows(fn, cfg, spec, stream, c, toks, heads):
 def attend_rows(cfg: Cfg, spec: Spec, stream: int, c: int, toks, heads) -> np.ndarray:
     """Cache-path attention output rows (tok, head) of chunk c: [n, D] fp64."""
     return _rows(lib().orc_attend_rows, cfg, spec, stream, c, toks, heads)
+
+
+def sink_pos(cfg: Cfg, f: int, c: int) -> float:
+    """Temporal position of sink frame f while chunk c is processed."""
+    return lib().orc_sink_pos(ctypes.byref(cfg), f, c)
+
+
+def sink_raw(cfg: Cfg, spec: Spec, stream: int, f: int, c: int, tensor: int) -> np.ndarray:
+    """Raw key (tensor K) or value (V) of sink frame f at chunk c, [F, H, D]."""
+    out = np.empty((cfg.fh * cfg.fw, cfg.H, cfg.D), dtype=np.float64)
+    _check(lib().orc_sink_raw(ctypes.byref(cfg), ctypes.byref(spec), stream, f, c, tensor,
+                              _ptr(out)), "orc_sink_raw")
+    return out
+
+
+def attend_rows_uncommitted(cfg: Cfg, spec_cache: Spec, spec_chunk: Spec, stream: int, c: int,
+                            toks, heads) -> np.ndarray:
+    """Rows of chunk c attended with uncommitted inputs: frames before the
+    chunk from spec_cache, the chunk's queries, keys and values from
+    spec_chunk. [n, D] fp64."""
+    toks = np.ascontiguousarray(toks, dtype=np.int32)
+    heads = np.ascontiguousarray(heads, dtype=np.int32)
+    assert toks.shape == heads.shape and toks.ndim == 1
+    out = np.empty((len(toks), cfg.D), dtype=np.float64)
+    _check(lib().orc_attend_rows_uncommitted(
+        ctypes.byref(cfg), ctypes.byref(spec_cache), ctypes.byref(spec_chunk), stream, c,
+        len(toks), _ptr(toks), _ptr(heads), _ptr(out)), "orc_attend_rows_uncommitted")
+    return out
 
 
 def bruteforce_rows(cfg: Cfg, spec: Spec, stream: int, c: int, toks, heads) -> np.ndarray:

@@ -187,6 +187,51 @@ int32_t orc_input_block(const orc_cfg* g, const ig_spec* sp, int64_t stream, int
 }
 
 /* ---------------------------------------------------------------------------
+ * Sink (StreamDiffusionV2, technical summary, section 2.A.2: sink tokens are
+ * updated adaptively; RoPE offsets are reset at block boundaries).
+ * Temporal position of sink frame f while chunk c is processed:
+ *   shift : f - base(c)  (the sink moves with every rebase; scores invariant)
+ *   repin : f - min(base(c), S)  -- before the first refresh base(c) = 0 and
+ *           the sink is at its own frame index; a refresh sets base >= S and
+ *           the sink then sits immediately before the oldest window frame,
+ *           which the refresh puts at t = 0.
+ * ------------------------------------------------------------------------- */
+double orc_sink_pos(const orc_cfg* g, int64_t f, int64_t c) {
+  int64_t base = orc_base_at(g, c);
+  if (g->sink_repin && base > g->S) base = g->S;
+  return (double)(f - base);
+}
+
+static int sink_update_due(const orc_cfg* g, int64_t u) {
+  return g->sink_update_period > 0 && u > 0 && u % g->sink_update_period == 0 &&
+         u * g->C >= g->S;
+}
+
+/* Raw (unrotated) key (IG_K) or value (IG_V) of sink frame f, [F][H][D], as
+ * held while chunk c is processed: the frame's input, then for every update
+ * before a chunk u in (0, c] in order
+ *   raw <- round((1 - alpha) * raw + alpha * new),
+ * new = frame f's rows of the update block drawn at chunk coordinate
+ * IG_SINK_UPDATE_CHUNK0 + u (rounding to the storage type; none when exact). */
+int32_t orc_sink_raw(const orc_cfg* g, const ig_spec* sp, int64_t stream, int64_t f,
+                     int64_t c, int32_t tensor, double* out) {
+  if (!g || !sp || !out || f < 0 || f >= g->S || (tensor != IG_K && tensor != IG_V)) return -1;
+  const int64_t F = frame_tokens(g), n = F * (int64_t)g->H * g->D;
+  gen_tokens(g, sp, stream, f / g->C, tensor, (f % g->C) * F, F, out);
+  if (g->sink_update_period <= 0) return 0;
+  double* nw = (double*)malloc(sizeof(double) * (size_t)n);
+  if (!nw) return -2;
+  const double a = g->sink_alpha;
+  for (int64_t u = g->sink_update_period; u <= c; u += g->sink_update_period) {
+    if (!sink_update_due(g, u)) continue;
+    gen_tokens(g, sp, stream, IG_SINK_UPDATE_CHUNK0 + u, tensor, f * F, F, nw);
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_round_store(g->store, (1.0 - a) * out[i] + a * nw[i]);
+  }
+  free(nw);
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
  * Stored key of frame f ([F][H][D]) as the cache holds it while chunk c is
  * processed (f must be visible at c).
  *  exact mode : R(f - base(c), y, x) k, no rounding.
@@ -204,11 +249,15 @@ int32_t orc_stored_key_frame(const orc_cfg* g, const ig_spec* sp, int64_t stream
   const int64_t cw = f / g->C;
   double* raw = (double*)malloc(sizeof(double) * (size_t)(F * H * D));
   if (!raw) return -2;
-  gen_tokens(g, sp, stream, cw, IG_K, (f % g->C) * F, F, raw);
-
   const int exact = g->store == ORC_EXACT;
   const int is_sink = f < g->S;
-  const int64_t base_rot = (exact || is_sink) ? orc_base_at(g, c) : orc_base_at(g, cw);
+  if (is_sink) {
+    if (orc_sink_raw(g, sp, stream, f, c, IG_K, raw) != 0) { free(raw); return -2; }
+  } else {
+    gen_tokens(g, sp, stream, cw, IG_K, (f % g->C) * F, F, raw);
+  }
+  const double pos = is_sink ? orc_sink_pos(g, f, c)
+                             : (double)(f - (exact ? orc_base_at(g, c) : orc_base_at(g, cw)));
   /* refreshes that re-rotate this stored ring key: r in (cw, c] */
   int64_t deltas[4096];
   int n_ref = 0;
@@ -225,7 +274,7 @@ int32_t orc_stored_key_frame(const orc_cfg* g, const ig_spec* sp, int64_t stream
     const double* kin = raw + th * D;
     double* ko = out + th * D;
     double tmp[512];
-    orc_rope_vec(g, kin, (double)(f - base_rot), y, x, tmp);
+    orc_rope_vec(g, kin, pos, y, x, tmp);
     for (int d = 0; d < D; ++d) ko[d] = orc_round_store(g->store, tmp[d]);
     for (int i = 0; i < n_ref; ++i) {
       orc_rope_tband(g, ko, -(double)deltas[i], tmp);
@@ -277,7 +326,10 @@ int32_t orc_cache_contents(const orc_cfg* g, const ig_spec* sp, int64_t stream, 
     const int64_t f = slot_frame[s];
     if (f < 0) continue;
     orc_stored_key_frame(g, sp, stream, f, c, kf);
-    gen_tokens(g, sp, stream, f / g->C, IG_V, (f % g->C) * F, F, vf);
+    if (f < g->S)
+      orc_sink_raw(g, sp, stream, f, c, IG_V, vf);
+    else
+      gen_tokens(g, sp, stream, f / g->C, IG_V, (f % g->C) * F, F, vf);
     for (int64_t j = 0; j < F; ++j)
       for (int h = 0; h < H; ++h)
         for (int d = 0; d < D; ++d) {
@@ -319,10 +371,16 @@ static void attend_one(const double* q, const double* keys, const double* vals, 
  * are the visible frames as stored in the cache (sink, then window, then the
  * current chunk); queries are rotated with the same base.
  * ------------------------------------------------------------------------- */
-int32_t orc_attend_rows(const orc_cfg* g, const ig_spec* sp, int64_t stream, int64_t c,
-                        int32_t n_rows, const int32_t* toks, const int32_t* heads,
-                        double* out) {
-  if (!g || !sp || !out || n_rows < 0 || (n_rows > 0 && (!toks || !heads))) return -1;
+/* Rows of the cache-path attention of chunk c. Frames before the chunk are
+ * stored keys / values drawn from sp_past; the chunk's own frames (keys,
+ * values) and its queries are drawn from sp_chunk. With sp_past == sp_chunk
+ * this is the committed path; otherwise the chunk is attended with inputs
+ * that the cache never keeps. */
+static int32_t attend_rows_two(const orc_cfg* g, const ig_spec* sp_past, const ig_spec* sp_chunk,
+                               int64_t stream, int64_t c, int32_t n_rows, const int32_t* toks,
+                               const int32_t* heads, double* out) {
+  if (!g || !sp_past || !sp_chunk || !out || n_rows < 0 || (n_rows > 0 && (!toks || !heads)))
+    return -1;
   const int64_t F = frame_tokens(g), Lc = (int64_t)g->C * F;
   const int H = g->H, D = g->D;
   if (D > 512) return -1;
@@ -345,8 +403,12 @@ int32_t orc_attend_rows(const orc_cfg* g, const ig_spec* sp, int64_t stream, int
   int64_t kpos = 0;
   for (int64_t f = 0; f < (c + 1) * g->C; ++f) {
     if (!orc_visible(g, c, f)) continue;
+    const ig_spec* sp = f < c * g->C ? sp_past : sp_chunk;
     orc_stored_key_frame(g, sp, stream, f, c, kf);
-    gen_tokens(g, sp, stream, f / g->C, IG_V, (f % g->C) * F, F, vf);
+    if (f < g->S)
+      orc_sink_raw(g, sp, stream, f, c, IG_V, vf);
+    else
+      gen_tokens(g, sp, stream, f / g->C, IG_V, (f % g->C) * F, F, vf);
     for (int64_t j = 0; j < F; ++j)
       for (int h = 0; h < H; ++h)
         for (int d = 0; d < D; ++d) {
@@ -355,7 +417,7 @@ int32_t orc_attend_rows(const orc_cfg* g, const ig_spec* sp, int64_t stream, int
         }
     kpos += F;
   }
-  orc_query_rot(g, sp, stream, c, qr);
+  orc_query_rot(g, sp_chunk, stream, c, qr);
   const double scale = softmax_scale(g);
 #pragma omp parallel for schedule(dynamic, 1)
   for (int32_t r = 0; r < n_rows; ++r) {
@@ -365,6 +427,25 @@ int32_t orc_attend_rows(const orc_cfg* g, const ig_spec* sp, int64_t stream, int
   }
   free(K); free(V); free(kf); free(vf); free(qr);
   return 0;
+}
+
+int32_t orc_attend_rows(const orc_cfg* g, const ig_spec* sp, int64_t stream, int64_t c,
+                        int32_t n_rows, const int32_t* toks, const int32_t* heads,
+                        double* out) {
+  return attend_rows_two(g, sp, sp, stream, c, n_rows, toks, heads, out);
+}
+
+/* Attention of chunk c over the committed context (frames before the chunk,
+ * drawn from sp_cache) and an uncommitted chunk (queries, keys and values of
+ * the chunk's frames drawn from sp_chunk). StreamDiffusionV2 (technical
+ * summary, section 2.B.2 "Stream-Batch"): every denoising step of a chunk is
+ * a forward pass over the same cached context with that step's latents;
+ * only the final step's keys and values are kept. */
+int32_t orc_attend_rows_uncommitted(const orc_cfg* g, const ig_spec* sp_cache,
+                                    const ig_spec* sp_chunk, int64_t stream, int64_t c,
+                                    int32_t n_rows, const int32_t* toks, const int32_t* heads,
+                                    double* out) {
+  return attend_rows_two(g, sp_cache, sp_chunk, stream, c, n_rows, toks, heads, out);
 }
 
 /* ---------------------------------------------------------------------------

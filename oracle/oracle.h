@@ -46,6 +46,13 @@ typedef struct {
   int64_t refresh_period; /* refresh before chunk c when c>0 and c % period == 0; 0 = never */
   int32_t store;          /* ORC_EXACT, ORC_STORE_F32 or ORC_STORE_BF16 */
   int32_t in_dtype;       /* IG_F32 or IG_BF16: how the generated inputs are stored */
+  int32_t sink_repin;     /* 0: the sink's positions rebase with the rest (shift);
+                             1: after a refresh the sink sits right before the
+                             oldest window frame (t = f - S) */
+  int32_t pad_;
+  int64_t sink_update_period; /* sink update before chunk u when u > 0, u % period == 0
+                                 and the sink is complete (uC >= S); 0 = never */
+  double sink_alpha;      /* weight of the new sink data in the update (1 = replace) */
 } orc_cfg;
 
 double orc_round_store(int32_t store, double x);
@@ -65,6 +72,9 @@ int64_t orc_n_keys(const orc_cfg* cfg, int64_t c);
 
 int32_t orc_input_block(const orc_cfg* cfg, const ig_spec* sp, int64_t stream, int64_t chunk,
                         int32_t tensor, double* out);
+double orc_sink_pos(const orc_cfg* cfg, int64_t f, int64_t c);
+int32_t orc_sink_raw(const orc_cfg* cfg, const ig_spec* sp, int64_t stream, int64_t f,
+                     int64_t c, int32_t tensor, double* out);
 int32_t orc_stored_key_frame(const orc_cfg* cfg, const ig_spec* sp, int64_t stream,
                              int64_t f, int64_t c, double* out);
 int32_t orc_query_rot(const orc_cfg* cfg, const ig_spec* sp, int64_t stream, int64_t c,
@@ -74,6 +84,10 @@ int32_t orc_cache_contents(const orc_cfg* cfg, const ig_spec* sp, int64_t stream
 int32_t orc_attend_rows(const orc_cfg* cfg, const ig_spec* sp, int64_t stream, int64_t c,
                         int32_t n_rows, const int32_t* toks, const int32_t* heads,
                         double* out);
+int32_t orc_attend_rows_uncommitted(const orc_cfg* cfg, const ig_spec* sp_cache,
+                                    const ig_spec* sp_chunk, int64_t stream, int64_t c,
+                                    int32_t n_rows, const int32_t* toks, const int32_t* heads,
+                                    double* out);
 int32_t orc_bruteforce_rows(const orc_cfg* cfg, const ig_spec* sp, int64_t stream,
                             int64_t c, int32_t n_rows, const int32_t* toks,
                             const int32_t* heads, double* out);

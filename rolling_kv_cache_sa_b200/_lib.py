@@ -12,6 +12,7 @@ SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_OOM, SA_ERR_CUDA, SA_ERR_S
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_OOM",
                 4: "SA_ERR_CUDA", 5: "SA_ERR_STATE", 6: "SA_ERR_DEVICE_TIMEOUT"}
 SA_F32, SA_BF16 = 0, 1
+SA_SINK_SHIFT, SA_SINK_REPIN = 0, 1
 SA_MAX_CHUNK_FRAMES = 32
 
 # every symbol include/sa.h declares
@@ -20,7 +21,8 @@ EXPORTED = (
     "sa_cache_destroy", "sa_append_attend_host", "sa_stream_state", "sa_cache_copy_out",
     "sa_get_device_status", "sa_plan_chunk", "sa_refresh_delta", "sa_profile_begin",
     "sa_profile_end", "sa_last_error_string", "sa_abi_version", "sa_append_attend_noalloc",
-    "sa_profile_launches",
+    "sa_profile_launches", "sa_wait_probe", "sa_attend", "sa_cache_set_sink_mode",
+    "sa_sink_update",
 )
 
 
@@ -68,6 +70,9 @@ def lib() -> ctypes.CDLL:
     sig = {
         "sa_cache_create": [P(sa_config), vp, P(vp)],
         "sa_append_attend": [vp, vp, vp, vp, vp, vp, vp],
+        "sa_attend": [vp, vp, vp, vp, vp, vp, vp],
+        "sa_cache_set_sink_mode": [vp, i32],
+        "sa_sink_update": [vp, vp, vp, ctypes.c_float, vp, vp],
         "sa_rope_refresh": [vp, vp, vp],
         "sa_cache_reset": [vp, vp],
         "sa_cache_destroy": [vp],
@@ -79,6 +84,7 @@ def lib() -> ctypes.CDLL:
         "sa_refresh_delta": [P(sa_config), i64, i64, P(i64)],
         "sa_profile_begin": [vp],
         "sa_profile_launches": [vp, P(i64)],
+        "sa_wait_probe": [ctypes.c_uint64, P(i64), vp],
         "sa_append_attend_noalloc": [P(sa_config), vp, vp, vp, P(i64), P(i64), vp, vp, vp, vp,
                                      vp, vp],
         "sa_profile_end": [vp, P(ctypes.c_double), P(i32), P(ctypes.c_double), P(i32),

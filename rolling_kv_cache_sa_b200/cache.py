@@ -61,6 +61,23 @@ def sa_append_attend(h: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
           "sa_append_attend")
 
 
+def sa_attend(h: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+              active=None, stream: Optional[torch.cuda.Stream] = None, batch: int = 0):
+    check(lib().sa_attend(h, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          _mask(active, batch or q.shape[0]), _stream_ptr(stream)), "sa_attend")
+
+
+def sa_cache_set_sink_mode(h: int, mode: int):
+    check(lib().sa_cache_set_sink_mode(h, mode), "sa_cache_set_sink_mode")
+
+
+def sa_sink_update(h: int, k_new: torch.Tensor, v_new: torch.Tensor, alpha: float, active=None,
+                   stream: Optional[torch.cuda.Stream] = None, batch: int = 0):
+    check(lib().sa_sink_update(h, k_new.data_ptr(), v_new.data_ptr(), ctypes.c_float(alpha),
+                               _mask(active, batch or k_new.shape[0]), _stream_ptr(stream)),
+          "sa_sink_update")
+
+
 def sa_rope_refresh(h: int, active=None, batch: int = 0,
                     stream: Optional[torch.cuda.Stream] = None):
     check(lib().sa_rope_refresh(h, _mask(active, batch), _stream_ptr(stream)), "sa_rope_refresh")
@@ -148,6 +165,14 @@ def sa_append_attend_noalloc(cfg: sa_config, k_cache: torch.Tensor, v_cache: tor
         _stream_ptr(stream)), "sa_append_attend_noalloc")
 
 
+def sa_wait_probe(limit_ns: int, stream: Optional[torch.cuda.Stream] = None):
+    """Runs the bounded-wait check; returns (status, [waited_ns warp0, warp1])
+    without raising (SA_ERR_DEVICE_TIMEOUT is the designed outcome)."""
+    w = (ctypes.c_int64 * 2)()
+    st = lib().sa_wait_probe(ctypes.c_uint64(limit_ns), w, ctypes.c_void_p(_stream_ptr(stream)))
+    return st, [w[0], w[1]]
+
+
 def sa_abi_version() -> int:
     return lib().sa_abi_version()
 
@@ -177,6 +202,25 @@ class SACache:
         for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
             self._check_tensor(t, n)
         sa_append_attend(self.h, q, k, v, out, active, stream, self.B)
+
+    def attend(self, q, k, v, out, active=None, stream=None):
+        """Attention of the next chunk without committing it (a denoising step
+        that is not the chunk's last)."""
+        for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+            self._check_tensor(t, n)
+        sa_attend(self.h, q, k, v, out, active, stream, self.B)
+
+    def set_sink_mode(self, mode: int):
+        sa_cache_set_sink_mode(self.h, mode)
+
+    def sink_update(self, k_new, v_new, alpha: float = 1.0, active=None, stream=None):
+        """Blends new data into the sink (k_new, v_new: [B, S*F, H, D])."""
+        shape = (self.B, self.cfg.sink_frames * self.F, self.H, self.D)
+        for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+            if t.device != self.device or t.dtype != self.dtype or not t.is_contiguous() or \
+                    tuple(t.shape) != shape:
+                raise ValueError(f"{n} must be a contiguous {self.dtype} tensor of shape {shape}")
+        sa_sink_update(self.h, k_new, v_new, alpha, active, stream, self.B)
 
     def append_attend_host(self, q, k, v, out, active=None, stream=None):
         sa_append_attend_host(self.h, q, k, v, out, active, stream)

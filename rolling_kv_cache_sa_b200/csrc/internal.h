@@ -43,7 +43,15 @@ struct AppendParams {
 // re-derived from raw keys at their new positions.
 struct RefreshParams {
   void* k_cache;
-  const void* k_raw;
+  void* k_raw;
+  // sink update (update != 0): raw sink keys and sink values become
+  // (1 - alpha) * old + alpha * new before the sink keys are re-derived;
+  // k_new / v_new are [B][S*F][H][D]; ring_rows must be 0
+  void* v_cache;
+  const void* k_new;
+  const void* v_new;
+  float alpha;
+  int32_t update;
   const float2* htab;
   const float2* wtab;
   int32_t H, D, fw, F, S;
@@ -83,6 +91,10 @@ struct AttnParams {
 size_t attend_partials_bytes(int D, int num_sms, int64_t max_units);
 
 cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStream_t st);
+// Bounded-wait check (wait_probe.cu); synchronises `st` and returns the
+// device status word and the two warps' waiting times.
+cudaError_t run_wait_probe(uint64_t limit_ns, cudaStream_t st, int* status,
+                           unsigned long long waited_ns[2]);
 cudaError_t launch_refresh(const RefreshParams& p, int dtype, int num_sms, cudaStream_t st);
 cudaError_t launch_attend_simt_f32(const AttnParams& p, int D, cudaStream_t st);
 // bf16 tensor-core attention. `partials` (attend_partials_bytes) lets the

@@ -39,6 +39,7 @@ struct Vec16<float> {
   __device__ __forceinline__ static void copy(void* dst, const void* src) {
     *reinterpret_cast<float4*>(dst) = __ldg(reinterpret_cast<const float4*>(src));
   }
+  __device__ __forceinline__ static void round(float (&)[4]) {}
 };
 
 template <>
@@ -69,6 +70,11 @@ struct Vec16<__nv_bfloat16> {
   }
   __device__ __forceinline__ static void copy(void* dst, const void* src) {
     *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+  }
+  // the value a store followed by a load gives (round to nearest even)
+  __device__ __forceinline__ static void round(float (&x)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
   }
 };
 
@@ -139,7 +145,9 @@ __global__ void __launch_bounds__(256) append_rope_kernel(const __grid_constant_
 
 // grid.y = stream of the launch. Ring part: only the vectors that hold
 // temporal-band pairs are read and written. Sink part: every vector of the
-// valid sink rows is re-derived from the raw keys.
+// valid sink rows is re-derived from the raw keys; in update mode the raw
+// keys and the sink values are first blended with the new sink data
+// (StreamDiffusionV2, section 2.A.2: adaptive sink tokens).
 template <typename T>
 __global__ void __launch_bounds__(256) refresh_kernel(const __grid_constant__ RefreshParams p) {
   using V = Vec16<T>;
@@ -180,7 +188,26 @@ __global__ void __launch_bounds__(256) refresh_kernel(const __grid_constant__ Re
       const int j = (int)(rr - (int64_t)s * p.F);
       const int y = j / p.fw, x = j - (j / p.fw) * p.fw;
       float k[N];
-      V::load(static_cast<const char*>(p.k_raw) + ((bh * p.sf + rr) * p.D + vc * N) * esz, k);
+      char* raw = static_cast<char*>(p.k_raw) + ((bh * p.sf + rr) * p.D + vc * N) * esz;
+      V::load_cache(raw, k);
+      if (p.update) {
+        // adaptive sink update: blend raw keys and values, round to storage
+        const int64_t in_off = (((int64_t)b * p.S * p.F + rr) * p.H + h) * p.D + vc * N;
+        char* vp = static_cast<char*>(p.v_cache) + ((bh * p.ntok + rr) * p.D + vc * N) * esz;
+        float kn[N], v[N], vn[N];
+        V::load(static_cast<const char*>(p.k_new) + in_off * esz, kn);
+        V::load_cache(vp, v);
+        V::load(static_cast<const char*>(p.v_new) + in_off * esz, vn);
+        const float a = p.alpha, am = 1.f - p.alpha;
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+          k[e] = am * k[e] + a * kn[e];
+          v[e] = am * v[e] + a * vn[e];
+        }
+        V::store(raw, k);
+        V::store(vp, v);
+        V::round(k);  // the rotation starts from the stored raw key
+      }
 #pragma unroll
       for (int pp = 0; pp < N / 2; ++pp) {
         const int pi = (int)vc * (N / 2) + pp;

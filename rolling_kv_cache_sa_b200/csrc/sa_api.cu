@@ -163,6 +163,7 @@ struct sa_cache {
   void* k_cache = nullptr;
   void* v_cache = nullptr;
   void* k_raw = nullptr;
+  int32_t sink_mode = SA_SINK_SHIFT;  // how the sink's positions follow a refresh
   void* q_ws = nullptr;
   float2* htab = nullptr;
   float2* wtab = nullptr;
@@ -173,6 +174,13 @@ struct sa_cache {
   CUtensorMap tm_q, tm_k, tm_v;
   // host-buffer staging (allocated by the first sa_append_attend_host)
   void* stage[4] = {nullptr, nullptr, nullptr, nullptr};
+  // pipelined host path (sa_append_attend_host_async): staging slots of
+  // q, k, v, out, two copy streams and per-slot events
+  static constexpr int kSlots = 3;
+  void* slot_buf[kSlots][4] = {};
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t in_done[kSlots] = {}, comp_done[kSlots] = {}, out_done[kSlots] = {};
+  int64_t async_calls = 0;
   // profiling
   bool profiling = false;
   std::vector<cudaEvent_t> ev;
@@ -182,6 +190,15 @@ struct sa_cache {
 };
 
 namespace {
+
+// Base that the sink's temporal positions are taken against: t = f - base.
+// Shift: the stream's base (the sink moves with every rebase). Re-pin: a
+// refresh sets base >= S and the sink then sits right before the oldest
+// window frame (t = f - S); before the first refresh base = 0.
+int64_t sink_base(const sa_cache* h, int64_t base) {
+  if (h->sink_mode == SA_SINK_REPIN && base > h->cfg.sink_frames) return h->cfg.sink_frames;
+  return base;
+}
 
 // A record into a capturing stream is made an external event node, so the event
 // still carries a time after each replay; the external flag is refused outside
@@ -207,10 +224,20 @@ void prof_after(sa_cache* h, cudaStream_t st) {
 }
 
 void free_all(sa_cache* h) {
+  if (h->copy_in) cudaStreamSynchronize(h->copy_in);
+  if (h->copy_out) cudaStreamSynchronize(h->copy_out);
   void* ptrs[] = {h->k_cache, h->v_cache, h->k_raw, h->q_ws, h->htab, h->wtab, h->d_status,
                   h->partials, h->stage[0], h->stage[1], h->stage[2], h->stage[3]};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  for (int s = 0; s < sa_cache::kSlots; ++s) {
+    for (int t = 0; t < 4; ++t)
+      if (h->slot_buf[s][t]) cudaFree(h->slot_buf[s][t]);
+    for (cudaEvent_t e : {h->in_done[s], h->comp_done[s], h->out_done[s]})
+      if (e) cudaEventDestroy(e);
+  }
+  if (h->copy_in) cudaStreamDestroy(h->copy_in);
+  if (h->copy_out) cudaStreamDestroy(h->copy_out);
   for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
 }
 
@@ -228,6 +255,32 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 extern "C" {
 
 int32_t sa_abi_version(void) { return SA_ABI_VERSION; }
+
+sa_status sa_wait_probe(uint64_t limit_ns, int64_t* waited_ns, sa_stream_t stream) {
+  if (limit_ns < 100000ull || limit_ns > 10000000000ull)
+    return fail(SA_ERR_INVALID_ARG, "limit_ns %llu outside [1e5, 1e10]",
+                (unsigned long long)limit_ns);
+  int dev = 0;
+  cudaDeviceProp prop;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return fail(SA_ERR_UNSUPPORTED, "no CUDA device: %s", cudaGetErrorString(e));
+  if (prop.major != 10)
+    return fail(SA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100a (B200)",
+                dev, prop.major, prop.minor);
+  int status = 0;
+  unsigned long long w[2] = {0, 0};
+  e = sa::run_wait_probe(limit_ns, static_cast<cudaStream_t>(stream), &status, w);
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe");
+  if (waited_ns) {
+    waited_ns[0] = (int64_t)w[0];
+    waited_ns[1] = (int64_t)w[1];
+  }
+  if (status & sa::kDeviceErrTimeout)
+    return fail(SA_ERR_DEVICE_TIMEOUT, "device wait expired after %llu ns (as designed)",
+                (unsigned long long)w[0]);
+  return SA_OK;
+}
 
 const char* sa_last_error_string(void) { return g_last_error.c_str(); }
 
@@ -377,8 +430,12 @@ sa_status sa_cache_reset(sa_cache* h, const uint8_t* streams) {
   return SA_OK;
 }
 
-sa_status sa_append_attend(sa_cache* h, const void* q, const void* k, const void* v, void* out,
-                           const uint8_t* active, sa_stream_t stream) {
+namespace {
+// RoPE + append of the next chunk, then attention; `commit` advances the
+// streams' frame counts (sa_append_attend), otherwise the chunk's rows are
+// rewritten by the next call (sa_attend).
+sa_status append_attend(sa_cache* h, const void* q, const void* k, const void* v, void* out,
+                        const uint8_t* active, sa_stream_t stream, bool commit) {
   if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
   if (!q || !k || !v || !out) return fail(SA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -455,8 +512,20 @@ sa_status sa_append_attend(sa_cache* h, const void* q, const void* k, const void
   prof_after(h, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   h->kernels += n_att;
-  for (int b : act) h->frames_written[b] += C;
+  if (commit)
+    for (int b : act) h->frames_written[b] += C;
   return SA_OK;
+}
+}  // namespace
+
+sa_status sa_append_attend(sa_cache* h, const void* q, const void* k, const void* v, void* out,
+                           const uint8_t* active, sa_stream_t stream) {
+  return append_attend(h, q, k, v, out, active, stream, true);
+}
+
+sa_status sa_attend(sa_cache* h, const void* q, const void* k, const void* v, void* out,
+                    const uint8_t* active, sa_stream_t stream) {
+  return append_attend(h, q, k, v, out, active, stream, false);
 }
 
 sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream) {
@@ -496,9 +565,10 @@ sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream
         const double ang = -(double)deltas[s0 + a] * theta(&c, 0, j);
         p.dcs[a][j] = make_float2((float)cos(ang), (float)sin(ang));
       }
+      const int64_t sb = sink_base(h, new_base);
       for (int s = 0; s < S; ++s)
         for (int j = 0; j < dt2; ++j) {
-          const double ang = (double)(s - new_base) * theta(&c, 0, j);
+          const double ang = (double)(s - sb) * theta(&c, 0, j);
           p.scs[a * S + s][j] = make_float2((float)cos(ang), (float)sin(ang));
         }
     }
@@ -509,6 +579,66 @@ sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream
     h->kernels += 1;
   }
   for (size_t i = 0; i < todo.size(); ++i) h->pos_base[todo[i]] += deltas[i];
+  return SA_OK;
+}
+
+sa_status sa_cache_set_sink_mode(sa_cache* h, int32_t mode) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (mode != SA_SINK_SHIFT && mode != SA_SINK_REPIN)
+    return fail(SA_ERR_INVALID_ARG, "sink mode %d is not SA_SINK_SHIFT or SA_SINK_REPIN", mode);
+  h->sink_mode = mode;
+  return SA_OK;
+}
+
+sa_status sa_sink_update(sa_cache* h, const void* k_new, const void* v_new, float alpha,
+                         const uint8_t* active, sa_stream_t stream) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  const sa_config& c = h->cfg;
+  const int S = c.sink_frames, dt2 = c.rope_dims[0] / 2;
+  if (S <= 0) return fail(SA_ERR_INVALID_ARG, "the cache has no sink (sink_frames = 0)");
+  if (!k_new || !v_new) return fail(SA_ERR_INVALID_ARG, "k_new and v_new must be non-NULL");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    return fail(SA_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+  if (!(alpha >= 0.f && alpha <= 1.f)) return fail(SA_ERR_INVALID_ARG, "alpha must be in [0, 1]");
+  if (S > sa::kMaxRefresh)
+    return fail(SA_ERR_UNSUPPORTED, "sink update supports at most %d sink frames", sa::kMaxRefresh);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<int> act;
+  active_list(h, active, act);
+  for (int b : act)
+    if (h->frames_written[b] < S)
+      return fail(SA_ERR_STATE, "stream %d: the sink is not complete (%lld of %d frames)", b,
+                  (long long)h->frames_written[b], S);
+  if (act.empty()) return SA_OK;
+  const int per_launch = std::max(1, sa::kMaxRefresh / S);
+  for (size_t s0 = 0; s0 < act.size(); s0 += per_launch) {
+    sa::RefreshParams p;
+    memset(&p, 0, sizeof(p));
+    p.k_cache = h->k_cache; p.k_raw = h->k_raw; p.htab = h->htab; p.wtab = h->wtab;
+    p.v_cache = h->v_cache; p.k_new = k_new; p.v_new = v_new; p.alpha = alpha; p.update = 1;
+    p.H = c.heads; p.D = c.head_dim; p.fw = c.frame_w; p.F = (int32_t)h->F; p.S = S;
+    p.ntok = h->ntok; p.sf = h->sf;
+    p.dt2 = dt2; p.dh2 = c.rope_dims[1] / 2; p.dw2 = c.rope_dims[2] / 2;
+    const size_t n = std::min(act.size() - s0, (size_t)per_launch);
+    p.n_streams = (int32_t)n;
+    for (size_t a = 0; a < n; ++a) {
+      const int b = act[s0 + a];
+      p.stream_of[a] = b;
+      p.sink_rows[a] = (int64_t)S * h->F;
+      p.ring_rows[a] = 0;
+      const int64_t sb = sink_base(h, h->pos_base[b]);
+      for (int s = 0; s < S; ++s)
+        for (int j = 0; j < dt2; ++j) {
+          const double ang = (double)(s - sb) * theta(&c, 0, j);
+          p.scs[a * S + s][j] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+    }
+    prof_before(h, st, KIND_REFRESH);
+    cudaError_t e = sa::launch_refresh(p, c.dtype, h->num_sms, st);
+    prof_after(h, st);
+    if (e != cudaSuccess) return cuda_fail(e, "sink update launch");
+    h->kernels += 1;
+  }
   return SA_OK;
 }
 
@@ -545,6 +675,77 @@ sa_status sa_append_attend_host(sa_cache* h, const void* q, const void* k, const
   }
   cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  return SA_OK;
+}
+
+sa_status sa_append_attend_host_async(sa_cache* h, const void* q, const void* k, const void* v,
+                                      void* out, const uint8_t* active, sa_stream_t stream) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (!q || !k || !v || !out) return fail(SA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t per = (size_t)(h->Lc * h->cfg.heads * h->cfg.head_dim) * h->esz;
+  const size_t total = per * (size_t)h->cfg.batch;
+  cudaError_t e = cudaSuccess;
+  if (!h->copy_in) {  // first call: streams, events and staging slots
+    e = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking);
+    for (int s = 0; s < sa_cache::kSlots && e == cudaSuccess; ++s) {
+      for (cudaEvent_t* ev : {&h->in_done[s], &h->comp_done[s], &h->out_done[s]})
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+      for (int t = 0; t < 4 && e == cudaSuccess; ++t) e = cudaMalloc(&h->slot_buf[s][t], total);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "host pipeline setup");
+  }
+  std::vector<int> act;
+  active_list(h, active, act);
+  if (act.empty()) return SA_OK;
+  // validate the chunk plans before any copy is queued
+  for (int b : act) {
+    sa_chunk_plan pl;
+    sa_status s = plan_chunk(&h->cfg, h->frames_written[b], h->pos_base[b], &pl);
+    if (s != SA_OK) return s;
+  }
+  const int slot = (int)(h->async_calls % sa_cache::kSlots);
+  void** buf = h->slot_buf[slot];
+  // copy-in: the slot's inputs are free once its previous compute finished
+  e = cudaStreamWaitEvent(h->copy_in, h->comp_done[slot], 0);
+  const void* src[3] = {q, k, v};
+  for (int t = 0; t < 3 && e == cudaSuccess; ++t)
+    for (int b : act) {
+      e = cudaMemcpyAsync(static_cast<char*>(buf[t]) + per * b,
+                          static_cast<const char*>(src[t]) + per * b, per,
+                          cudaMemcpyHostToDevice, h->copy_in);
+      if (e != cudaSuccess) break;
+    }
+  if (e == cudaSuccess) e = cudaEventRecord(h->in_done[slot], h->copy_in);
+  // compute on the caller's stream after the inputs landed and after the
+  // slot's previous output left the device
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, h->in_done[slot], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, h->out_done[slot], 0);
+  if (e != cudaSuccess) return cuda_fail(e, "host pipeline copy-in");
+  sa_status s = sa_append_attend(h, buf[0], buf[1], buf[2], buf[3], active, stream);
+  if (s != SA_OK) return s;
+  e = cudaEventRecord(h->comp_done[slot], st);
+  // copy-out once the chunk is computed
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(h->copy_out, h->comp_done[slot], 0);
+  for (int b : act) {
+    if (e != cudaSuccess) break;
+    e = cudaMemcpyAsync(static_cast<char*>(out) + per * b,
+                        static_cast<const char*>(buf[3]) + per * b, per,
+                        cudaMemcpyDeviceToHost, h->copy_out);
+  }
+  if (e == cudaSuccess) e = cudaEventRecord(h->out_done[slot], h->copy_out);
+  if (e != cudaSuccess) return cuda_fail(e, "host pipeline copy-out");
+  ++h->async_calls;
+  return SA_OK;
+}
+
+sa_status sa_host_wait(sa_cache* h) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  cudaError_t e = cudaSuccess;
+  if (h->copy_in) e = cudaStreamSynchronize(h->copy_in);
+  if (e == cudaSuccess && h->copy_out) e = cudaStreamSynchronize(h->copy_out);
+  if (e != cudaSuccess) return cuda_fail(e, "host pipeline wait");
   return SA_OK;
 }
 

@@ -8,7 +8,7 @@ from __future__ import annotations
 
 from typing import Optional, Sequence
 
-from .cache import SACache
+from .cache import SACache, sa_refresh_delta
 
 
 class StreamSession:
@@ -27,8 +27,13 @@ class StreamSession:
         mask = []
         for b in range(self.cache.B):
             on = active is None or bool(active[b])
-            c = self.next_chunk(b)
-            mask.append(on and c > 0 and c % self.period == 0)
+            fw, base = self.cache.state(b)
+            c = fw // self.C
+            # a refresh whose offset is already 0 (the chunk's uncommitted
+            # steps refreshed it) changes nothing and is skipped
+            due = on and c > 0 and c % self.period == 0 and \
+                sa_refresh_delta(self.cache.cfg, fw, base) != 0
+            mask.append(due)
         return mask if any(mask) else None
 
     def step(self, q, k, v, out, active: Optional[Sequence[bool]] = None, stream=None):
@@ -38,6 +43,16 @@ class StreamSession:
         if mask is not None:
             self.cache.rope_refresh(mask, stream)
         self.cache.append_attend(q, k, v, out, active, stream)
+
+    def step_uncommitted(self, q, k, v, out, active: Optional[Sequence[bool]] = None,
+                         stream=None):
+        """A denoising step of the next chunk that is not kept: refresh if due
+        (the chunk's later steps then find nothing to rebase), then attention over the cached context and this
+        step's keys and values without advancing the streams."""
+        mask = self.refresh_mask(active)
+        if mask is not None:
+            self.cache.rope_refresh(mask, stream)
+        self.cache.attend(q, k, v, out, active, stream)
 
     def step_host(self, q, k, v, out, active: Optional[Sequence[bool]] = None, stream=None):
         """Same as step with host tensors (copies inside the call)."""

@@ -68,6 +68,20 @@ def test_state_errors():
     assert b"NULL" in _lib.lib().sa_last_error_string()
 
 
+def test_wait_probe_validates_its_limit():
+    for bad in (0, 99_999, 10_000_000_001):
+        st, _ = S.sa_wait_probe(bad) if torch.cuda.is_available() else \
+            (_lib.lib().sa_wait_probe(ctypes.c_uint64(bad), None, None), None)
+        assert st == _lib.SA_ERR_INVALID_ARG
+    assert b"limit_ns" in _lib.lib().sa_last_error_string()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device refusal")
+def test_wait_probe_without_device_is_refused():
+    assert _lib.lib().sa_wait_probe(ctypes.c_uint64(2_000_000), None, None) == \
+        _lib.SA_ERR_UNSUPPORTED
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device refusal")
 def test_create_without_device_is_refused():
     h = ctypes.c_void_p()

@@ -292,6 +292,152 @@ def test_window_zero_is_sink_plus_self(C, S):
 
 
 # --------------------------------------------------------------------------
+# Uncommitted chunk (a denoising step that is not kept): the committed context
+# from one input draw, the chunk's queries, keys and values from another --
+# assembled by hand from the pinned rotation and attended by torch SDPA
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("C,S,W", [(2, 1, 2), (1, 1, 3), (2, 0, 4)])
+def test_uncommitted_chunk_matches_torch_sdpa(C, S, W):
+    w = TINY.with_(C=C, S=S, W=W)
+    w2 = w.with_(seed=w.seed + 7)
+    cfg = _cfg(w)
+    sp_past, sp_chunk = spec_for(w), spec_for(w2)
+    F, H = w.F, w.H
+    for c in (0, 1, 3, 6):
+        frames = [f for f in range((c + 1) * C) if f < S or f >= c * C - W]
+        ks, vs = [], []
+        for f in frames:
+            sp = sp_past if f < c * C else sp_chunk
+            blk_k = O.input_block(cfg, sp, 0, f // C, K)
+            blk_v = O.input_block(cfg, sp, 0, f // C, V)
+            for j in range(F):
+                i = (f % C) * F + j
+                ks.append([O.rope_vec(cfg, blk_k[i, h], f, j // w.fw, j % w.fw) for h in range(H)])
+                vs.append(blk_v[i])
+        qb = O.input_block(cfg, sp_chunk, 0, c, Q)
+        qs = [[O.rope_vec(cfg, qb[i, h], c * C + i // F, (i % F) // w.fw, (i % F) % w.fw)
+               for h in range(H)] for i in range(w.Lc)]
+        qt = torch.tensor(np.array(qs)).permute(1, 0, 2)[None]
+        kt = torch.tensor(np.array(ks)).permute(1, 0, 2)[None]
+        vt = torch.tensor(np.array(vs)).permute(1, 0, 2)[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).numpy()[0]
+        toks, heads = _all_rows(w)
+        got = O.attend_rows_uncommitted(cfg, sp_past, sp_chunk, 0, c, toks, heads)
+        np.testing.assert_allclose(got, ref[heads, toks], rtol=0, atol=1e-12)
+        # one draw for both reduces to the committed path
+        np.testing.assert_array_equal(O.attend_rows_uncommitted(cfg, sp_past, sp_past, 0, c, toks, heads),
+                                      O.attend_rows(cfg, sp_past, 0, c, toks, heads))
+
+
+# --------------------------------------------------------------------------
+# Sink variants (StreamDiffusionV2 2.A.2): the re-pinned sink and the adaptive
+# sink update, each against torch SDPA over a context assembled by hand from
+# the pinned rotation and the generator's blocks
+# --------------------------------------------------------------------------
+def _sdpa_chunk(w, cfg, sp, c, key_pos, sink_k=None, sink_v=None):
+    """Exact attention of chunk c with keys of frame f rotated at key_pos(f)
+    and the sink frames' raw keys / values optionally replaced."""
+    F, H, C = w.F, w.H, w.C
+    base = O.base_at(cfg, c)
+    frames = [f for f in range((c + 1) * C) if f < w.S or f >= c * C - w.W]
+    ks, vs = [], []
+    for f in frames:
+        blk_k = O.input_block(cfg, sp, 0, f // C, K)
+        blk_v = O.input_block(cfg, sp, 0, f // C, V)
+        for j in range(F):
+            i = (f % C) * F + j
+            kin = sink_k[f][j] if (sink_k is not None and f < w.S) else blk_k[i]
+            vin = sink_v[f][j] if (sink_v is not None and f < w.S) else blk_v[i]
+            ks.append([O.rope_vec(cfg, kin[h], key_pos(f), j // w.fw, j % w.fw) for h in range(H)])
+            vs.append(vin)
+    qb = O.input_block(cfg, sp, 0, c, Q)
+    qs = [[O.rope_vec(cfg, qb[i, h], c * C + i // F - base, (i % F) // w.fw, (i % F) % w.fw)
+           for h in range(H)] for i in range(w.Lc)]
+    qt = torch.tensor(np.array(qs)).permute(1, 0, 2)[None]
+    kt = torch.tensor(np.array(ks)).permute(1, 0, 2)[None]
+    vt = torch.tensor(np.array(vs)).permute(1, 0, 2)[None]
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).numpy()[0]
+
+
+@pytest.mark.parametrize("C,S,W", [(2, 1, 2), (1, 2, 3)])
+def test_repinned_sink_matches_torch_sdpa(C, S, W):
+    w = TINY.with_(C=C, S=S, W=W, refresh_period=3, sink_repin=True)
+    cfg = _cfg(w)
+    sp = spec_for(w)
+    toks, heads = _all_rows(w)
+    for c in (1, 3, 4, 7):
+        base = O.base_at(cfg, c)
+        pos = lambda f: f - min(base, S) if f < S else f - base  # noqa: E731
+        ref = _sdpa_chunk(w, cfg, sp, c, pos)
+        got = O.attend_rows(cfg, sp, 0, c, toks, heads)
+        np.testing.assert_allclose(got, ref[heads, toks], rtol=0, atol=1e-12)
+        assert O.sink_pos(cfg, 0, c) == -min(base, S)
+    # before the first refresh the two modes agree; after it the re-pinned
+    # sink is not refresh-invariant while the shifted one is
+    shift = _cfg(w.with_(sink_repin=False))
+    np.testing.assert_array_equal(O.attend_rows(cfg, sp, 0, 2, toks, heads),
+                                  O.attend_rows(shift, sp, 0, 2, toks, heads))
+    norf = _cfg(w.with_(sink_repin=False), period=0)
+    c = 7
+    assert np.abs(O.attend_rows(cfg, sp, 0, c, toks, heads) -
+                  O.attend_rows(norf, sp, 0, c, toks, heads)).max() > 1e-6
+    np.testing.assert_allclose(O.attend_rows(shift, sp, 0, c, toks, heads),
+                               O.attend_rows(norf, sp, 0, c, toks, heads), rtol=0, atol=1e-9)
+
+
+@pytest.mark.parametrize("alpha", [1.0, 0.5])
+def test_sink_update_matches_torch_sdpa(alpha):
+    import inputgen as IG
+    w = TINY.with_(C=1, S=2, W=2, refresh_period=4, sink_update_period=3, sink_alpha=alpha)
+    cfg = _cfg(w)
+    sp = spec_for(w)
+    F = w.F
+    toks, heads = _all_rows(w)
+    for c in (2, 3, 5, 6, 9):
+        # raw sink after the updates before chunks 3, 6, 9 that are <= c
+        sk = {f: O.input_block(cfg, sp, 0, f // w.C, K)[(f % w.C) * F:(f % w.C + 1) * F]
+              for f in range(w.S)}
+        sv = {f: O.input_block(cfg, sp, 0, f // w.C, V)[(f % w.C) * F:(f % w.C + 1) * F]
+              for f in range(w.S)}
+        for u in range(3, c + 1, 3):
+            nk = IG.fill_host_f32(w, 0, IG.sink_update_chunk(u), K, tok0=0, n_tok=w.S * F)
+            nv = IG.fill_host_f32(w, 0, IG.sink_update_chunk(u), V, tok0=0, n_tok=w.S * F)
+            for f in range(w.S):
+                sk[f] = (1 - alpha) * sk[f] + alpha * nk[f * F:(f + 1) * F]
+                sv[f] = (1 - alpha) * sv[f] + alpha * nv[f * F:(f + 1) * F]
+        base = O.base_at(cfg, c)
+        ref = _sdpa_chunk(w, cfg, sp, c, lambda f: f - base, sk, sv)
+        got = O.attend_rows(cfg, sp, 0, c, toks, heads)
+        np.testing.assert_allclose(got, ref[heads, toks], rtol=0, atol=1e-12)
+        for f in range(w.S):
+            np.testing.assert_allclose(O.sink_raw(cfg, sp, 0, f, c, K), sk[f], rtol=0, atol=1e-15)
+
+
+def test_sink_update_weight_zero_is_no_update_and_rounds_like_torch():
+    w = TINY.with_(C=2, S=1, W=2, sink_update_period=2, sink_alpha=0.0)
+    sp = spec_for(w)
+    toks, heads = _all_rows(w)
+    np.testing.assert_array_equal(O.attend_rows(_cfg(w), sp, 0, 5, toks, heads),
+                                  O.attend_rows(_cfg(w.with_(sink_update_period=0)), sp, 0, 5,
+                                                toks, heads))
+    # storage mode: one update at weight 0.3, rounded once to bf16 by the
+    # (separately pinned) storage rounding; torch's fp64 -> bf16 cast passes
+    # through fp32 (two roundings), so it may differ by one ulp next to a tie
+    import inputgen as IG
+    wb = w.with_(dtype="bf16", sink_alpha=0.3)
+    cb = _cfg(wb, store=O.STORE_BF16)
+    spb = spec_for(wb)
+    raw0 = O.input_block(cb, spb, 0, 0, V)[:wb.F]
+    new = IG.fill_host_f32(wb, 0, IG.sink_update_chunk(2), V, tok0=0, n_tok=wb.F)
+    blend = (1.0 - 0.3) * raw0 + 0.3 * new.astype(np.float64)
+    want = np.vectorize(lambda x: O.round_store(O.STORE_BF16, float(x)))(blend)
+    got = O.sink_raw(cb, spb, 0, 0, 3, V)
+    np.testing.assert_array_equal(got, want)
+    via_torch = torch.tensor(blend).to(torch.bfloat16).double().numpy()
+    assert np.abs(got - via_torch).max() <= np.abs(got).max() * 2.0 ** -7
+
+
+# --------------------------------------------------------------------------
 # T5: closed-form special cases
 # --------------------------------------------------------------------------
 @pytest.mark.parametrize("store", [O.EXACT, O.STORE_BF16])
