@@ -22,7 +22,7 @@ EXPORTED = (
     "sa_get_device_status", "sa_plan_chunk", "sa_refresh_delta", "sa_profile_begin",
     "sa_profile_end", "sa_last_error_string", "sa_abi_version", "sa_append_attend_noalloc",
     "sa_profile_launches", "sa_wait_probe", "sa_attend", "sa_cache_set_sink_mode",
-    "sa_sink_update",
+    "sa_sink_update", "sa_append_attend_host_async", "sa_host_wait",
 )
 
 
@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         "sa_cache_reset": [vp, vp],
         "sa_cache_destroy": [vp],
         "sa_append_attend_host": [vp, vp, vp, vp, vp, vp, vp],
+        "sa_append_attend_host_async": [vp, vp, vp, vp, vp, vp, vp],
+        "sa_host_wait": [vp],
         "sa_stream_state": [vp, i32, P(i64), P(i64)],
         "sa_cache_copy_out": [vp, i32, vp, vp, vp],
         "sa_get_device_status": [vp, vp],

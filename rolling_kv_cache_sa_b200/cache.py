@@ -101,6 +101,20 @@ def sa_append_attend_host(h: int, q: torch.Tensor, k: torch.Tensor, v: torch.Ten
           "sa_append_attend_host")
 
 
+def sa_append_attend_host_async(h: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                out: torch.Tensor, active=None,
+                                stream: Optional[torch.cuda.Stream] = None):
+    for t in (q, k, v, out):
+        assert t.device.type == "cpu" and t.is_contiguous()
+    check(lib().sa_append_attend_host_async(h, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            out.data_ptr(), _mask(active, q.shape[0]),
+                                            _stream_ptr(stream)), "sa_append_attend_host_async")
+
+
+def sa_host_wait(h: int):
+    check(lib().sa_host_wait(h), "sa_host_wait")
+
+
 def sa_stream_state(h: int, b: int):
     fw, base = ctypes.c_int64(), ctypes.c_int64()
     check(lib().sa_stream_state(h, b, ctypes.byref(fw), ctypes.byref(base)), "sa_stream_state")
@@ -209,6 +223,14 @@ class SACache:
         for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
             self._check_tensor(t, n)
         sa_attend(self.h, q, k, v, out, active, stream, self.B)
+
+    def append_attend_host_async(self, q, k, v, out, active=None, stream=None):
+        """Queues the host-buffer step and returns; host_wait() before reading
+        out or reusing the inputs."""
+        sa_append_attend_host_async(self.h, q, k, v, out, active, stream)
+
+    def host_wait(self):
+        sa_host_wait(self.h)
 
     def set_sink_mode(self, mode: int):
         sa_cache_set_sink_mode(self.h, mode)

@@ -54,6 +54,15 @@ class StreamSession:
             self.cache.rope_refresh(mask, stream)
         self.cache.attend(q, k, v, out, active, stream)
 
+    def step_host_async(self, q, k, v, out, active: Optional[Sequence[bool]] = None,
+                        stream=None):
+        """Same as step_host, queued without waiting (pipelined copies); call
+        cache.host_wait() before reading out."""
+        mask = self.refresh_mask(active)
+        if mask is not None:
+            self.cache.rope_refresh(mask, stream)
+        self.cache.append_attend_host_async(q, k, v, out, active, stream)
+
     def step_host(self, q, k, v, out, active: Optional[Sequence[bool]] = None, stream=None):
         """Same as step with host tensors (copies inside the call)."""
         mask = self.refresh_mask(active)

@@ -158,6 +158,42 @@ def test_host_buffer_entry_matches_device_entry():
         b.close()
 
 
+def test_pipelined_host_entry_matches_device_entry():
+    """The queued host path (three staging slots in rotation, copies on their
+    own streams) gives the device path's outputs bit for bit, across a
+    refresh and with every chunk's host buffers queued before one wait."""
+    w = Workload("pipe", B=2, H=4, D=128, fh=8, fw=16, C=2, S=1, W=4, n_chunks=9, dtype="bf16",
+                 refresh_period=4, starts=(0, 1))
+    a, b = Runner(w), Runner(w)
+    try:
+        n = w.n_steps
+        shape = (n,) + tuple(a.q.shape)
+        qh = torch.empty(shape, dtype=a.q.dtype).pin_memory()
+        kh, vh = torch.empty_like(qh).pin_memory(), torch.empty_like(qh).pin_memory()
+        oh = torch.zeros_like(qh).pin_memory()
+        ref = torch.zeros(shape, dtype=a.q.dtype)
+        acts = []
+        for g in range(n):
+            chunks, active = a.step(g)
+            acts.append(active)
+            torch.cuda.synchronize()
+            qh[g].copy_(a.q)
+            kh[g].copy_(a.k)
+            vh[g].copy_(a.v)
+            ref[g].copy_(a.out.cpu())
+        for g in range(n):
+            b.sess.step_host_async(qh[g], kh[g], vh[g], oh[g], acts[g])
+        b.cache.host_wait()
+        for g in range(n):
+            for s_, on in enumerate(acts[g]):
+                if on:
+                    assert torch.equal(oh[g][s_], ref[g][s_]), (g, s_)
+        assert b.device_status() == 0
+    finally:
+        a.close()
+        b.close()
+
+
 def test_invalid_arguments_leave_state_unchanged():
     from rolling_kv_cache_sa_b200 import SAError, sa_append_attend
     w = Workload("inv", B=1, H=2, D=128, fh=8, fw=16, C=1, S=1, W=2, n_chunks=2, dtype="bf16")
