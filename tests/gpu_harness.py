@@ -145,4 +145,4 @@ def assert_cache(w, runner, b, c, sink_ulps=0):
         tol = np.abs(kr) * 2.0 ** -22 + rowmax * 2.0 ** -21 + 1e-9
     bad = kd > tol
     assert not bad.any(), (b, c, int(bad.sum()), float(kd.max()))
-    return float(kd.max())
+    return float(kd.max()) if kd.size else 0.0
