@@ -344,8 +344,9 @@ def main():
     att_flops_per_launch = step_flops * prof_steps / max(att_n, 1)
     att_avg_s = att_ms / 1000.0 / max(att_n, 1)
     achieved = att_flops_per_launch / att_avg_s / 1e12
-    app_avg_s = app_ms / 1000.0 / max(app_n, 1)
-    append_gbs = append_bytes_per_chunk * w.B / app_avg_s / 1e9 if app_n else None
+    # append bytes: every active (stream, chunk) of the profiled steps
+    append_gbs = (append_bytes_per_chunk * chunks_per_step * prof_steps / (app_ms / 1000.0) / 1e9
+                  if app_n and app_ms > 0 else None)
 
     e2e = None
     if not args.no_e2e:
