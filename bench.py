@@ -406,7 +406,7 @@ def main():
         "config": config_json(w, world),
         "ms_per_chunk": ms_step / chunks_per_step,
         "attention_tflops_whole_step": att_tflops_step,
-        "attention_frac_of_peak_whole_step": att_tflops_step / pk_burst,
+        "attention_frac_of_peak_whole_step": att_tflops_step / pk_sust,
         "append_gbs": append_gbs,
         "append_frac_of_hbm": (append_gbs / hbm) if append_gbs else None,
         "kernel_ms_per_step": {"attend": att_ms / prof_steps, "append": app_ms / prof_steps,
@@ -415,10 +415,14 @@ def main():
         "launch_mode": "cuda graph of one step, replayed" if graph is not None else "eager",
         "eager_chunks_per_s": chunks_per_step * world / (ms_eager / 1000.0),
         "eager_ms_per_step": ms_eager,
+        # the kernel is timed inside long back-to-back stepping (the eager
+        # pass and the replays run continuously under the power cap), so the
+        # denominator is the sustained bf16 figure; the burst one is kept too
         "roofline": {"bound": "tensor", "kernel": "attend_tc_kernel<128>",
-                     "achieved": achieved, "peak": pk_burst, "unit": "TFLOP/s",
-                     "frac": achieved / pk_burst, "peak_source": f"{pk_src} bf16 burst",
-                     "frac_of_sustained": achieved / pk_sust,
+                     "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
+                     "frac": achieved / pk_sust,
+                     "peak_source": f"{pk_src} bf16 sustained (timed inside long stepping)",
+                     "frac_of_burst": achieved / pk_burst,
                      "duration": "mean of the library's CUDA events around each launch, on "
                                  "its launch stream, over the eager timed pass",
                      "traffic": PROFILED_TRAFFIC.get(attend_source_hash()),
