@@ -90,6 +90,12 @@ def test_long_stress_10000_chunks():
     ("d64", dict(D=64)),
     ("odd_frame_tails", dict(fh=5, fw=7, C=3, S=1, W=3)),
     ("single_partial_tile", dict(fh=4, fw=5, C=1, S=1, W=1)),
+    # 64 streams (the handle's maximum), ragged: several append and refresh
+    # launches per call, stream-K units spanning many streams
+    ("max_streams_64", dict(B=64, H=2, fh=4, fw=8, C=1, S=1, W=2, n_chunks=6,
+                            starts=tuple(i % 5 for i in range(64)))),
+    ("multi_frame_chunk", dict(C=4, S=2, W=4, fh=8, fw=8)),
+    ("many_heads", dict(H=32, fh=8, fw=8)),
 ])
 def test_bf16_edge_cases_every_row(name, kw):
     base = Workload("edge_" + name, B=2, H=3, D=128, fh=16, fw=12, C=1, S=1, W=2, n_chunks=9,
