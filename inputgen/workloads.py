@@ -49,6 +49,8 @@ class Workload:
     sink_repin: bool = False  # after a refresh the sink sits right before the window
     sink_update_period: int = 0  # sink update before chunk u (u > 0, u % period == 0); 0 = never
     sink_alpha: float = 1.0  # weight of the new sink data (1 = replace)
+    cache: str = ""  # "" = the cache keeps dtype; "e4m3" = bf16 in/out, e4m3 cache and MMAs
+    fp8_scales: Tuple = ()  # e4m3 cache: ((q scales per head), (k ...), (v ...)); () = 1
 
     @property
     def F(self) -> int:

@@ -17,7 +17,7 @@ from inputgen.workloads import Workload
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
-EXACT, STORE_F32, STORE_BF16 = 0, 1, 2
+EXACT, STORE_F32, STORE_BF16, STORE_E4M3 = 0, 1, 2, 3
 
 
 class Cfg(ctypes.Structure):
@@ -29,6 +29,7 @@ class Cfg(ctypes.Structure):
         ("refresh_period", ctypes.c_int64), ("store", ctypes.c_int32),
         ("in_dtype", ctypes.c_int32), ("sink_repin", ctypes.c_int32), ("pad_", ctypes.c_int32),
         ("sink_update_period", ctypes.c_int64), ("sink_alpha", ctypes.c_double),
+        ("fp8_scale", ctypes.c_void_p),
     ]
 
 
@@ -87,9 +88,15 @@ def cfg_for(w: Workload, store: int | None = None, refresh_period: int | None = 
     c.scale = 0.0
     c.refresh_period = w.refresh_period if refresh_period is None else refresh_period
     if store is None:
-        store = STORE_BF16 if w.dtype == "bf16" else STORE_F32
+        store = STORE_E4M3 if w.cache == "e4m3" else (STORE_BF16 if w.dtype == "bf16" else STORE_F32)
     c.store = store
     c.in_dtype = 1 if w.dtype == "bf16" else 0
+    if w.fp8_scales:
+        arr = np.ascontiguousarray(np.asarray(w.fp8_scales, dtype=np.float64).reshape(3, w.H))
+        c._scales = arr  # keeps the array alive with the struct
+        c.fp8_scale = arr.ctypes.data
+    else:
+        c.fp8_scale = None
     c.sink_repin = 1 if w.sink_repin else 0
     c.sink_update_period = w.sink_update_period
     c.sink_alpha = w.sink_alpha

@@ -41,10 +41,42 @@ static double round_to_bits(double x, int bits) {
   return ldexp(r, e - bits);
 }
 
+/* e4m3 (OCP FP8 E4M3, no infinities): 1 sign, 4 exponent bits (bias 7), 3
+ * mantissa bits; normal numbers 2^-6 .. 448, subnormals in steps of 2^-9.
+ * Round to nearest, ties to even, on that grid; magnitudes beyond 448
+ * saturate to 448 (a conversion with saturation to the largest finite). */
+static double round_e4m3(double x) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  const double a = fabs(x);
+  int e;
+  frexp(a, &e);                       /* a in [2^(e-1), 2^e) */
+  int k = e - 1;
+  if (k < -6) k = -6;                 /* subnormal range keeps the 2^-9 step */
+  const double q = ldexp(1.0, k - 3); /* grid step: 3 mantissa bits */
+  double r = nearbyint(a / q) * q;
+  if (r > 448.0) r = 448.0;
+  return copysign(r, x);
+}
+
 double orc_round_store(int32_t store, double x) {
   if (store == ORC_STORE_F32) return (double)(float)x;
   if (store == ORC_STORE_BF16) return round_to_bits(x, 8);
+  if (store == ORC_STORE_E4M3) return round_e4m3(x);
   return x;
+}
+
+/* Stored value of a rotated query (which = 0), rotated key (1) or value (2)
+ * of head h: the storage rounding, with the head's scale in e4m3 mode. */
+static double round_head(const orc_cfg* g, int which, int h, double x) {
+  if (g->store != ORC_STORE_E4M3) return orc_round_store(g->store, x);
+  const double s = g->fp8_scale ? g->fp8_scale[which * g->H + h] : 1.0;
+  return round_e4m3(x * s) / s;
+}
+
+/* Precision of the raw (unrotated) sink keys: the cache type, except in
+ * e4m3 mode where the raw sink keeps the bf16 input precision. */
+static int32_t raw_store(const orc_cfg* g) {
+  return g->store == ORC_STORE_E4M3 ? ORC_STORE_BF16 : g->store;
 }
 
 /* ---------------------------------------------------------------------------
@@ -218,6 +250,12 @@ int32_t orc_sink_raw(const orc_cfg* g, const ig_spec* sp, int64_t stream, int64_
   if (!g || !sp || !out || f < 0 || f >= g->S || (tensor != IG_K && tensor != IG_V)) return -1;
   const int64_t F = frame_tokens(g), n = F * (int64_t)g->H * g->D;
   gen_tokens(g, sp, stream, f / g->C, tensor, (f % g->C) * F, F, out);
+  /* values are kept as stored (e4m3 mode: the cache's own rounding, per
+   * head); raw keys at raw_store precision */
+  const int v_stored = tensor == IG_V && g->store == ORC_STORE_E4M3;
+#define SINK_ROUND(i, x) \
+  (v_stored ? round_head(g, 2, (int)(((i) / g->D) % g->H), (x)) : orc_round_store(raw_store(g), (x)))
+  for (int64_t i = 0; i < n; ++i) out[i] = SINK_ROUND(i, out[i]);
   if (g->sink_update_period <= 0) return 0;
   double* nw = (double*)malloc(sizeof(double) * (size_t)n);
   if (!nw) return -2;
@@ -225,8 +263,9 @@ int32_t orc_sink_raw(const orc_cfg* g, const ig_spec* sp, int64_t stream, int64_
   for (int64_t u = g->sink_update_period; u <= c; u += g->sink_update_period) {
     if (!sink_update_due(g, u)) continue;
     gen_tokens(g, sp, stream, IG_SINK_UPDATE_CHUNK0 + u, tensor, f * F, F, nw);
-    for (int64_t i = 0; i < n; ++i) out[i] = orc_round_store(g->store, (1.0 - a) * out[i] + a * nw[i]);
+    for (int64_t i = 0; i < n; ++i) out[i] = SINK_ROUND(i, (1.0 - a) * out[i] + a * nw[i]);
   }
+#undef SINK_ROUND
   free(nw);
   return 0;
 }
@@ -274,11 +313,12 @@ int32_t orc_stored_key_frame(const orc_cfg* g, const ig_spec* sp, int64_t stream
     const double* kin = raw + th * D;
     double* ko = out + th * D;
     double tmp[512];
+    const int h = (int)(th % H);
     orc_rope_vec(g, kin, pos, y, x, tmp);
-    for (int d = 0; d < D; ++d) ko[d] = orc_round_store(g->store, tmp[d]);
+    for (int d = 0; d < D; ++d) ko[d] = round_head(g, 1, h, tmp[d]);
     for (int i = 0; i < n_ref; ++i) {
       orc_rope_tband(g, ko, -(double)deltas[i], tmp);
-      for (int d = 0; d < D; ++d) ko[d] = orc_round_store(g->store, tmp[d]);
+      for (int d = 0; d < D; ++d) ko[d] = round_head(g, 1, h, tmp[d]);
     }
   }
   free(raw);
@@ -303,7 +343,7 @@ int32_t orc_query_rot(const orc_cfg* g, const ig_spec* sp, int64_t stream, int64
     double tmp[512];
     orc_rope_vec(g, raw + th * D, (double)(f - base), (double)(j / g->fw),
                  (double)(j % g->fw), tmp);
-    for (int d = 0; d < D; ++d) out[th * D + d] = orc_round_store(g->store, tmp[d]);
+    for (int d = 0; d < D; ++d) out[th * D + d] = round_head(g, 0, (int)(th % H), tmp[d]);
   }
   free(raw);
   return 0;
@@ -326,10 +366,13 @@ int32_t orc_cache_contents(const orc_cfg* g, const ig_spec* sp, int64_t stream, 
     const int64_t f = slot_frame[s];
     if (f < 0) continue;
     orc_stored_key_frame(g, sp, stream, f, c, kf);
-    if (f < g->S)
+    if (f < g->S) {
       orc_sink_raw(g, sp, stream, f, c, IG_V, vf);
-    else
+    } else {
       gen_tokens(g, sp, stream, f / g->C, IG_V, (f % g->C) * F, F, vf);
+      if (g->store == ORC_STORE_E4M3)
+        for (int64_t i = 0; i < F * H * D; ++i) vf[i] = round_head(g, 2, (int)((i / D) % H), vf[i]);
+    }
     for (int64_t j = 0; j < F; ++j)
       for (int h = 0; h < H; ++h)
         for (int d = 0; d < D; ++d) {
@@ -405,10 +448,13 @@ static int32_t attend_rows_two(const orc_cfg* g, const ig_spec* sp_past, const i
     if (!orc_visible(g, c, f)) continue;
     const ig_spec* sp = f < c * g->C ? sp_past : sp_chunk;
     orc_stored_key_frame(g, sp, stream, f, c, kf);
-    if (f < g->S)
+    if (f < g->S) {
       orc_sink_raw(g, sp, stream, f, c, IG_V, vf);
-    else
+    } else {
       gen_tokens(g, sp, stream, f / g->C, IG_V, (f % g->C) * F, F, vf);
+      if (g->store == ORC_STORE_E4M3)
+        for (int64_t i = 0; i < F * H * D; ++i) vf[i] = round_head(g, 2, (int)((i / D) % H), vf[i]);
+    }
     for (int64_t j = 0; j < F; ++j)
       for (int h = 0; h < H; ++h)
         for (int d = 0; d < D; ++d) {

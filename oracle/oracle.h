@@ -35,7 +35,7 @@
 extern "C" {
 #endif
 
-enum { ORC_EXACT = 0, ORC_STORE_F32 = 1, ORC_STORE_BF16 = 2 };
+enum { ORC_EXACT = 0, ORC_STORE_F32 = 1, ORC_STORE_BF16 = 2, ORC_STORE_E4M3 = 3 };
 
 typedef struct {
   int32_t H, D, fh, fw;
@@ -53,6 +53,8 @@ typedef struct {
   int64_t sink_update_period; /* sink update before chunk u when u > 0, u % period == 0
                                  and the sink is complete (uC >= S); 0 = never */
   double sink_alpha;      /* weight of the new sink data in the update (1 = replace) */
+  const double* fp8_scale; /* ORC_STORE_E4M3: [3][H] per-head scales of q, k, v; a value x
+                              is stored as round_e4m3(x * s) / s; NULL = all 1 */
 } orc_cfg;
 
 double orc_round_store(int32_t store, double x);

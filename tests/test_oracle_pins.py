@@ -438,6 +438,62 @@ def test_sink_update_weight_zero_is_no_update_and_rounds_like_torch():
 
 
 # --------------------------------------------------------------------------
+# e4m3 cache storage (NEXT-4): the rounding against torch's float8_e4m3fn
+# cast, and the e4m3-stored attention with per-head scales against torch
+# SDPA over a context stored through that cast
+# --------------------------------------------------------------------------
+def _e4m3(x):
+    return torch.tensor(np.asarray(x, dtype=np.float32)).to(torch.float8_e4m3fn).double().numpy()
+
+
+def test_round_store_e4m3_matches_torch_cast():
+    rng = np.random.default_rng(3)
+    vals = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.uniform(-4, 2.6, 20000),
+        np.ldexp(np.arange(-64, 65), -9),                 # subnormal grid and beyond
+        np.array([448.0, -448.0, 0.0, 2.0 ** -6, 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -11]),
+    ]).astype(np.float32)
+    vals = vals[np.abs(vals) <= 448.0]
+    ours = np.array([O.round_store(O.STORE_E4M3, float(v)) for v in vals])
+    np.testing.assert_array_equal(ours, _e4m3(vals))
+    # saturation to the largest finite value; the tie 464 goes to even (448)
+    assert O.round_store(O.STORE_E4M3, 1000.0) == 448.0
+    assert O.round_store(O.STORE_E4M3, -470.0) == -448.0
+    assert O.round_store(O.STORE_E4M3, 464.0) == 448.0
+    assert O.round_store(O.STORE_E4M3, 2.0 ** -10) == 0.0   # tie below the smallest subnormal
+
+
+def test_e4m3_storage_attention_matches_torch_sdpa():
+    w = TINY.with_(dtype="bf16", cache="e4m3", C=2, S=1, W=2,
+                   fp8_scales=((2.0, 0.75), (4.0, 1.5), (8.0, 0.5)))
+    cfg = O.cfg_for(w)
+    sp = spec_for(w)
+    F, H, C = w.F, w.H, w.C
+    sq, sk, sv = (np.asarray(x) for x in w.fp8_scales)
+    toks, heads = _all_rows(w)
+    for c in (0, 2, 5):
+        frames = [f for f in range((c + 1) * C) if f < w.S or f >= c * C - w.W]
+        ks, vs = [], []
+        for f in frames:
+            blk_k = O.input_block(cfg, sp, 0, f // C, K)
+            blk_v = O.input_block(cfg, sp, 0, f // C, V)
+            for j in range(F):
+                i = (f % C) * F + j
+                ks.append([_e4m3(O.rope_vec(cfg, blk_k[i, h], f, j // w.fw, j % w.fw) * sk[h]) / sk[h]
+                           for h in range(H)])
+                vs.append([_e4m3(blk_v[i, h] * sv[h]) / sv[h] for h in range(H)])
+        qb = O.input_block(cfg, sp, 0, c, Q)
+        qs = [[_e4m3(O.rope_vec(cfg, qb[i, h], c * C + i // F, (i % F) // w.fw, (i % F) % w.fw)
+                     * sq[h]) / sq[h] for h in range(H)] for i in range(w.Lc)]
+        qt = torch.tensor(np.array(qs)).permute(1, 0, 2)[None]
+        kt = torch.tensor(np.array(ks)).permute(1, 0, 2)[None]
+        vt = torch.tensor(np.array(vs)).permute(1, 0, 2)[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).numpy()[0]
+        got = O.attend_rows(cfg, sp, 0, c, toks, heads)
+        np.testing.assert_allclose(got, ref[heads, toks], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
 # T5: closed-form special cases
 # --------------------------------------------------------------------------
 @pytest.mark.parametrize("store", [O.EXACT, O.STORE_BF16])
