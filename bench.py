@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="512p_32x32_h24")
+    ap.add_argument("--cache", default="", choices=["", "e4m3"],
+                    help="e4m3: bf16 in/out with an e4m3 K'/V cache and fp8 attention MMAs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -192,6 +194,7 @@ def config_json(w, world):
             "frame": f"{w.fh}x{w.fw}", "chunk_frames": w.C, "sink_frames": w.S,
             "window_frames": w.W, "chunks_per_stream": w.n_chunks,
             "refresh_every": w.refresh_period, "rope_dims": list(w.dims),
+            "cache": "e4m3 (per-head scales 1)" if w.cache == "e4m3" else w.dtype,
             "parallelism": f"independent streams per GPU x{world} (no collective)",
             "l2": "inputs larger than L2 (every chunk of the step resident, "
                   f"{3 * w.n_chunks * w.B * w.Lc * w.H * w.D * (2 if w.dtype == 'bf16' else 4) / 1e9:.1f}"
@@ -209,6 +212,8 @@ def main():
     w = BY_NAME[args.workload]
     if args.chunks:
         w = w.with_(n_chunks=args.chunks)
+    if args.cache:
+        w = w.with_(cache=args.cache)
 
     if args.impl == "reference":
         run_reference(args, w, rank, world)
@@ -254,7 +259,8 @@ def main():
     for c in range(w.n_chunks):
         step_flops += w.B * attention_flops(cfg, sa_plan_chunk(cfg, c * w.C, 0).n_keys)
     esz = 2 if w.dtype == "bf16" else 4
-    append_bytes_per_chunk = 6 * w.Lc * w.H * w.D * esz  # read q,k,v; write q',k',v
+    cesz = 1 if w.cache == "e4m3" else esz  # cache element bytes
+    append_bytes_per_chunk = 3 * w.Lc * w.H * w.D * (esz + cesz)  # read q,k,v; write q',k',v
 
     def run_step():
         cache.reset()
@@ -338,6 +344,9 @@ def main():
     value = aggregate_rate(chunks_per_step * args.steps, world, ms)
 
     hbm, pk_burst, pk_sust, pk_src = peaks()
+    f8 = w.cache == "e4m3"
+    if f8:  # fp8 contraction: the measured bf16 peaks x the nominal 2x (4.5 / 2.25 PFLOP/s)
+        pk_burst, pk_sust = 2.0 * pk_burst, 2.0 * pk_sust
     att_ms, att_n = prof["attend"]
     app_ms, app_n = prof["append"]
     ref_ms, ref_n = prof["refresh"]
@@ -401,7 +410,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "chunks/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if f8 else "bf16",
         "data": "synthetic (seeded counter generator; Irwin-Hall N(0,1) inputs)",
         "config": config_json(w, world),
         "ms_per_chunk": ms_step / chunks_per_step,
@@ -418,14 +428,16 @@ def main():
         # the kernel is timed inside long back-to-back stepping (the eager
         # pass and the replays run continuously under the power cap), so the
         # denominator is the sustained bf16 figure; the burst one is kept too
-        "roofline": {"bound": "tensor", "kernel": "attend_tc_kernel<128>",
+        "roofline": {"bound": "tensor",
+                     "kernel": "attend_tc_kernel<128, e4m3>" if f8 else "attend_tc_kernel<128>",
                      "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
                      "frac": achieved / pk_sust,
-                     "peak_source": f"{pk_src} bf16 sustained (timed inside long stepping)",
+                     "peak_source": (f"{pk_src} bf16 sustained x 2 (fp8 nominal ratio)" if f8 else
+                                     f"{pk_src} bf16 sustained (timed inside long stepping)"),
                      "frac_of_burst": achieved / pk_burst,
                      "duration": "mean of the library's CUDA events around each launch, on "
                                  "its launch stream, over the eager timed pass",
-                     "traffic": PROFILED_TRAFFIC.get(attend_source_hash()),
+                     "traffic": PROFILED_TRAFFIC.get(attend_source_hash() + ("/e4m3" if f8 else "")),
                      "traffic_note": "ncu dram read+write bytes of one steady-state launch "
                                      "(7168 keys, cold L2); algorithmic minimum 113 MB; the "
                                      "excess is split-unit fp32 partials written and read "

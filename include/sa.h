@@ -62,7 +62,16 @@ typedef enum {
   SA_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up on a bounded wait (see sa_get_device_status) */
 } sa_status;
 
-typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
+/* SA_F32, SA_BF16: q, k, v, out and the cache in that type.
+ * SA_BF16_E4M3: q, k, v, out in bf16; the rotated keys and values in the
+ * cache, the rotated queries and the attention's P in e4m3 (OCP FP8 E4M3,
+ * round to nearest even, saturating to +-448) with per-head scales
+ * (sa_cache_set_fp8_scales): a value x of head h is stored as
+ * e4m3(x * s[h]); both attention products run on the tensor cores in fp8
+ * with fp32 accumulation. Raw sink keys stay bf16. head_dim must be 128.
+ * (SANA-Streaming, system co-design: mixed-precision policy that keeps
+ * sensitive layers in BF16/FP8; here applied to the cache.) */
+typedef enum { SA_F32 = 0, SA_BF16 = 1, SA_BF16_E4M3 = 2 } sa_dtype;
 
 typedef void* sa_stream_t; /* a cudaStream_t */
 
@@ -78,7 +87,7 @@ typedef struct {
   int32_t rope_dims[3];   /* (d_t, d_h, d_w): even, sum = D, d_t <= 128 */
   float rope_base;        /* theta base (> 0), e.g. 10000 */
   float softmax_scale;    /* 0 means 1/sqrt(D) */
-  int32_t dtype;          /* sa_dtype of q, k, v, out and the cache */
+  int32_t dtype;          /* sa_dtype: of q, k, v, out and the cache */
 } sa_config;
 
 typedef struct sa_cache sa_cache; /* opaque */
@@ -199,7 +208,8 @@ sa_status sa_stream_state(const sa_cache* h, int32_t b, int64_t* frames_written,
                           int64_t* pos_base);
 
 /* Copies stream b's cache to host: host_k and host_v receive [H][(S+R)F][D]
- * each in cfg dtype (rows of never-written slots are zero). Synchronous. */
+ * each in the cache's element type (SA_BF16_E4M3: e4m3 bytes, scaled by the
+ * head's k or v scale); rows of never-written slots are zero. Synchronous. */
 sa_status sa_cache_copy_out(const sa_cache* h, int32_t b, void* host_k, void* host_v,
                             sa_stream_t stream);
 
@@ -266,6 +276,19 @@ sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cache, void* v_
 
 /* Number of kernels the handle launched since sa_profile_begin (host count). */
 sa_status sa_profile_launches(const sa_cache* h, int64_t* launches);
+
+/*
+ * Per-head scales of an SA_BF16_E4M3 cache: q_scale, k_scale, v_scale are
+ * host arrays of H positive finite floats (NULL = all 1). A rotated query,
+ * rotated key or value x of head h is stored as e4m3(x * scale[h]); scores
+ * are divided by q_scale[h] * k_scale[h] and outputs by v_scale[h], so the
+ * scales choose where in the e4m3 range (2^-9 .. 448) each head's values
+ * fall. Call before any stream holds a frame (SA_ERR_STATE otherwise);
+ * SA_ERR_INVALID_ARG for another dtype or a non-positive scale. Copies the
+ * scales to the device (synchronous on the handle's create stream).
+ */
+sa_status sa_cache_set_fp8_scales(sa_cache* h, const float* q_scale, const float* k_scale,
+                                  const float* v_scale);
 
 /* Sink position modes (sa_cache_set_sink_mode). */
 #define SA_SINK_SHIFT 0 /* a refresh rebases the sink with every other position: scores invariant */

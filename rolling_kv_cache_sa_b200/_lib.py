@@ -11,7 +11,7 @@ SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_OOM, SA_ERR_CUDA, SA_ERR_S
     SA_ERR_DEVICE_TIMEOUT = range(7)
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_OOM",
                 4: "SA_ERR_CUDA", 5: "SA_ERR_STATE", 6: "SA_ERR_DEVICE_TIMEOUT"}
-SA_F32, SA_BF16 = 0, 1
+SA_F32, SA_BF16, SA_BF16_E4M3 = 0, 1, 2
 SA_SINK_SHIFT, SA_SINK_REPIN = 0, 1
 SA_MAX_CHUNK_FRAMES = 32
 
@@ -22,7 +22,7 @@ EXPORTED = (
     "sa_get_device_status", "sa_plan_chunk", "sa_refresh_delta", "sa_profile_begin",
     "sa_profile_end", "sa_last_error_string", "sa_abi_version", "sa_append_attend_noalloc",
     "sa_profile_launches", "sa_wait_probe", "sa_attend", "sa_cache_set_sink_mode",
-    "sa_sink_update", "sa_append_attend_host_async", "sa_host_wait",
+    "sa_sink_update", "sa_append_attend_host_async", "sa_host_wait", "sa_cache_set_fp8_scales",
 )
 
 
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
         "sa_append_attend": [vp, vp, vp, vp, vp, vp, vp],
         "sa_attend": [vp, vp, vp, vp, vp, vp, vp],
         "sa_cache_set_sink_mode": [vp, i32],
+        "sa_cache_set_fp8_scales": [vp, vp, vp, vp],
         "sa_sink_update": [vp, vp, vp, ctypes.c_float, vp, vp],
         "sa_rope_refresh": [vp, vp, vp],
         "sa_cache_reset": [vp, vp],

@@ -10,7 +10,7 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-from ._lib import SA_BF16, SA_F32, check, lib, sa_chunk_plan, sa_config
+from ._lib import SA_BF16, SA_BF16_E4M3, SA_F32, check, lib, sa_chunk_plan, sa_config
 
 
 def make_config(batch: int, heads: int, head_dim: int, frame_h: int, frame_w: int,
@@ -25,13 +25,14 @@ def make_config(batch: int, heads: int, head_dim: int, frame_h: int, frame_w: in
         c.rope_dims[i] = int(rope_dims[i])
     c.rope_base = rope_base
     c.softmax_scale = softmax_scale
-    c.dtype = SA_BF16 if dtype == "bf16" else SA_F32
+    c.dtype = {"bf16": SA_BF16, "f32": SA_F32, "bf16_e4m3": SA_BF16_E4M3}[dtype]
     return c
 
 
 def config_for(w) -> sa_config:
     """sa_config of a workload description (inputgen.workloads.Workload)."""
-    return make_config(w.B, w.H, w.D, w.fh, w.fw, w.C, w.S, w.W, w.dims, w.rope_base, 0.0, w.dtype)
+    dtype = "bf16_e4m3" if getattr(w, "cache", "") == "e4m3" else w.dtype
+    return make_config(w.B, w.H, w.D, w.fh, w.fw, w.C, w.S, w.W, w.dims, w.rope_base, 0.0, dtype)
 
 
 def _mask(active, n: int):
@@ -69,6 +70,12 @@ def sa_attend(h: int, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: to
 
 def sa_cache_set_sink_mode(h: int, mode: int):
     check(lib().sa_cache_set_sink_mode(h, mode), "sa_cache_set_sink_mode")
+
+
+def sa_cache_set_fp8_scales(h: int, q_scale=None, k_scale=None, v_scale=None):
+    arrs = [None if x is None else (ctypes.c_float * len(x))(*[float(v) for v in x])
+            for x in (q_scale, k_scale, v_scale)]
+    check(lib().sa_cache_set_fp8_scales(h, *arrs), "sa_cache_set_fp8_scales")
 
 
 def sa_sink_update(h: int, k_new: torch.Tensor, v_new: torch.Tensor, alpha: float, active=None,
@@ -202,7 +209,9 @@ class SACache:
         self.Lc = cfg.chunk_frames * self.F
         self.R = cfg.window_frames + cfg.chunk_frames
         self.ntok = (cfg.sink_frames + self.R) * self.F
-        self.dtype = torch.bfloat16 if cfg.dtype == SA_BF16 else torch.float32
+        self.dtype = torch.float32 if cfg.dtype == SA_F32 else torch.bfloat16
+        self.fp8 = cfg.dtype == SA_BF16_E4M3
+        self.scales = np.ones((3, cfg.heads))
         self.device = torch.device("cuda", torch.cuda.current_device())
         self.h = sa_cache_create(cfg, stream)
 
@@ -232,6 +241,12 @@ class SACache:
     def host_wait(self):
         sa_host_wait(self.h)
 
+    def set_fp8_scales(self, q_scale=None, k_scale=None, v_scale=None):
+        """Per-head scales of an e4m3 cache (before the first chunk)."""
+        sa_cache_set_fp8_scales(self.h, q_scale, k_scale, v_scale)
+        for i, x in enumerate((q_scale, k_scale, v_scale)):
+            self.scales[i] = 1.0 if x is None else np.asarray(x, dtype=np.float64)
+
     def set_sink_mode(self, mode: int):
         sa_cache_set_sink_mode(self.h, mode)
 
@@ -259,6 +274,13 @@ class SACache:
     def copy_out(self, b: int):
         """(K', V) of stream b as float32 numpy arrays [H, (S+R)F, D]."""
         shape = (self.H, self.ntok, self.D)
+        if self.fp8:  # e4m3 bytes, scaled by the head's k or v scale
+            kb = np.empty(shape, np.uint8)
+            vb = np.empty(shape, np.uint8)
+            sa_cache_copy_out(self.h, b, kb, vb)
+            dec = lambda x: torch.from_numpy(x).view(torch.float8_e4m3fn).float().numpy()  # noqa: E731
+            return (dec(kb) / self.scales[1][:, None, None]).astype(np.float64), \
+                (dec(vb) / self.scales[2][:, None, None]).astype(np.float64)
         if self.cfg.dtype == SA_BF16:
             kb = np.empty(shape, np.uint16)
             vb = np.empty(shape, np.uint16)

@@ -60,6 +60,8 @@ struct TcParams {
   float2* part_ml;    // [slots][2][128] (m in log2 units, l)
   int* counters;      // [units][2][128] pieces counted in; back to 0 after the merge
   int* status;
+  float inv_qk[kMaxF8Heads];  // e4m3: 1 / (q_scale * k_scale) per head
+  float inv_v[kMaxF8Heads];   // e4m3: 1 / v_scale per head
   int32_t stream_of[kMaxAttnStreams];
   int32_t n_keys[kMaxAttnStreams];
   int32_t nkv[kMaxAttnStreams];
@@ -178,10 +180,11 @@ __device__ __noinline__ void merge_row(const TcParams& p, int ti, int row, int c
   }
 }
 
-template <int HD>
+// F8: e4m3 operands, a 128-element row is one 128-byte panel
+template <int HD, bool F8 = false>
 struct Layout {
-  static constexpr int kStages = HD == 128 ? 2 : 4;
-  static constexpr uint32_t kPanels = HD / 64;
+  static constexpr int kStages = F8 ? 4 : (HD == 128 ? 2 : 4);
+  static constexpr uint32_t kPanels = F8 ? 1 : HD / 64;
   static constexpr uint32_t kTile = kPanels * PANEL;  // one Q, K or V tile
   static constexpr uint32_t q0 = 0;
   static constexpr uint32_t k0 = 2 * kTile;
@@ -234,7 +237,7 @@ __device__ __noinline__ void rescale_o(uint32_t obuf, float alpha) {
 // rate (moving a share of the exponentials to a polynomial on the FMA pipe
 // made it slower). Adds the row sum
 // of P to l (after scaling l by alpha). Returns false if a wait gave up.
-template <int HD>
+template <int HD, bool F8>
 __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int valid, bool first,
                                             float& m, float& l, float sl2, uint32_t bar_od,
                                             uint32_t od_parity, uint32_t bar_pa, uint32_t bar_pb,
@@ -283,9 +286,21 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
                                   sl2v, nmv);
       const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
       ls[e & 3] = __fadd2_rn(ls[e & 3], pe);
-      w[e] = ptx::pack_bf16x2(pe.x, pe.y);
+      if constexpr (F8) {
+        // four e4m3 per column: pairs e and e+1 share a word
+        const uint32_t pp = ptx::pack_e4m3x2(pe.x, pe.y);
+        if (e & 1)
+          w[e >> 1] |= pp << 16;
+        else
+          w[e >> 1] = pp;
+      } else {
+        w[e] = ptx::pack_bf16x2(pe.x, pe.y);
+      }
     }
-    ptx::tmem_st16u(sbuf + (uint32_t)(q * 16), w);
+    if constexpr (F8)
+      ptx::tmem_st8u(sbuf + (uint32_t)(q * 8), w);
+    else
+      ptx::tmem_st16u(sbuf + (uint32_t)(q * 16), w);
     if (q == 1 && __any_sync(0xffffffffu, alpha < 1.f)) {
       // O holds PV of the previous key tile: MMAs complete in issue order and
       // QK of this tile (issued after that PV) has completed
@@ -305,14 +320,18 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
   return true;
 }
 
-template <int HD>
+template <int HD, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ TcParams p) {
-  using L = Layout<HD>;
+  using L = Layout<HD, F8>;
   constexpr int ST = L::kStages;
+  // MMAs per QK^T tile, per half of a PV tile, and V bytes per PV MMA
+  constexpr int kQkSteps = F8 ? HD / 32 : HD / 16;
+  constexpr int kPvHalf = F8 ? BN / 64 : BN / 32;
+  constexpr uint32_t kVStep = F8 ? 4096u : 2048u;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = ptx::smem_u32(smem);
   if (base & 1023u) {  // 128B-swizzled tiles need 1024-byte alignment
@@ -418,8 +437,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(BM, BN, false);
-      constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(BM, HD, true);
+      constexpr uint32_t idesc_qk =
+          F8 ? ptx::idesc_e4m3_f32(BM, BN, false) : ptx::idesc_bf16_f32(BM, BN, false);
+      constexpr uint32_t idesc_pv =
+          F8 ? ptx::idesc_e4m3_f32(BM, HD, true) : ptx::idesc_bf16_f32(BM, HD, true);
+      // K offset of QK^T step kk inside a K-major tile (32 bytes per step)
+      auto qk_off = [](int kk) -> uint32_t {
+        return F8 ? (uint32_t)kk * 32u : (uint32_t)(kk >> 2) * PANEL + (uint32_t)(kk & 3) * 32u;
+      };
+      auto mma_ss = [](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        if constexpr (F8) ptx::umma_ss_f8(d, a, b, id, acc); else ptx::umma_ss(d, a, b, id, acc);
+      };
+      auto mma_ts = [](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        if constexpr (F8) ptx::umma_ts_f8(d, a, b, id, acc); else ptx::umma_ts(d, a, b, id, acc);
+      };
       const uint32_t o0 = tmem + 256u, o1 = tmem + 256u + HD;
       int n = 0, g = 0, g1 = 0, nseg1 = 0;
       bool ok = true;
@@ -438,11 +469,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             return false;
           ptx::tc_fence_after();
 #pragma unroll
-          for (int k2 = 0; k2 < BN / 32; ++k2) {
-            const int kk = h2 * (BN / 32) + k2;
-            ptx::umma_ts(o1, tmem + 128u + (uint32_t)kk * 8u,
-                         ptx::sdesc_sw128(vb + (uint32_t)kk * 2048u, PANEL, 1024), idesc_pv,
-                         (!pend_first || kk > 0) ? 1u : 0u);
+          for (int k2 = 0; k2 < kPvHalf; ++k2) {
+            const int kk = h2 * kPvHalf + k2;
+            mma_ts(o1, tmem + 128u + (uint32_t)kk * 8u,
+                   ptx::sdesc_sw128(vb + (uint32_t)kk * kVStep, PANEL, 1024), idesc_pv,
+                   (!pend_first || kk > 0) ? 1u : 0u);
           }
         }
         ptx::umma_commit(bar(L::B_OD + 1));
@@ -462,19 +493,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tc_fence_after();
           const uint32_t kb = base + L::k0 + s * L::kTile;
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (uint32_t)(kk >> 2) * PANEL + (uint32_t)(kk & 3) * 32u;
-            ptx::umma_ss(tmem, ptx::sdesc_sw128(base + L::q0 + off, 16, 1024),
-                         ptx::sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kQkSteps; ++kk) {
+            const uint32_t off = qk_off(kk);
+            mma_ss(tmem, ptx::sdesc_sw128(base + L::q0 + off, 16, 1024),
+                   ptx::sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
           }
           ptx::umma_commit(bar(L::B_SF + 0));
           if (pend && !issue_pv1()) { ok = false; break; }
           if (sg.two) {
 #pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk) {
-              const uint32_t off = (uint32_t)(kk >> 2) * PANEL + (uint32_t)(kk & 3) * 32u;
-              ptx::umma_ss(tmem + 128u, ptx::sdesc_sw128(base + L::q0 + L::kTile + off, 16, 1024),
-                           ptx::sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kQkSteps; ++kk) {
+              const uint32_t off = qk_off(kk);
+              mma_ss(tmem + 128u, ptx::sdesc_sw128(base + L::q0 + L::kTile + off, 16, 1024),
+                     ptx::sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
             }
             ptx::umma_commit(bar(L::B_SF + 1));
           }
@@ -495,11 +526,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_after();
 #pragma unroll
-            for (int k2 = 0; k2 < BN / 32; ++k2) {
-              const int kk = h2 * (BN / 32) + k2;
-              ptx::umma_ts(o0, tmem + (uint32_t)kk * 8u,
-                           ptx::sdesc_sw128(vb + (uint32_t)kk * 2048u, PANEL, 1024), idesc_pv,
-                           (kv > sg.lo || kk > 0) ? 1u : 0u);
+            for (int k2 = 0; k2 < kPvHalf; ++k2) {
+              const int kk = h2 * kPvHalf + k2;
+              mma_ts(o0, tmem + (uint32_t)kk * 8u,
+                     ptx::sdesc_sw128(vb + (uint32_t)kk * kVStep, PANEL, 1024), idesc_pv,
+                     (kv > sg.lo || kk > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
@@ -532,7 +563,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t sbuf = t_lane + (uint32_t)ti * 128u;
     const uint32_t obuf = t_lane + 256u + (uint32_t)(ti * HD);
-    const float sl2 = p.scale_log2;
     int gi = 0;
     bool ok = true, first = true;
     for (int64_t t = r0; ok && t < r1;) {
@@ -541,6 +571,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool seg_first = first;
       first = false;
       if (ti == 1 && !sg.two) continue;
+      // e4m3: scores carry the head's q and k scales, O its v scale
+      const float sl2 = F8 ? p.scale_log2 * p.inv_qk[sg.h] : p.scale_log2;
+      const float o_scale = F8 ? p.inv_v[sg.h] : 1.f;
       const int n_keys = p.n_keys[sg.a];
       float m_used = 0.f, l = 0.f;
       for (int kv = sg.lo; kv < sg.hi; ++kv, ++gi) {
@@ -552,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         const int valid = n_keys - kv * BN;
-        if (!row_softmax<HD>(sbuf, obuf, valid, kv == sg.lo, m_used, l, sl2, bar(L::B_OD + ti),
+        if (!row_softmax<HD, F8>(sbuf, obuf, valid, kv == sg.lo, m_used, l, sl2, bar(L::B_OD + ti),
                              (uint32_t)(gi - 1) & 1, bar(L::B_PF + ti), bar(L::B_PB + ti),
                              abort_flag)) {
           ok = false;
@@ -569,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue of this unit piece
       const int tok = (2 * sg.qp + ti) * BM + row;
       if (!sg.partial) {
-        const float inv = 1.f / l;
+        const float inv = o_scale / l;
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
                              (((int64_t)sg.b * p.Lc + tok) * p.H + sg.h) * HD;
 #pragma unroll
@@ -598,9 +631,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_ld32(obuf + c * 32, ov);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int g4 = 0; g4 < 8; ++g4)
-            po[(c * 8 + g4) * BM] =
-                make_float4(ov[g4 * 4], ov[g4 * 4 + 1], ov[g4 * 4 + 2], ov[g4 * 4 + 3]);
+          for (int g4 = 0; g4 < 8; ++g4)  // partials in output units (v scale removed)
+            po[(c * 8 + g4) * BM] = make_float4(ov[g4 * 4] * o_scale, ov[g4 * 4 + 1] * o_scale,
+                                                ov[g4 * 4 + 2] * o_scale, ov[g4 * 4 + 3] * o_scale);
         }
         p.part_ml[((int64_t)slot * 2 + ti) * BM + row] = make_float2(m_used, l);
       }
@@ -632,16 +665,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
 
-template <int HD>
+template <int HD, bool F8>
 cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtensorMap* tk,
                       const CUtensorMap* tv, void* partials, size_t partials_bytes, int num_sms,
                       cudaStream_t st, int* n_kernels) {
-  using L = Layout<HD>;
+  using L = Layout<HD, F8>;
   static unsigned configured = 0;  // one bit per device ordinal < 32
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 32 || !(configured & (1u << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<HD>,
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<HD, F8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);
     if (e != cudaSuccess) return e;
     if (dev < 32) configured |= 1u << dev;
@@ -657,6 +690,11 @@ cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtenso
   p.scale_log2 = ap.scale_log2;
   p.out = ap.out;
   p.status = ap.status;
+  if (F8)
+    for (int hh = 0; hh < ap.H && hh < kMaxF8Heads; ++hh) {
+      p.inv_qk[hh] = ap.inv_qk[hh];
+      p.inv_v[hh] = ap.inv_v[hh];
+    }
   int64_t total = 0;
   for (int a = 0; a < ap.n_streams; ++a) {
     p.stream_of[a] = ap.stream_of[a];
@@ -681,7 +719,7 @@ cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtenso
     w += (size_t)2 * G * 2 * BM * sizeof(float2);
     p.counters = reinterpret_cast<int*>(w);
   }
-  attend_tc_kernel<HD><<<G, kThreads, L::bytes, st>>>(*tq, *tk, *tv, p);
+  attend_tc_kernel<HD, F8><<<G, kThreads, L::bytes, st>>>(*tq, *tk, *tv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int launched = 1;
@@ -700,10 +738,16 @@ cudaError_t launch_attend_tc_bf16(const AttnParams& p, int D, const CUtensorMap*
                                   const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                   void* partials, size_t partials_bytes, int num_sms,
                                   cudaStream_t st, int* n_kernels) {
+  if (p.fp8)
+    return D == 128 ? launch_tc<128, true>(p, tm_q, tm_k, tm_v, partials, partials_bytes, num_sms,
+                                           st, n_kernels)
+                    : cudaErrorInvalidValue;
   if (D == 128)
-    return launch_tc<128>(p, tm_q, tm_k, tm_v, partials, partials_bytes, num_sms, st, n_kernels);
+    return launch_tc<128, false>(p, tm_q, tm_k, tm_v, partials, partials_bytes, num_sms, st,
+                                 n_kernels);
   if (D == 64)
-    return launch_tc<64>(p, tm_q, tm_k, tm_v, partials, partials_bytes, num_sms, st, n_kernels);
+    return launch_tc<64, false>(p, tm_q, tm_k, tm_v, partials, partials_bytes, num_sms, st,
+                                n_kernels);
   return cudaErrorInvalidValue;
 }
 

@@ -12,6 +12,7 @@
 namespace sa {
 
 constexpr int kMaxEntries = 32;   // (stream, frame) entries per append launch
+constexpr int kMaxF8Heads = 128;   // heads of an e4m3 cache
 constexpr int kMaxRefresh = 16;   // streams, and (stream, sink frame) entries, per refresh launch
 constexpr int kMaxDt2 = 64;       // d_t / 2 <= 64
 constexpr int kMaxAttnStreams = SA_MAX_STREAMS;
@@ -33,6 +34,7 @@ struct AppendParams {
   int64_t ntok, sf;    // cache rows per (b, h); sink rows per (b, h)
   int32_t dt2, dh2, dw2;
   int32_t n_streams;   // streams in this launch
+  const float* fp8_scale;  // e4m3 cache: [3][H] per-head scales of q, k, v (device)
   int32_t stream_of[kMaxEntries];
   int64_t dest_row[kMaxEntries];   // cache row of the frame's first token
   int64_t raw_row[kMaxEntries];    // raw-sink row of the frame, or -1
@@ -52,6 +54,7 @@ struct RefreshParams {
   const void* v_new;
   float alpha;
   int32_t update;
+  const float* fp8_scale;  // e4m3 cache: [3][H] per-head scales of q, k, v (device)
   const float2* htab;
   const float2* wtab;
   int32_t H, D, fw, F, S;
@@ -78,8 +81,11 @@ struct AttnParams {
   const void* k_cache; // (SIMT path)
   const void* v_cache; // (SIMT path)
   int* status;
+  int32_t fp8;         // e4m3 operands (SA_BF16_E4M3)
   int32_t stream_of[kMaxAttnStreams];
   int32_t n_keys[kMaxAttnStreams];
+  float inv_qk[kMaxF8Heads];  // e4m3: 1 / (q_scale * k_scale) per head
+  float inv_v[kMaxF8Heads];   // e4m3: 1 / v_scale per head
 };
 
 // Workspace the bf16 attention may use for split work units: per slot (two

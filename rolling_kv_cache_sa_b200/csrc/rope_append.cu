@@ -15,6 +15,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace sa {
 namespace {
@@ -220,16 +221,166 @@ __global__ void __launch_bounds__(256) refresh_kernel(const __grid_constant__ Re
   }
 }
 
+// ---------------------------------------------------------------- e4m3 cache
+// bf16 inputs; rotated queries, rotated keys and values stored as e4m3 of the
+// value times the head's scale (q, k, v scales: fp8_scale[0..2][h]); raw sink
+// keys stay bf16. One thread per 8-element vector: 16-byte input loads,
+// 8-byte e4m3 stores.
+__device__ __forceinline__ uint2 to_e4m3x8(const float (&x)[8], float s) {
+  return make_uint2(ptx::pack_e4m3x4(x[0] * s, x[1] * s, x[2] * s, x[3] * s),
+                    ptx::pack_e4m3x4(x[4] * s, x[5] * s, x[6] * s, x[7] * s));
+}
+
+__device__ __forceinline__ void from_e4m3x8(const uint2 v, float inv_s, float (&x)[8]) {
+  const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float2 a = ptx::unpack_e4m3x2(w[i] & 0xFFFFu), b = ptx::unpack_e4m3x2(w[i] >> 16);
+    x[4 * i + 0] = a.x * inv_s;
+    x[4 * i + 1] = a.y * inv_s;
+    x[4 * i + 2] = b.x * inv_s;
+    x[4 * i + 3] = b.y * inv_s;
+  }
+}
+
+__global__ void __launch_bounds__(256) append_rope_e4m3_kernel(const __grid_constant__ AppendParams p) {
+  using V = Vec16<__nv_bfloat16>;
+  constexpr int N = 8;
+  const uint32_t nvec = (uint32_t)p.D / N;
+  const uint32_t per_tok = (uint32_t)p.H * nvec;
+  const uint32_t per_stream = (uint32_t)p.Lc * per_tok;
+  const uint32_t total = per_stream * (uint32_t)p.n_streams;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += gridDim.x * blockDim.x) {
+    const uint32_t a = i / per_stream;
+    const uint32_t r = i - a * per_stream;
+    const uint32_t tok = r / per_tok;
+    const uint32_t r2 = r - tok * per_tok;
+    const uint32_t h = r2 / nvec;
+    const uint32_t vc = r2 - h * nvec;
+    const int b = p.stream_of[a];
+    const int fi = (int)(tok / (uint32_t)p.F);
+    const int j = (int)(tok - (uint32_t)fi * (uint32_t)p.F);
+    const int y = j / p.fw, x = j - (j / p.fw) * p.fw;
+    const int e = (int)a * p.C + fi;
+    const int64_t in_off = (((int64_t)b * p.Lc + tok) * p.H + h) * p.D + (int64_t)vc * N;
+    float q[N], k[N], v[N];
+    V::load(static_cast<const char*>(p.q) + in_off * 2, q);
+    V::load(static_cast<const char*>(p.k) + in_off * 2, k);
+    V::load(static_cast<const char*>(p.v) + in_off * 2, v);
+    const int64_t bh = (int64_t)b * p.H + h;
+    const int64_t row = p.dest_row[e] + j;
+    const int64_t cache_off = (bh * p.ntok + row) * p.D + (int64_t)vc * N;
+    const float sq = __ldg(&p.fp8_scale[h]), sk = __ldg(&p.fp8_scale[p.H + h]),
+                sv = __ldg(&p.fp8_scale[2 * p.H + h]);
+    *reinterpret_cast<uint2*>(static_cast<char*>(p.v_cache) + cache_off) = to_e4m3x8(v, sv);
+    if (p.raw_row[e] >= 0) {
+      const int64_t raw_off = (bh * p.sf + p.raw_row[e] + j) * p.D + (int64_t)vc * N;
+      V::store(static_cast<char*>(p.k_raw) + raw_off * 2, k);
+    }
+#pragma unroll
+    for (int pp = 0; pp < N / 2; ++pp) {
+      const int pi = (int)vc * (N / 2) + pp;
+      const float2 cs = pair_cs(pi, y, x, p.tcs[e], p.dt2, p.dh2, p.dw2, p.htab, p.wtab);
+      rotate(q[2 * pp], q[2 * pp + 1], cs);
+      rotate(k[2 * pp], k[2 * pp + 1], cs);
+    }
+    const int64_t q_off = (bh * p.Lc + tok) * p.D + (int64_t)vc * N;
+    *reinterpret_cast<uint2*>(static_cast<char*>(p.q_ws) + q_off) = to_e4m3x8(q, sq);
+    *reinterpret_cast<uint2*>(static_cast<char*>(p.k_cache) + cache_off) = to_e4m3x8(k, sk);
+  }
+}
+
+// Refresh / sink update of an e4m3 cache: ring keys' temporal band is
+// dequantised, rotated by -Delta and requantised; sink keys are re-derived
+// from the bf16 raw keys; in update mode the raw keys (bf16) and the stored
+// sink values (e4m3) are first blended with the new data.
+__global__ void __launch_bounds__(256) refresh_e4m3_kernel(const __grid_constant__ RefreshParams p) {
+  using V = Vec16<__nv_bfloat16>;
+  constexpr int N = 8;
+  const int a = blockIdx.y;
+  const int b = p.stream_of[a];
+  const int64_t nvec = p.D / N;
+  const int64_t nvt = (2 * p.dt2 + N - 1) / N;
+  const int64_t ring_work = (int64_t)p.H * p.ring_rows[a] * nvt;
+  const int64_t sink_work = (int64_t)p.H * p.sink_rows[a] * nvec;
+  const int64_t total = ring_work + sink_work;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    if (i < ring_work) {
+      const int64_t per_h = p.ring_rows[a] * nvt;
+      const int64_t h = i / per_h;
+      const int64_t rr = (i - h * per_h) / nvt;
+      const int64_t vc = i - h * per_h - rr * nvt;
+      const int64_t off = (((int64_t)b * p.H + h) * p.ntok + p.sf + rr) * p.D + vc * N;
+      uint2* ptr = reinterpret_cast<uint2*>(static_cast<char*>(p.k_cache) + off);
+      const float sk = __ldg(&p.fp8_scale[p.H + h]);
+      float k[N];
+      from_e4m3x8(*ptr, 1.f / sk, k);
+#pragma unroll
+      for (int pp = 0; pp < N / 2; ++pp) {
+        const int pi = (int)vc * (N / 2) + pp;
+        if (pi < p.dt2) rotate(k[2 * pp], k[2 * pp + 1], p.dcs[a][pi]);
+      }
+      *ptr = to_e4m3x8(k, sk);
+    } else {
+      const int64_t ii = i - ring_work;
+      const int64_t per_h = p.sink_rows[a] * nvec;
+      const int64_t h = ii / per_h;
+      const int64_t rr = (ii - h * per_h) / nvec;
+      const int64_t vc = ii - h * per_h - rr * nvec;
+      const int64_t bh = (int64_t)b * p.H + h;
+      const int s = (int)(rr / p.F);
+      const int j = (int)(rr - (int64_t)s * p.F);
+      const int y = j / p.fw, x = j - (j / p.fw) * p.fw;
+      const float sk = __ldg(&p.fp8_scale[p.H + h]);
+      float k[N];
+      char* raw = static_cast<char*>(p.k_raw) + ((bh * p.sf + rr) * p.D + vc * N) * 2;
+      V::load_cache(raw, k);
+      if (p.update) {
+        const int64_t in_off = (((int64_t)b * p.S * p.F + rr) * p.H + h) * p.D + vc * N;
+        uint2* vp = reinterpret_cast<uint2*>(static_cast<char*>(p.v_cache) +
+                                             (bh * p.ntok + rr) * p.D + vc * N);
+        const float sv = __ldg(&p.fp8_scale[2 * p.H + h]);
+        float kn[N], v[N], vn[N];
+        V::load(static_cast<const char*>(p.k_new) + in_off * 2, kn);
+        from_e4m3x8(*vp, 1.f / sv, v);
+        V::load(static_cast<const char*>(p.v_new) + in_off * 2, vn);
+        const float al = p.alpha, am = 1.f - p.alpha;
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+          k[e] = am * k[e] + al * kn[e];
+          v[e] = am * v[e] + al * vn[e];
+        }
+        V::store(raw, k);
+        *vp = to_e4m3x8(v, sv);
+        V::round(k);  // the rotation starts from the stored raw key
+      }
+#pragma unroll
+      for (int pp = 0; pp < N / 2; ++pp) {
+        const int pi = (int)vc * (N / 2) + pp;
+        const float2 cs =
+            pair_cs(pi, y, x, p.scs[a * p.S + s], p.dt2, p.dh2, p.dw2, p.htab, p.wtab);
+        rotate(k[2 * pp], k[2 * pp + 1], cs);
+      }
+      *reinterpret_cast<uint2*>(static_cast<char*>(p.k_cache) + (bh * p.ntok + rr) * p.D + vc * N) =
+          to_e4m3x8(k, sk);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStream_t st) {
-  const int64_t vec = dtype == SA_BF16 ? 8 : 4;
+  const int64_t vec = dtype == SA_F32 ? 4 : 8;
   const int64_t total = (int64_t)p.n_streams * p.Lc * p.H * (p.D / vec);
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = (int64_t)num_sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  if (dtype == SA_BF16)
+  if (dtype == SA_BF16_E4M3)
+    append_rope_e4m3_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
+  else if (dtype == SA_BF16)
     append_rope_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p);
   else
     append_rope_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p);
@@ -239,7 +390,9 @@ cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStr
 cudaError_t launch_refresh(const RefreshParams& p, int dtype, int num_sms, cudaStream_t st) {
   const int per_stream = (num_sms * 8 + p.n_streams - 1) / p.n_streams;
   dim3 grid((unsigned)(per_stream > 0 ? per_stream : 1), (unsigned)p.n_streams);
-  if (dtype == SA_BF16)
+  if (dtype == SA_BF16_E4M3)
+    refresh_e4m3_kernel<<<grid, 256, 0, st>>>(p);
+  else if (dtype == SA_BF16)
     refresh_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(p);
   else
     refresh_kernel<float><<<grid, 256, 0, st>>>(p);

@@ -68,8 +68,11 @@ sa_status validate_config(const sa_config* c) {
   if (!(c->rope_base > 0.f)) return fail(SA_ERR_INVALID_ARG, "rope_base must be > 0");
   if (c->softmax_scale < 0.f || !isfinite(c->softmax_scale))
     return fail(SA_ERR_INVALID_ARG, "softmax_scale must be >= 0 (0 = 1/sqrt(D))");
-  if (c->dtype != SA_F32 && c->dtype != SA_BF16)
-    return fail(SA_ERR_INVALID_ARG, "dtype must be SA_F32 or SA_BF16");
+  if (c->dtype != SA_F32 && c->dtype != SA_BF16 && c->dtype != SA_BF16_E4M3)
+    return fail(SA_ERR_INVALID_ARG, "dtype must be SA_F32, SA_BF16 or SA_BF16_E4M3");
+  if (c->dtype == SA_BF16_E4M3 && (c->head_dim != 128 || c->heads > sa::kMaxF8Heads))
+    return fail(SA_ERR_UNSUPPORTED, "SA_BF16_E4M3 needs head_dim 128 and at most %d heads",
+                sa::kMaxF8Heads);
   const int64_t F = (int64_t)c->frame_h * c->frame_w;
   const int64_t Lc = F * c->chunk_frames;
   const int64_t ntok = F * ((int64_t)c->sink_frames + c->window_frames + c->chunk_frames);
@@ -133,16 +136,20 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 3D bf16 map over [planes][rows][D] with 64 x 128 x 1 boxes, 128-byte swizzle.
-// Rows past `rows` of a plane read as zeros.
-bool make_map(CUtensorMap* m, void* base, int64_t D, int64_t rows, int64_t planes) {
+// 3D map over [planes][rows][D] with 128-byte x 128-row x 1 boxes (64 bf16 or
+// 128 e4m3 elements per row), 128-byte swizzle. Rows past `rows` of a plane
+// read as zeros.
+bool make_map(CUtensorMap* m, void* base, int64_t D, int64_t rows, int64_t planes,
+              bool e4m3 = false) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
+  const int64_t es_b = e4m3 ? 1 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)planes};
-  cuuint64_t strides[2] = {(cuuint64_t)(D * 2), (cuuint64_t)(rows * D * 2)};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)(D * es_b), (cuuint64_t)(rows * D * es_b)};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / es_b), 128, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
+  return enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base,
+             dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -158,8 +165,11 @@ struct sa_cache {
   int num_sms = 148;
   cudaStream_t create_stream = nullptr;
   int64_t F = 0, Lc = 0, R = 0, ntok = 0, sf = 0;
-  size_t esz = 2;
+  size_t esz = 2;   // q, k, v, out elements
+  size_t cesz = 2;  // cache and rotated-query elements (1 for e4m3)
   float scale = 0.f;
+  float* d_fp8_scale = nullptr;     // e4m3: [3][H] q, k, v scales (device)
+  std::vector<float> fp8_scale;     // host copy
   void* k_cache = nullptr;
   void* v_cache = nullptr;
   void* k_raw = nullptr;
@@ -227,7 +237,8 @@ void free_all(sa_cache* h) {
   if (h->copy_in) cudaStreamSynchronize(h->copy_in);
   if (h->copy_out) cudaStreamSynchronize(h->copy_out);
   void* ptrs[] = {h->k_cache, h->v_cache, h->k_raw, h->q_ws, h->htab, h->wtab, h->d_status,
-                  h->partials, h->stage[0], h->stage[1], h->stage[2], h->stage[3]};
+                  h->partials, h->stage[0], h->stage[1], h->stage[2], h->stage[3],
+                  h->d_fp8_scale};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   for (int s = 0; s < sa_cache::kSlots; ++s) {
@@ -328,14 +339,15 @@ sa_status sa_cache_create(const sa_config* cfg, sa_stream_t stream, sa_cache** o
   h->R = (int64_t)cfg->window_frames + cfg->chunk_frames;
   h->sf = h->F * cfg->sink_frames;
   h->ntok = h->sf + h->R * h->F;
-  h->esz = cfg->dtype == SA_BF16 ? 2 : 4;
+  h->esz = cfg->dtype == SA_F32 ? 4 : 2;
+  h->cesz = cfg->dtype == SA_BF16_E4M3 ? 1 : h->esz;
   h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : (float)(1.0 / sqrt((double)cfg->head_dim));
   h->frames_written.assign(cfg->batch, 0);
   h->pos_base.assign(cfg->batch, 0);
   const int64_t B = cfg->batch, H = cfg->heads, D = cfg->head_dim;
-  const size_t cache_bytes = (size_t)(B * H * h->ntok * D) * h->esz;
+  const size_t cache_bytes = (size_t)(B * H * h->ntok * D) * h->cesz;
   const size_t raw_bytes = (size_t)(B * H * std::max<int64_t>(h->sf, 1) * D) * h->esz;
-  const size_t ws_bytes = (size_t)(B * H * h->Lc * D) * h->esz;
+  const size_t ws_bytes = (size_t)(B * H * h->Lc * D) * h->cesz;
   const int dh2 = cfg->rope_dims[1] / 2, dw2 = cfg->rope_dims[2] / 2;
   cudaStream_t cs = h->create_stream;
   struct Alloc { void** p; size_t n; } allocs[] = {
@@ -379,7 +391,20 @@ sa_status sa_cache_create(const sa_config* cfg, sa_stream_t stream, sa_cache** o
     delete h;
     return cuda_fail(e, "table upload");
   }
-  if (cfg->dtype == SA_BF16) {
+  if (cfg->dtype == SA_BF16_E4M3) {  // per-head scales, all 1 until set
+    h->fp8_scale.assign((size_t)(3 * H), 1.f);
+    e = cudaMalloc(&h->d_fp8_scale, sizeof(float) * h->fp8_scale.size());
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(h->d_fp8_scale, h->fp8_scale.data(), sizeof(float) * h->fp8_scale.size(),
+                          cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) {
+      free_all(h);
+      delete h;
+      return cuda_fail(e, "fp8 scales");
+    }
+  }
+  if (cfg->dtype != SA_F32) {
     const int64_t max_units = B * H * ((h->Lc + 255) / 256);
     h->partials_bytes = sa::attend_partials_bytes((int)D, h->num_sms, max_units);
     e = cudaMalloc(&h->partials, h->partials_bytes);
@@ -400,9 +425,10 @@ sa_status sa_cache_create(const sa_config* cfg, sa_stream_t stream, sa_cache** o
       delete h;
       return cuda_fail(e, "cudaMalloc(partials)");
     }
-    if (!make_map(&h->tm_q, h->q_ws, D, h->Lc, B * H) ||
-        !make_map(&h->tm_k, h->k_cache, D, h->ntok, B * H) ||
-        !make_map(&h->tm_v, h->v_cache, D, h->ntok, B * H)) {
+    const bool f8 = cfg->dtype == SA_BF16_E4M3;
+    if (!make_map(&h->tm_q, h->q_ws, D, h->Lc, B * H, f8) ||
+        !make_map(&h->tm_k, h->k_cache, D, h->ntok, B * H, f8) ||
+        !make_map(&h->tm_v, h->v_cache, D, h->ntok, B * H, f8)) {
       free_all(h);
       delete h;
       return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
@@ -460,6 +486,7 @@ sa_status append_attend(sa_cache* h, const void* q, const void* k, const void* v
     memset(&p, 0, sizeof(p));
     p.q = q; p.k = k; p.v = v;
     p.q_ws = h->q_ws; p.k_cache = h->k_cache; p.v_cache = h->v_cache; p.k_raw = h->k_raw;
+    p.fp8_scale = h->d_fp8_scale;
     p.htab = h->htab; p.wtab = h->wtab;
     p.H = c.heads; p.D = c.head_dim; p.fw = c.frame_w; p.F = (int32_t)h->F; p.C = C;
     p.Lc = (int32_t)h->Lc; p.ntok = h->ntok; p.sf = h->sf;
@@ -498,13 +525,19 @@ sa_status append_attend(sa_cache* h, const void* q, const void* k, const void* v
   ap.scale_log2 = (float)((double)h->scale * 1.4426950408889634);
   ap.out = out; ap.q_ws = h->q_ws; ap.k_cache = h->k_cache; ap.v_cache = h->v_cache;
   ap.status = h->d_status;
+  ap.fp8 = c.dtype == SA_BF16_E4M3;
+  if (ap.fp8)
+    for (int hh = 0; hh < c.heads; ++hh) {
+      ap.inv_qk[hh] = 1.f / (h->fp8_scale[hh] * h->fp8_scale[c.heads + hh]);
+      ap.inv_v[hh] = 1.f / h->fp8_scale[2 * c.heads + hh];
+    }
   for (size_t i = 0; i < act.size(); ++i) {
     ap.stream_of[i] = act[order[i]];
     ap.n_keys[i] = (int32_t)plans[order[i]].n_keys;
   }
   prof_before(h, st, KIND_ATTEND);
   int n_att = 1;
-  cudaError_t e = c.dtype == SA_BF16
+  cudaError_t e = c.dtype != SA_F32
                       ? sa::launch_attend_tc_bf16(ap, c.head_dim, &h->tm_q, &h->tm_k, &h->tm_v,
                                                   h->partials, h->partials_bytes, h->num_sms, st,
                                                   &n_att)
@@ -549,6 +582,7 @@ sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream
     sa::RefreshParams p;
     memset(&p, 0, sizeof(p));
     p.k_cache = h->k_cache; p.k_raw = h->k_raw; p.htab = h->htab; p.wtab = h->wtab;
+    p.fp8_scale = h->d_fp8_scale; p.v_cache = h->v_cache;
     p.H = c.heads; p.D = c.head_dim; p.fw = c.frame_w; p.F = (int32_t)h->F; p.S = S;
     p.ntok = h->ntok; p.sf = h->sf;
     p.dt2 = dt2; p.dh2 = c.rope_dims[1] / 2; p.dw2 = c.rope_dims[2] / 2;
@@ -579,6 +613,31 @@ sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream
     h->kernels += 1;
   }
   for (size_t i = 0; i < todo.size(); ++i) h->pos_base[todo[i]] += deltas[i];
+  return SA_OK;
+}
+
+sa_status sa_cache_set_fp8_scales(sa_cache* h, const float* q_scale, const float* k_scale,
+                                  const float* v_scale) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (h->cfg.dtype != SA_BF16_E4M3)
+    return fail(SA_ERR_INVALID_ARG, "per-head fp8 scales need dtype SA_BF16_E4M3");
+  for (int b = 0; b < h->cfg.batch; ++b)
+    if (h->frames_written[b] > 0)
+      return fail(SA_ERR_STATE, "scales must be set before any stream holds a frame");
+  const int H = h->cfg.heads;
+  std::vector<float> sc((size_t)(3 * H), 1.f);
+  const float* src[3] = {q_scale, k_scale, v_scale};
+  for (int t = 0; t < 3; ++t)
+    for (int i = 0; i < H && src[t]; ++i) {
+      if (!(src[t][i] > 0.f) || !isfinite(src[t][i]))
+        return fail(SA_ERR_INVALID_ARG, "scale %d of tensor %d is not positive and finite", i, t);
+      sc[(size_t)t * H + i] = src[t][i];
+    }
+  cudaError_t e = cudaMemcpyAsync(h->d_fp8_scale, sc.data(), sizeof(float) * sc.size(),
+                                  cudaMemcpyHostToDevice, h->create_stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(h->create_stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8 scale upload");
+  h->fp8_scale = sc;
   return SA_OK;
 }
 
@@ -615,6 +674,7 @@ sa_status sa_sink_update(sa_cache* h, const void* k_new, const void* v_new, floa
     sa::RefreshParams p;
     memset(&p, 0, sizeof(p));
     p.k_cache = h->k_cache; p.k_raw = h->k_raw; p.htab = h->htab; p.wtab = h->wtab;
+    p.fp8_scale = h->d_fp8_scale; p.v_cache = h->v_cache;
     p.v_cache = h->v_cache; p.k_new = k_new; p.v_new = v_new; p.alpha = alpha; p.update = 1;
     p.H = c.heads; p.D = c.head_dim; p.fw = c.frame_w; p.F = (int32_t)h->F; p.S = S;
     p.ntok = h->ntok; p.sf = h->sf;
@@ -764,7 +824,7 @@ sa_status sa_cache_copy_out(const sa_cache* h, int32_t b, void* host_k, void* ho
   if (b < 0 || b >= h->cfg.batch) return fail(SA_ERR_INVALID_ARG, "stream index out of range");
   if (!host_k || !host_v) return fail(SA_ERR_INVALID_ARG, "host buffers must be non-NULL");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t n = (size_t)(h->cfg.heads * h->ntok * h->cfg.head_dim) * h->esz;
+  const size_t n = (size_t)(h->cfg.heads * h->ntok * h->cfg.head_dim) * h->cesz;
   cudaError_t e = cudaMemcpyAsync(host_k, static_cast<const char*>(h->k_cache) + n * b, n,
                                   cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess)
@@ -912,6 +972,8 @@ extern "C" sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cach
                                               const uint8_t* active, sa_stream_t stream) {
   sa_status st = validate_config(cfg);
   if (st != SA_OK) return st;
+  if (cfg->dtype == SA_BF16_E4M3)
+    return fail(SA_ERR_UNSUPPORTED, "the allocation-free entry runs SA_F32 and SA_BF16 caches");
   if (!k_cache || !v_cache || !frames_written || !pos_base || !q || !k || !v || !out)
     return fail(SA_ERR_INVALID_ARG, "cache buffers, stream state, q, k, v and out must be non-NULL");
   if (cfg->sink_frames > 0 && !k_raw)

@@ -16,6 +16,9 @@ from rolling_kv_cache_sa_b200.session import StreamSession
 BF16_MAX_ABS = 2e-2
 BF16_MEAN_ABS = 2e-3
 F32_MAX_ABS = 1e-4
+# e4m3 cache: q', k', v stored with 3 mantissa bits and P rounded to e4m3
+E4M3_MAX_ABS = 1e-1
+E4M3_MEAN_ABS = 1e-2
 
 
 def torch_dtype(w):
@@ -28,6 +31,8 @@ class Runner:
     def __init__(self, w):
         self.w = w
         self.cache = SACache(config_for(w))
+        if getattr(w, "fp8_scales", ()):
+            self.cache.set_fp8_scales(*w.fp8_scales)
         self.sess = StreamSession(self.cache, w.refresh_period)
         shape = (w.B, w.Lc, w.H, w.D)
         dt = torch_dtype(w)
@@ -89,12 +94,21 @@ def assert_rows(w, b, c, out_b, toks, heads=None):
     mx, mean, ref, got = compare_rows(w, b, c, out_b, toks, heads)
     log_line(f"{w.name} stream {b} chunk {c}: rows {len(toks) * (len(heads) if heads else w.H)} "
              f"max_abs {mx:.3e} mean_abs {mean:.3e}")
-    if w.dtype == "bf16":
+    if getattr(w, "cache", "") == "e4m3":
+        assert mx <= E4M3_MAX_ABS and mean <= E4M3_MEAN_ABS, (b, c, mx, mean)
+    elif w.dtype == "bf16":
         assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, (b, c, mx, mean)
     else:
         assert mx <= F32_MAX_ABS, (b, c, mx, mean)
     assert np.isfinite(got).all()
     return mx, mean
+
+
+def e4m3_ulp(x):
+    """Spacing of the e4m3 grid at |x| (3 mantissa bits; 2^-9 below 2^-6)."""
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return 2.0 ** (np.maximum(e, -6.0) - 3.0)
 
 
 def bf16_ulp(x):
@@ -116,6 +130,19 @@ def assert_cache(w, runner, b, c, sink_ulps=0):
     assert base == O.base_at(cfg, c)
     rows = np.concatenate([np.arange(s * w.F, (s + 1) * w.F) for s, f in enumerate(slot_frame)
                            if f >= 0]).astype(np.int64)
+    if getattr(w, "cache", "") == "e4m3":
+        # values: one e4m3 step (the GPU scales in fp32 before rounding);
+        # rotated keys: two steps of the rotation pair's magnitude
+        sk = runner.cache.scales[1][:, None, None]
+        sv = runner.cache.scales[2][:, None, None]
+        vr, vg = v_ref[:, rows], v_got[:, rows]
+        assert (np.abs(vg - vr) <= e4m3_ulp(vr * sv) / sv + 1e-12).all(), (b, c)
+        kr, kg = k_ref[:, rows], k_got[:, rows]
+        ak = np.abs(kr)
+        pm = np.maximum(ak[..., 0::2], ak[..., 1::2]).repeat(2, axis=-1)
+        kd = np.abs(kg - kr)
+        assert (kd <= 2 * e4m3_ulp(pm * sk) / sk + 1e-12).all(), (b, c, float(kd.max()))
+        return float(kd.max()) if kd.size else 0.0
     if sink_ulps and w.S > 0:
         srows = np.arange(w.S * w.F)
         vs_ref = v_ref[:, srows]

@@ -1,0 +1,99 @@
+"""e4m3 cache (SA_BF16_E4M3): bf16 inputs and output, rotated keys, values,
+rotated queries and P in e4m3 with per-head scales, both attention products
+on the tensor cores in fp8. Compared with the oracle's e4m3 storage mode
+(which mirrors every stored rounding, not P's): every output row on small
+ragged streams with refreshes and a sink update, sampled rows on the 512p
+workload, and the cache contents after every chunk."""
+import numpy as np
+import pytest
+import torch
+
+import inputgen as IG
+from gpu_harness import Runner, assert_cache, assert_rows, log_line, sample_tokens
+from inputgen.workloads import P512, Workload
+
+pytestmark = pytest.mark.gpu
+
+POW2 = ((1.0, 2.0, 0.5, 4.0), (2.0, 1.0, 4.0, 0.25), (1.0, 8.0, 0.5, 2.0))
+ODD = ((1.5, 3.0, 0.7, 12.0), (0.9, 2.5, 5.0, 0.3), (6.0, 1.25, 0.45, 3.3))
+FP8_SMALL = Workload("e4m3_8x16_b2", B=2, H=4, D=128, fh=8, fw=16, C=2, S=1, W=4, n_chunks=9,
+                     dtype="bf16", cache="e4m3", refresh_period=4, starts=(0, 2), fp8_scales=POW2)
+
+
+@pytest.fixture(autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+
+
+def _stream(w, rows="all", check_every=1, cache=True, sink_update=False):
+    r = Runner(w)
+    try:
+        if sink_update:
+            kn = torch.empty((w.B, w.S * w.F, w.H, w.D), dtype=torch.bfloat16, device="cuda")
+            vn = torch.empty_like(kn)
+        st = torch.cuda.current_stream().cuda_stream
+        for g in range(w.n_steps):
+            chunks = w.local_chunks(g)
+            if sink_update:
+                upd = [c > 0 and c % w.sink_update_period == 0 and c * w.C >= w.S for c in chunks]
+                if any(upd):
+                    coords = [IG.sink_update_chunk(c) if u else -1 for c, u in zip(chunks, upd)]
+                    IG.fill_device(w, list(range(w.B)), coords, IG.K, kn.data_ptr(), st,
+                                   n_tok=w.S * w.F)
+                    IG.fill_device(w, list(range(w.B)), coords, IG.V, vn.data_ptr(), st,
+                                   n_tok=w.S * w.F)
+                    r.cache.sink_update(kn, vn, w.sink_alpha, upd)
+            r.step(g)
+            if g % check_every:
+                continue
+            torch.cuda.synchronize()
+            out = r.out.float().cpu()
+            for b, c in enumerate(chunks):
+                if c < 0:
+                    continue
+                toks = list(range(w.Lc)) if rows == "all" else sample_tokens(w, seed=g * 7 + b)
+                assert_rows(w, b, c, out[b], toks)
+                if cache:
+                    assert_cache(w, r, b, c)
+        assert r.device_status() == 0
+    finally:
+        r.close()
+
+
+def test_e4m3_small_every_row():
+    _stream(FP8_SMALL)
+
+
+def test_e4m3_non_power_of_two_scales():
+    _stream(FP8_SMALL.with_(name="e4m3_odd_scales", fp8_scales=ODD))
+
+
+def test_e4m3_sink_update():
+    w = FP8_SMALL.with_(name="e4m3_sink_update", C=1, S=2, W=3, sink_update_period=3,
+                        sink_alpha=0.5)
+    _stream(w, sink_update=True)
+
+
+def test_e4m3_512p_sampled():
+    w = P512.with_(name="e4m3_512p", cache="e4m3", n_chunks=40)
+    _stream(w, rows="sample", check_every=13, cache=False)
+
+
+def test_e4m3_output_close_to_bf16_cache():
+    """The e4m3 cache's output stays near the bf16 cache's on the same inputs
+    (a property at any size: the two differ only by the e4m3 roundings)."""
+    w16 = P512.with_(name="bf16_ref", n_chunks=6)
+    w8 = w16.with_(name="e4m3_vs_bf16", cache="e4m3")
+    a, b = Runner(w16), Runner(w8)
+    try:
+        for g in range(w16.n_steps):
+            a.step(g)
+            b.step(g)
+        torch.cuda.synchronize()
+        d = (a.out.float() - b.out.float()).abs()
+        log_line(f"e4m3 vs bf16 cache 512p chunk 5: max {d.max().item():.3e} mean {d.mean().item():.3e}")
+        assert d.mean().item() < 1e-2 and d.max().item() < 2e-1
+    finally:
+        a.close()
+        b.close()
