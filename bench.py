@@ -35,7 +35,7 @@ METRIC = "streamed chunks/s and attention TFLOP/s (% of B200 BF16 peak) per conf
 # DRAM bytes (read + write) per launch of the attention kernel, from the ncu
 # capture summarised in profiles/ (512p, steady chunk with 7168 keys), keyed by
 # a hash of the kernel sources it was taken on: a changed kernel reports null.
-PROFILED_TRAFFIC = {"fff8e35f79fc94b1": 183.66e6}
+PROFILED_TRAFFIC = {"5f5b6d7179026db9": 173.32e6, "5f5b6d7179026db9/e4m3": 64.06e6}
 
 
 def attend_source_hash() -> str:
@@ -438,10 +438,13 @@ def main():
                      "duration": "mean of the library's CUDA events around each launch, on "
                                  "its launch stream, over the eager timed pass",
                      "traffic": PROFILED_TRAFFIC.get(attend_source_hash() + ("/e4m3" if f8 else "")),
-                     "traffic_note": "ncu dram read+write bytes of one steady-state launch "
-                                     "(7168 keys, cold L2); algorithmic minimum 113 MB; the "
-                                     "excess is split-unit fp32 partials written and read "
-                                     "back (~39 MB) and K/V re-reads past L2"},
+                     "traffic_note": ("ncu dram read+write bytes of one steady-state launch "
+                                      "(7168 keys, cold L2); algorithmic minimum 63 MB (e4m3 "
+                                      "Q', K', V in, bf16 O out)") if f8 else
+                                     ("ncu dram read+write bytes of one steady-state launch "
+                                      "(7168 keys, cold L2); algorithmic minimum 113 MB; the "
+                                      "excess is split-unit fp32 partials written and read "
+                                      "back and K/V re-reads past L2")},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
