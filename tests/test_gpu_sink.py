@@ -31,8 +31,11 @@ def _update_due(w, c):
     return c > 0 and c % w.sink_update_period == 0 and c * w.C >= w.S
 
 
+SINK_E4M3 = SINK_BF16.with_(name="sink_update_e4m3_8x12", cache="e4m3")
+
+
 @pytest.mark.parametrize("repin", [False, True], ids=["shift", "repin"])
-@pytest.mark.parametrize("w0", [SINK_BF16, SINK_F32], ids=lambda w: w.name)
+@pytest.mark.parametrize("w0", [SINK_BF16, SINK_F32, SINK_E4M3], ids=lambda w: w.name)
 def test_sink_update_and_modes_match_oracle(w0, repin):
     w = w0.with_(sink_repin=repin)
     r = Runner(w)

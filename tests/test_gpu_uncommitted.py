@@ -13,8 +13,8 @@ import torch
 
 import inputgen as IG
 import oracle as O
-from gpu_harness import (BF16_MAX_ABS, BF16_MEAN_ABS, F32_MAX_ABS, Runner, assert_cache,
-                         assert_rows, log_line)
+from gpu_harness import (BF16_MAX_ABS, BF16_MEAN_ABS, E4M3_MAX_ABS, E4M3_MEAN_ABS, F32_MAX_ABS,
+                         Runner, assert_cache, assert_rows, log_line)
 from inputgen import spec_for
 from inputgen.workloads import Workload
 
@@ -22,6 +22,9 @@ pytestmark = pytest.mark.gpu
 
 UNC_BF16 = Workload("uncommitted_bf16_8x12", B=2, H=4, D=128, fh=8, fw=12, C=2, S=1, W=4,
                     n_chunks=9, dtype="bf16", refresh_period=4, starts=(0, 3))
+UNC_E4M3 = UNC_BF16.with_(name="uncommitted_e4m3_8x12", cache="e4m3",
+                          fp8_scales=((1.0, 2.0, 0.5, 4.0), (2.0, 1.0, 4.0, 0.25),
+                                      (1.0, 8.0, 0.5, 2.0)))
 UNC_F32 = Workload("uncommitted_f32_8x8", B=1, H=2, D=64, fh=8, fw=8, C=1, S=1, W=2,
                    n_chunks=8, dtype="f32", refresh_period=4)
 
@@ -38,7 +41,7 @@ def _fill(r, w_draw, chunks):
         IG.fill_device(w_draw, list(range(r.w.B)), chunks, t, buf.data_ptr(), st)
 
 
-@pytest.mark.parametrize("w", [UNC_BF16, UNC_F32], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [UNC_BF16, UNC_F32, UNC_E4M3], ids=lambda w: w.name)
 def test_uncommitted_steps_then_commit(w):
     draws = [dataclasses.replace(w, seed=w.seed + 101 + i) for i in range(2)]
     cfg = O.cfg_for(w)
@@ -66,7 +69,9 @@ def test_uncommitted_steps_then_commit(w):
                     err = np.abs(got - ref)
                     log_line(f"{w.name} uncommitted stream {b} chunk {c}: max_abs {err.max():.3e} "
                              f"mean_abs {err.mean():.3e}")
-                    if w.dtype == "bf16":
+                    if w.cache == "e4m3":
+                        assert err.max() <= E4M3_MAX_ABS and err.mean() <= E4M3_MEAN_ABS, (b, c)
+                    elif w.dtype == "bf16":
                         assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (b, c)
                     else:
                         assert err.max() <= F32_MAX_ABS, (b, c, err.max())
