@@ -254,6 +254,60 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
     for (int i = 0; i < BN; ++i)
       if (i >= valid) sv[i] = __float_as_uint(-INFINITY);
   }
+  if (F8 && !first) {
+    // e4m3 operands: optimistic pass with the running max, the tile max
+    // tracked on the way; P stays in registers until the max is checked and
+    // is then published whole. (With the shorter fp8 MMAs, taking the max off
+    // the critical path gains more than starting the first half of PV early;
+    // for bf16 it is the other way round.)
+    constexpr int kW = BN / 4;
+    uint32_t wo[kW];
+    const float2 sl2o = make_float2(sl2, sl2), nmo = make_float2(-m, -m);
+    float2 lo[4];
+    float mo[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) lo[i] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mo[i] = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < BN / 2; ++e) {
+      const float s0 = __uint_as_float(sv[2 * e]), s1 = __uint_as_float(sv[2 * e + 1]);
+      mo[e & 7] = ptx::fmax3(mo[e & 7], s0, s1);
+      const float2 x = __ffma2_rn(make_float2(s0, s1), sl2o, nmo);
+      const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+      lo[e & 3] = __fadd2_rn(lo[e & 3], pe);
+      const uint32_t pp = ptx::pack_e4m3x2(pe.x, pe.y);
+      if (e & 1)
+        wo[e >> 1] |= pp << 16;
+      else
+        wo[e >> 1] = pp;
+    }
+    const float tm = ptx::fmax3(ptx::fmax3(mo[0], mo[1], mo[2]), ptx::fmax3(mo[3], mo[4], mo[5]),
+                                fmaxf(mo[6], mo[7])) * sl2;
+    if (!__any_sync(0xffffffffu, tm > m + 8.0f)) {
+#pragma unroll
+      for (int q = 0; q < BN / 32; ++q) ptx::tmem_st8u(sbuf + (uint32_t)(q * 8), wo + q * 8);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar_pa);
+      ptx::mbar_arrive(bar_pb);
+      const float2 l2 = __fadd2_rn(__fadd2_rn(lo[0], lo[1]), __fadd2_rn(lo[2], lo[3]));
+      l += l2.x + l2.y;
+      return true;
+    }
+    // rare: nothing is stored yet, so S is intact in TMEM; take the exact path
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) ptx::tmem_ld32u(sbuf + (uint32_t)c * 32u, sv + c * 32);
+    ptx::tmem_wait_ld_dep(sv);
+    ptx::tmem_wait_ld_dep(sv + 32);
+    ptx::tmem_wait_ld_dep(sv + 64);
+    ptx::tmem_wait_ld_dep(sv + 96);
+    if (valid < BN) {
+#pragma unroll
+      for (int i = 0; i < BN; ++i)
+        if (i >= valid) sv[i] = __float_as_uint(-INFINITY);
+    }
+  }
   float mx[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) mx[i] = fmaxf(__uint_as_float(sv[i]), __uint_as_float(sv[i + 8]));

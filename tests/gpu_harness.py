@@ -17,8 +17,12 @@ BF16_MAX_ABS = 2e-2
 BF16_MEAN_ABS = 2e-3
 F32_MAX_ABS = 1e-4
 # e4m3 cache: q', k', v stored with 3 mantissa bits and P rounded to e4m3
+# (not mirrored by the oracle; relative error <= 2^-4 per element). Diffuse
+# attention (>= 30 effective keys): independent errors give ~0.05 -> 0.1.
+# Worst case, rows dominated by a few keys: 2^-4 * max|v|.
 E4M3_MAX_ABS = 1e-1
 E4M3_MEAN_ABS = 1e-2
+E4M3_WORST_MAX_ABS = 2.0 ** -4 * 6.0  # |v| <= 6 for the generator's N(0,1)
 
 
 def torch_dtype(w):
@@ -90,12 +94,12 @@ def log_line(text):
             f.write(text + "\n")
 
 
-def assert_rows(w, b, c, out_b, toks, heads=None):
+def assert_rows(w, b, c, out_b, toks, heads=None, max_abs=None):
     mx, mean, ref, got = compare_rows(w, b, c, out_b, toks, heads)
     log_line(f"{w.name} stream {b} chunk {c}: rows {len(toks) * (len(heads) if heads else w.H)} "
              f"max_abs {mx:.3e} mean_abs {mean:.3e}")
     if getattr(w, "cache", "") == "e4m3":
-        assert mx <= E4M3_MAX_ABS and mean <= E4M3_MEAN_ABS, (b, c, mx, mean)
+        assert mx <= (max_abs or E4M3_MAX_ABS) and mean <= E4M3_MEAN_ABS, (b, c, mx, mean)
     elif w.dtype == "bf16":
         assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS, (b, c, mx, mean)
     else:
