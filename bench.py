@@ -53,7 +53,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", default="512p_32x32_h24")
+    ap.add_argument("--workload", default="512p_32x32_h24",
+                    help="workload name, or C1..C5 for the five configurations in order")
     ap.add_argument("--cache", default="", choices=["", "e4m3"],
                     help="e4m3: bf16 in/out with an e4m3 K'/V cache and fp8 attention MMAs")
     ap.add_argument("--no-e2e", action="store_true")
@@ -208,8 +209,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    from inputgen.workloads import BY_NAME
-    w = BY_NAME[args.workload]
+    from inputgen.workloads import ALL, BY_NAME
+    # C1..C5: the five configurations in order (tiny fp32, 512p, 480x832 ragged,
+    # 1280x704, long-stream stress)
+    aliases = {f"C{i + 1}": wl.name for i, wl in enumerate(ALL)}
+    w = BY_NAME[aliases.get(args.workload, args.workload)]
     if args.chunks:
         w = w.with_(n_chunks=args.chunks)
     if args.cache:

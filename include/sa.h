@@ -201,6 +201,27 @@ sa_status sa_append_attend_host_async(sa_cache* h, const void* q, const void* k,
  * has completed (and with them the computations they follow). */
 sa_status sa_host_wait(sa_cache* h);
 
+/* ---- checkpoint / resume ---- */
+
+/* Bytes of a handle's checkpoint: a header (configuration, per-stream
+ * frames_written and pos_base, sink mode, e4m3 scales) followed by the K' and
+ * V cache and the raw sink keys. */
+sa_status sa_cache_export_size(const sa_cache* h, size_t* bytes);
+
+/* Writes the checkpoint into the host buffer dst (cap >= export size;
+ * SA_ERR_INVALID_ARG otherwise). Copies on `stream` after the work queued
+ * before it, then synchronises `stream`. The rotated-query workspace and the
+ * attention's split-unit counters are not part of it (rewritten by every
+ * call; zero between calls). A stream's continuation from an imported
+ * checkpoint is bit-identical to the original's. */
+sa_status sa_cache_export(const sa_cache* h, void* dst, size_t cap, sa_stream_t stream);
+
+/* Restores a checkpoint written by sa_cache_export into a handle created
+ * with the same configuration (SA_ERR_INVALID_ARG for another configuration,
+ * a wrong size or a damaged header; nothing changes then). Copies on
+ * `stream` and synchronises it. */
+sa_status sa_cache_import(sa_cache* h, const void* src, size_t size, sa_stream_t stream);
+
 /* ---- introspection (tests, benchmarks) ---- */
 
 /* frames_written and pos_base of stream b (host bookkeeping; no sync). */

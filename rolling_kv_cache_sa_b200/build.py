@@ -30,7 +30,7 @@ def is_stale() -> bool:
 
 
 def build(verbose: bool = False) -> str:
-    cmd = ["nvcc", *NVCC_FLAGS, *sources(), "-o", LIB, "-lcuda"]
+    cmd = ["nvcc", *NVCC_FLAGS, *sources(), "-o", LIB, "-lcuda", "-ldl"]
     if verbose:
         print(" ".join(cmd))
     r = subprocess.run(cmd, capture_output=True, text=True)

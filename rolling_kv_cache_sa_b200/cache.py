@@ -122,6 +122,22 @@ def sa_host_wait(h: int):
     check(lib().sa_host_wait(h), "sa_host_wait")
 
 
+def sa_cache_export(h: int, stream: Optional[torch.cuda.Stream] = None) -> np.ndarray:
+    """The handle's checkpoint as a uint8 host array."""
+    n = ctypes.c_size_t()
+    check(lib().sa_cache_export_size(h, ctypes.byref(n)), "sa_cache_export_size")
+    buf = np.empty(n.value, dtype=np.uint8)
+    check(lib().sa_cache_export(h, buf.ctypes.data, n.value, _stream_ptr(stream)),
+          "sa_cache_export")
+    return buf
+
+
+def sa_cache_import(h: int, blob: np.ndarray, stream: Optional[torch.cuda.Stream] = None):
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    check(lib().sa_cache_import(h, blob.ctypes.data, blob.size, _stream_ptr(stream)),
+          "sa_cache_import")
+
+
 def sa_stream_state(h: int, b: int):
     fw, base = ctypes.c_int64(), ctypes.c_int64()
     check(lib().sa_stream_state(h, b, ctypes.byref(fw), ctypes.byref(base)), "sa_stream_state")
@@ -240,6 +256,19 @@ class SACache:
 
     def host_wait(self):
         sa_host_wait(self.h)
+
+    def export(self, stream=None) -> np.ndarray:
+        """Checkpoint (cache contents and stream state) as a host byte array."""
+        return sa_cache_export(self.h, stream)
+
+    def import_(self, blob, stream=None):
+        """Restores a checkpoint of a handle with the same configuration."""
+        sa_cache_import(self.h, blob, stream)
+        if self.fp8:  # scales travel with the checkpoint
+            hdr = 8 + 4 + 4 + ctypes.sizeof(sa_config) + 24
+            off = hdr + 16 * self.B
+            self.scales = np.frombuffer(np.asarray(blob, np.uint8)[off:off + 12 * self.H].tobytes(),
+                                        dtype=np.float32).reshape(3, self.H).astype(np.float64)
 
     def set_fp8_scales(self, q_scale=None, k_scale=None, v_scale=None):
         """Per-head scales of an e4m3 cache (before the first chunk)."""

@@ -21,6 +21,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 
 namespace {
@@ -200,6 +202,15 @@ struct sa_cache {
 };
 
 namespace {
+
+// NVTX range around a library call or launch (a no-op unless a profiler is
+// attached): sa.append, sa.attend, sa.refresh, sa.sink_update.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Base that the sink's temporal positions are taken against: t = f - base.
 // Shift: the stream's base (the sink moves with every rebase). Re-pin: a
@@ -506,6 +517,7 @@ sa_status append_attend(sa_cache* h, const void* q, const void* k, const void* v
         }
       }
     }
+    NvtxRange nv("sa.append");
     prof_before(h, st, KIND_APPEND);
     cudaError_t e = sa::launch_append(p, c.dtype, h->num_sms, st);
     prof_after(h, st);
@@ -535,6 +547,7 @@ sa_status append_attend(sa_cache* h, const void* q, const void* k, const void* v
     ap.stream_of[i] = act[order[i]];
     ap.n_keys[i] = (int32_t)plans[order[i]].n_keys;
   }
+  NvtxRange nv("sa.attend");
   prof_before(h, st, KIND_ATTEND);
   int n_att = 1;
   cudaError_t e = c.dtype != SA_F32
@@ -606,6 +619,7 @@ sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream
           p.scs[a * S + s][j] = make_float2((float)cos(ang), (float)sin(ang));
         }
     }
+    NvtxRange nv("sa.refresh");
     prof_before(h, st, KIND_REFRESH);
     cudaError_t e = sa::launch_refresh(p, c.dtype, h->num_sms, st);
     prof_after(h, st);
@@ -693,6 +707,7 @@ sa_status sa_sink_update(sa_cache* h, const void* k_new, const void* v_new, floa
           p.scs[a * S + s][j] = make_float2((float)cos(ang), (float)sin(ang));
         }
     }
+    NvtxRange nv("sa.sink_update");
     prof_before(h, st, KIND_REFRESH);
     cudaError_t e = sa::launch_refresh(p, c.dtype, h->num_sms, st);
     prof_after(h, st);
@@ -806,6 +821,113 @@ sa_status sa_host_wait(sa_cache* h) {
   if (h->copy_in) e = cudaStreamSynchronize(h->copy_in);
   if (e == cudaSuccess && h->copy_out) e = cudaStreamSynchronize(h->copy_out);
   if (e != cudaSuccess) return cuda_fail(e, "host pipeline wait");
+  return SA_OK;
+}
+
+namespace {
+// Checkpoint header; followed by frames_written[B], pos_base[B] (int64),
+// the e4m3 scales [3H] (float, e4m3 caches only), then K', V, raw sink keys.
+struct CkptHeader {
+  char magic[8];  // "SACKPT01"
+  int32_t abi;
+  int32_t sink_mode;
+  sa_config cfg;
+  uint64_t cache_bytes, raw_bytes, total_bytes;
+};
+
+void ckpt_sizes(const sa_cache* h, size_t& meta, size_t& cache, size_t& raw, size_t& total) {
+  const sa_config& c = h->cfg;
+  cache = (size_t)(c.batch * (int64_t)c.heads * h->ntok * c.head_dim) * h->cesz;
+  raw = (size_t)(c.batch * (int64_t)c.heads * std::max<int64_t>(h->sf, 1) * c.head_dim) * h->esz;
+  meta = sizeof(CkptHeader) + 2 * sizeof(int64_t) * (size_t)c.batch +
+         (c.dtype == SA_BF16_E4M3 ? sizeof(float) * 3 * (size_t)c.heads : 0);
+  meta = (meta + 255) & ~(size_t)255;
+  total = meta + 2 * cache + raw;
+}
+}  // namespace
+
+sa_status sa_cache_export_size(const sa_cache* h, size_t* bytes) {
+  if (!h || !bytes) return fail(SA_ERR_INVALID_ARG, "handle and bytes must be non-NULL");
+  size_t meta, cache, raw, total;
+  ckpt_sizes(h, meta, cache, raw, total);
+  *bytes = total;
+  return SA_OK;
+}
+
+sa_status sa_cache_export(const sa_cache* h, void* dst, size_t cap, sa_stream_t stream) {
+  if (!h || !dst) return fail(SA_ERR_INVALID_ARG, "handle and dst must be non-NULL");
+  size_t meta, cache, raw, total;
+  ckpt_sizes(h, meta, cache, raw, total);
+  if (cap < total) return fail(SA_ERR_INVALID_ARG, "checkpoint needs %zu bytes, got %zu", total, cap);
+  char* out = static_cast<char*>(dst);
+  memset(out, 0, meta);
+  CkptHeader hd;
+  memset(&hd, 0, sizeof(hd));
+  memcpy(hd.magic, "SACKPT01", 8);
+  hd.abi = SA_ABI_VERSION;
+  hd.sink_mode = h->sink_mode;
+  hd.cfg = h->cfg;
+  hd.cache_bytes = cache;
+  hd.raw_bytes = raw;
+  hd.total_bytes = total;
+  memcpy(out, &hd, sizeof(hd));
+  const size_t B = (size_t)h->cfg.batch;
+  memcpy(out + sizeof(hd), h->frames_written.data(), sizeof(int64_t) * B);
+  memcpy(out + sizeof(hd) + sizeof(int64_t) * B, h->pos_base.data(), sizeof(int64_t) * B);
+  if (h->cfg.dtype == SA_BF16_E4M3)
+    memcpy(out + sizeof(hd) + 2 * sizeof(int64_t) * B, h->fp8_scale.data(),
+           sizeof(float) * h->fp8_scale.size());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(out + meta, h->k_cache, cache, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(out + meta + cache, h->v_cache, cache, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(out + meta + 2 * cache, h->k_raw, raw, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "checkpoint export");
+  return SA_OK;
+}
+
+sa_status sa_cache_import(sa_cache* h, const void* src, size_t size, sa_stream_t stream) {
+  if (!h || !src) return fail(SA_ERR_INVALID_ARG, "handle and src must be non-NULL");
+  size_t meta, cache, raw, total;
+  ckpt_sizes(h, meta, cache, raw, total);
+  if (size != total) return fail(SA_ERR_INVALID_ARG, "checkpoint of %zu bytes, expected %zu", size, total);
+  const char* in = static_cast<const char*>(src);
+  CkptHeader hd;
+  memcpy(&hd, in, sizeof(hd));
+  if (memcmp(hd.magic, "SACKPT01", 8) != 0 || hd.abi != SA_ABI_VERSION)
+    return fail(SA_ERR_INVALID_ARG, "not a checkpoint of this library version");
+  if (memcmp(&hd.cfg, &h->cfg, sizeof(sa_config)) != 0 || hd.cache_bytes != cache ||
+      hd.raw_bytes != raw || hd.total_bytes != total)
+    return fail(SA_ERR_INVALID_ARG, "checkpoint of another configuration");
+  if (hd.sink_mode != SA_SINK_SHIFT && hd.sink_mode != SA_SINK_REPIN)
+    return fail(SA_ERR_INVALID_ARG, "damaged checkpoint header");
+  const size_t B = (size_t)h->cfg.batch;
+  std::vector<int64_t> fw(B), pb(B);
+  memcpy(fw.data(), in + sizeof(hd), sizeof(int64_t) * B);
+  memcpy(pb.data(), in + sizeof(hd) + sizeof(int64_t) * B, sizeof(int64_t) * B);
+  for (size_t b = 0; b < B; ++b)
+    if (fw[b] < 0 || fw[b] % h->cfg.chunk_frames != 0 || pb[b] < 0 || pb[b] > fw[b])
+      return fail(SA_ERR_INVALID_ARG, "damaged checkpoint stream state");
+  std::vector<float> sc = h->fp8_scale;
+  if (h->cfg.dtype == SA_BF16_E4M3)
+    memcpy(sc.data(), in + sizeof(hd) + 2 * sizeof(int64_t) * B, sizeof(float) * sc.size());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(h->k_cache, in + meta, cache, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(h->v_cache, in + meta + cache, cache, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(h->k_raw, in + meta + 2 * cache, raw, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && h->cfg.dtype == SA_BF16_E4M3)
+    e = cudaMemcpyAsync(h->d_fp8_scale, sc.data(), sizeof(float) * sc.size(),
+                        cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "checkpoint import");
+  h->frames_written = fw;
+  h->pos_base = pb;
+  h->sink_mode = hd.sink_mode;
+  h->fp8_scale = sc;
   return SA_OK;
 }
 
