@@ -15,6 +15,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -43,6 +44,20 @@ sa_status cuda_fail(cudaError_t e, const char* what) {
   if (e == cudaErrorMemoryAllocation)
     return fail(SA_ERR_OOM, "%s: %s", what, cudaGetErrorString(e));
   return fail(SA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Host fault injection for tests of the error paths (no GPU fault involved),
+// read from SA_FAULT when a handle is created: "alloc" makes the cache
+// allocation report out-of-memory; "launch" makes every hot call report a
+// launch failure before anything is launched; "launch_once" does so once.
+enum { FAULT_NONE = 0, FAULT_ALLOC = 1, FAULT_LAUNCH = 2, FAULT_LAUNCH_ONCE = 3 };
+int fault_from_env() {
+  const char* f = getenv("SA_FAULT");
+  if (!f) return FAULT_NONE;
+  if (!strcmp(f, "alloc")) return FAULT_ALLOC;
+  if (!strcmp(f, "launch")) return FAULT_LAUNCH;
+  if (!strcmp(f, "launch_once")) return FAULT_LAUNCH_ONCE;
+  return FAULT_NONE;
 }
 
 // ---------------------------------------------------------------- config
@@ -176,6 +191,7 @@ struct sa_cache {
   void* v_cache = nullptr;
   void* k_raw = nullptr;
   int32_t sink_mode = SA_SINK_SHIFT;  // how the sink's positions follow a refresh
+  int fault = 0;                      // injected host fault (SA_FAULT), tests only
   void* q_ws = nullptr;
   float2* htab = nullptr;
   float2* wtab = nullptr;
@@ -361,6 +377,12 @@ sa_status sa_cache_create(const sa_config* cfg, sa_stream_t stream, sa_cache** o
   const size_t ws_bytes = (size_t)(B * H * h->Lc * D) * h->cesz;
   const int dh2 = cfg->rope_dims[1] / 2, dw2 = cfg->rope_dims[2] / 2;
   cudaStream_t cs = h->create_stream;
+  h->fault = fault_from_env();
+  if (h->fault == FAULT_ALLOC) {
+    free_all(h);
+    delete h;
+    return cuda_fail(cudaErrorMemoryAllocation, "cudaMalloc (injected by SA_FAULT=alloc)");
+  }
   struct Alloc { void** p; size_t n; } allocs[] = {
       {&h->k_cache, cache_bytes}, {&h->v_cache, cache_bytes}, {&h->k_raw, raw_bytes},
       {&h->q_ws, ws_bytes},
@@ -490,6 +512,10 @@ sa_status append_attend(sa_cache* h, const void* q, const void* k, const void* v
     if (s != SA_OK) return s;
   }
   const int C = c.chunk_frames, dt2 = c.rope_dims[0] / 2;
+  if (h->fault == FAULT_LAUNCH || h->fault == FAULT_LAUNCH_ONCE) {
+    if (h->fault == FAULT_LAUNCH_ONCE) h->fault = FAULT_NONE;
+    return cuda_fail(cudaErrorLaunchFailure, "append launch (injected by SA_FAULT)");
+  }
   // ---- K1: fused RoPE + append, up to kMaxEntries (stream, frame) entries per launch
   const int per_launch = std::max(1, sa::kMaxEntries / C);
   for (size_t s0 = 0; s0 < act.size(); s0 += per_launch) {

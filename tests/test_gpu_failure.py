@@ -1,7 +1,9 @@
 """Failure detection on the GPU without any fault: a bounded device wait on a
 barrier that nothing completes runs out, the host reads SA_ERR_DEVICE_TIMEOUT,
 a second waiter leaves through the abort flag, and the CUDA context stays
-usable (a cache created afterwards still matches the oracle)."""
+usable (a cache created afterwards still matches the oracle). Host-injected
+failures (SA_FAULT) take the allocation and launch error paths: the status is
+reported, nothing changes, and the next call succeeds."""
 import pytest
 import torch
 
@@ -42,5 +44,36 @@ def test_bounded_wait_expires_and_context_survives():
         assert r.cache.device_status() == 0
         out = r.out.float().cpu()
         assert_rows(w, 0, chunks[0], out[0], list(range(w.Lc)))
+    finally:
+        r.close()
+
+
+def test_injected_allocation_failure(monkeypatch):
+    from rolling_kv_cache_sa_b200 import SACache, SAError, config_for
+    from rolling_kv_cache_sa_b200._lib import SA_ERR_OOM
+    monkeypatch.setenv("SA_FAULT", "alloc")
+    with pytest.raises(SAError) as e:
+        SACache(config_for(TINY_F32))
+    assert e.value.status == SA_ERR_OOM
+
+
+def test_injected_launch_failure_leaves_state_and_recovers(monkeypatch):
+    from gpu_harness import Runner
+    from rolling_kv_cache_sa_b200 import SAError
+    from rolling_kv_cache_sa_b200._lib import SA_ERR_CUDA
+    monkeypatch.setenv("SA_FAULT", "launch_once")
+    w = TINY_F32
+    r = Runner(w)
+    monkeypatch.delenv("SA_FAULT")
+    try:
+        with pytest.raises(SAError) as e:
+            r.step(0)
+        assert e.value.status == SA_ERR_CUDA
+        assert r.cache.state(0) == (0, 0)
+        for g in range(3):
+            chunks, _ = r.step(g)
+        torch.cuda.synchronize()
+        assert r.cache.state(0)[0] == 3 * w.C
+        assert_rows(w, 0, chunks[0], r.out.float().cpu()[0], list(range(w.Lc)))
     finally:
         r.close()
