@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
   SA_OK = 0,
   SA_ERR_INVALID_ARG = 1,    /* a pointer, size or configuration is invalid */
-  SA_ERR_UNSUPPORTED = 2,    /* no B200-class device, or a shape this build does not run */
+  SA_ERR_UNSUPPORTED = 2,    /* no B200-class device, or a shape the library does not run */
   SA_ERR_OOM = 3,            /* device or pinned-host allocation failed */
   SA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
   SA_ERR_STATE = 5,          /* call not valid in the handle's current state */
