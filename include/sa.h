@@ -311,6 +311,12 @@ sa_status sa_profile_launches(const sa_cache* h, int64_t* launches);
 sa_status sa_cache_set_fp8_scales(sa_cache* h, const float* q_scale, const float* k_scale,
                                   const float* v_scale);
 
+/* Copies the handle's per-head scales of an SA_BF16_E4M3 cache to host arrays
+ * of H floats each (any may be NULL); SA_ERR_INVALID_ARG for another dtype.
+ * Host only. */
+sa_status sa_cache_get_fp8_scales(const sa_cache* h, float* q_scale, float* k_scale,
+                                  float* v_scale);
+
 /* Sink position modes (sa_cache_set_sink_mode). */
 #define SA_SINK_SHIFT 0 /* a refresh rebases the sink with every other position: scores invariant */
 #define SA_SINK_REPIN 1 /* after a refresh the sink sits right before the oldest window frame */

@@ -23,7 +23,7 @@ EXPORTED = (
     "sa_profile_end", "sa_last_error_string", "sa_abi_version", "sa_append_attend_noalloc",
     "sa_profile_launches", "sa_wait_probe", "sa_attend", "sa_cache_set_sink_mode",
     "sa_sink_update", "sa_append_attend_host_async", "sa_host_wait", "sa_cache_set_fp8_scales",
-    "sa_cache_export_size", "sa_cache_export", "sa_cache_import",
+    "sa_cache_export_size", "sa_cache_export", "sa_cache_import", "sa_cache_get_fp8_scales",
 )
 
 
@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
         "sa_attend": [vp, vp, vp, vp, vp, vp, vp],
         "sa_cache_set_sink_mode": [vp, i32],
         "sa_cache_set_fp8_scales": [vp, vp, vp, vp],
+        "sa_cache_get_fp8_scales": [vp, vp, vp, vp],
         "sa_cache_export_size": [vp, P(ctypes.c_size_t)],
         "sa_cache_export": [vp, vp, ctypes.c_size_t, vp],
         "sa_cache_import": [vp, vp, ctypes.c_size_t, vp],

@@ -78,6 +78,13 @@ def sa_cache_set_fp8_scales(h: int, q_scale=None, k_scale=None, v_scale=None):
     check(lib().sa_cache_set_fp8_scales(h, *arrs), "sa_cache_set_fp8_scales")
 
 
+def sa_cache_get_fp8_scales(h: int, heads: int) -> np.ndarray:
+    """The handle's e4m3 scales as a [3, H] array (q, k, v)."""
+    arrs = [(ctypes.c_float * heads)() for _ in range(3)]
+    check(lib().sa_cache_get_fp8_scales(h, *arrs), "sa_cache_get_fp8_scales")
+    return np.array([list(a) for a in arrs], dtype=np.float64)
+
+
 def sa_sink_update(h: int, k_new: torch.Tensor, v_new: torch.Tensor, alpha: float, active=None,
                    stream: Optional[torch.cuda.Stream] = None, batch: int = 0):
     check(lib().sa_sink_update(h, k_new.data_ptr(), v_new.data_ptr(), ctypes.c_float(alpha),
@@ -264,11 +271,8 @@ class SACache:
     def import_(self, blob, stream=None):
         """Restores a checkpoint of a handle with the same configuration."""
         sa_cache_import(self.h, blob, stream)
-        if self.fp8:  # scales travel with the checkpoint
-            hdr = 8 + 4 + 4 + ctypes.sizeof(sa_config) + 24
-            off = hdr + 16 * self.B
-            self.scales = np.frombuffer(np.asarray(blob, np.uint8)[off:off + 12 * self.H].tobytes(),
-                                        dtype=np.float32).reshape(3, self.H).astype(np.float64)
+        if self.fp8:  # the scales travel with the checkpoint
+            self.scales = sa_cache_get_fp8_scales(self.h, self.H)
 
     def set_fp8_scales(self, q_scale=None, k_scale=None, v_scale=None):
         """Per-head scales of an e4m3 cache (before the first chunk)."""

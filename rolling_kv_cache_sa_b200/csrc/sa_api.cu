@@ -681,6 +681,18 @@ sa_status sa_cache_set_fp8_scales(sa_cache* h, const float* q_scale, const float
   return SA_OK;
 }
 
+sa_status sa_cache_get_fp8_scales(const sa_cache* h, float* q_scale, float* k_scale,
+                                  float* v_scale) {
+  if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
+  if (h->cfg.dtype != SA_BF16_E4M3)
+    return fail(SA_ERR_INVALID_ARG, "per-head fp8 scales need dtype SA_BF16_E4M3");
+  float* dst[3] = {q_scale, k_scale, v_scale};
+  const size_t H = (size_t)h->cfg.heads;
+  for (int t = 0; t < 3; ++t)
+    if (dst[t]) memcpy(dst[t], h->fp8_scale.data() + t * H, sizeof(float) * H);
+  return SA_OK;
+}
+
 sa_status sa_cache_set_sink_mode(sa_cache* h, int32_t mode) {
   if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
   if (mode != SA_SINK_SHIFT && mode != SA_SINK_REPIN)
