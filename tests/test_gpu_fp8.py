@@ -90,6 +90,31 @@ def test_e4m3_512p_sampled():
     _stream(w, rows="sample", check_every=13, cache=False)
 
 
+def test_e4m3_long_stream_no_drift():
+    """1,500 chunks with a refresh every 64: ring keys are requantised at each
+    refresh they cross (at most one in their lifetime), sink keys re-derived
+    from bf16 raw keys, so late chunks match the oracle like early ones."""
+    w = Workload("e4m3_long_b2", B=2, H=4, D=128, fh=8, fw=16, C=2, S=1, W=6, n_chunks=1500,
+                 dtype="bf16", cache="e4m3", refresh_period=64, starts=(0, 5),
+                 outlier_frac=0.01, outlier_scale=20.0)
+    r = Runner(w)
+    checks = {3, 64, 65, 700, 1427, w.n_steps - 1}
+    try:
+        for g in range(w.n_steps):
+            chunks, _ = r.step(g)
+            if g in checks:
+                torch.cuda.synchronize()
+                out = r.out.float().cpu()
+                for b, c in enumerate(chunks):
+                    if c >= 0:
+                        assert_rows(w, b, c, out[b], sample_tokens(w, seed=g + b),
+                                    max_abs=E4M3_WORST_MAX_ABS)
+                        assert_cache(w, r, b, c)
+        assert r.device_status() == 0
+    finally:
+        r.close()
+
+
 def test_e4m3_output_close_to_bf16_cache():
     """The e4m3 cache's output stays near the bf16 cache's on the same inputs
     (a property at any size: the two differ only by the e4m3 roundings)."""
