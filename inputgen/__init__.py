@@ -17,6 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
 Q, K, V = 0, 1, 2
+GATE, BETA = 4, 5
 SINK_UPDATE_CHUNK0 = 1 << 40  # chunk coordinate base of sink-update blocks (sa_inputgen.h)
 F32, BF16 = 0, 1
 
@@ -47,6 +48,10 @@ def lib():
                                      ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
         L.ig_fill_device.restype = ctypes.c_int
+        L.ig_fill_gates_host.argtypes = [ctypes.POINTER(Spec), ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                         ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
+        L.ig_fill_gates_host.restype = ctypes.c_int
         _LIB = L
     return _LIB
 
@@ -77,6 +82,21 @@ def fill_host(w: Workload, stream: int, chunk: int, tensor: int, tok0: int = 0,
     if rc != 0:
         raise RuntimeError(f"ig_fill_host failed ({rc})")
     return out
+
+
+def fill_gates_host(w: Workload, stream: int, chunk: int, g_scale: float, tok0: int = 0,
+                    n_tok: int | None = None):
+    """Gated DeltaNet gate inputs of one chunk: (g, beta), float32 [n_tok, H]
+    each; g = log decay in (-g_scale, 0), beta in (0, 1)."""
+    n_tok = w.Lc - tok0 if n_tok is None else n_tok
+    g = np.empty((n_tok, w.H), dtype=np.float32)
+    beta = np.empty((n_tok, w.H), dtype=np.float32)
+    sp = spec_for(w)
+    rc = lib().ig_fill_gates_host(ctypes.byref(sp), stream, chunk, tok0, n_tok, w.H,
+                                  ctypes.c_float(g_scale), g.ctypes.data, beta.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"ig_fill_gates_host failed ({rc})")
+    return g, beta
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:

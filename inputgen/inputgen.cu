@@ -36,6 +36,23 @@ int ig_fill_host(const ig_spec* sp, int64_t stream, int64_t chunk, int32_t tenso
   return 0;
 }
 
+/* Gate inputs of tokens [tok0, tok0+n_tok) of one chunk of one stream:
+ * g and beta, [n_tok][H] fp32 each (either may be NULL). Returns 0, or -1 on a
+ * bad argument. */
+int ig_fill_gates_host(const ig_spec* sp, int64_t stream, int64_t chunk, int64_t tok0,
+                       int64_t n_tok, int32_t H, float g_scale, float* g, float* beta) {
+  if (!sp || H <= 0 || n_tok < 0 || tok0 < 0) return -1;
+  const uint64_t gkey = ig_key(sp->seed, stream, chunk, IG_GATE);
+  const uint64_t bkey = ig_key(sp->seed, stream, chunk, IG_BETA);
+  const int64_t n = n_tok * (int64_t)H;
+  const uint64_t base = (uint64_t)tok0 * (uint64_t)H;
+  for (int64_t i = 0; i < n; ++i) {
+    if (g) g[i] = ig_gate_log_decay(gkey, base + (uint64_t)i, g_scale);
+    if (beta) beta[i] = ig_gate_beta(bkey, base + (uint64_t)i);
+  }
+  return 0;
+}
+
 struct IgDevArgs {
   uint64_t key[IG_MAX_STREAMS];
   uint64_t okey[IG_MAX_STREAMS];

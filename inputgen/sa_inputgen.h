@@ -19,6 +19,11 @@
  *                uniforms" approximation of N(0,1); support [-6, 6].
  *   IG_UNIFORM : U(-1,1) on the 2^23-point midpoint grid (2i+1)/2^23 - 1.
  *   IG_ZERO, IG_ONES : the constants 0 and 1 (degenerate test inputs).
+ * Gate inputs of the Gated DeltaNet block (one value per token and head):
+ *   IG_GATE    : log decay g = g_scale * (u - 1) / 2 in (-g_scale, 0);
+ *   IG_BETA    : write strength beta = (u + 1) / 2 in (0, 1);
+ *                u the IG_UNIFORM draw; exact in fp32 up to the product with
+ *                g_scale.
  * Optional row outliers (K only): a (token, head) row is selected with
  * probability `outlier_frac` by its own hash and multiplied by
  * `outlier_scale` in fp32 before the storage rounding.
@@ -40,7 +45,7 @@ extern "C" {
 #endif
 
 enum { IG_NORMAL = 0, IG_UNIFORM = 1, IG_ZERO = 2, IG_ONES = 3 };
-enum { IG_Q = 0, IG_K = 1, IG_V = 2, IG_OUTLIER = 3 };
+enum { IG_Q = 0, IG_K = 1, IG_V = 2, IG_OUTLIER = 3, IG_GATE = 4, IG_BETA = 5 };
 enum { IG_F32 = 0, IG_BF16 = 1 };
 
 typedef struct {
@@ -92,6 +97,15 @@ IG_FN float ig_uniform(uint64_t key, uint64_t idx) {
   uint64_t z = ig_draw(key, idx, 0);
   uint32_t i = (uint32_t)(z >> 41); /* 23 bits */
   return (float)(2u * i + 1u) * (1.0f / 8388608.0f) - 1.0f;
+}
+
+/* Gate values of element idx = tok*H + h of an IG_GATE / IG_BETA block. */
+IG_FN float ig_gate_log_decay(uint64_t key, uint64_t idx, float g_scale) {
+  return g_scale * ((ig_uniform(key, idx) - 1.0f) * 0.5f);
+}
+
+IG_FN float ig_gate_beta(uint64_t key, uint64_t idx) {
+  return (ig_uniform(key, idx) + 1.0f) * 0.5f;
 }
 
 /* Selection threshold for a row-outlier fraction: frac * 2^64, saturated. */

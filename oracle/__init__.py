@@ -67,6 +67,7 @@ def lib():
             "orc_attend_rows_uncommitted": ([C, S, S, i64, i64, i32, _D, _D, _D], i32),
             "orc_sink_pos": ([C, i64, i64], ctypes.c_double),
             "orc_sink_raw": ([C, S, i64, i64, i64, i32, _D], i32),
+            "orc_gdn_chunk": ([i32, i32, i64, ctypes.c_double, _D, _D, _D, _D, _D, _D, _D], i32),
             "orc_num_threads": ([], i32),
         }
         for name, (args, res) in sig.items():
@@ -243,6 +244,51 @@ def attend_rows_uncommitted(cfg: Cfg, spec_cache: Spec, spec_chunk: Spec, stream
 def bruteforce_rows(cfg: Cfg, spec: Spec, stream: int, c: int, toks, heads) -> np.ndarray:
     """Brute-force masked full-sequence attention rows (exact, absolute positions)."""
     return _rows(lib().orc_bruteforce_rows, cfg, spec, stream, c, toks, heads)
+
+
+def gdn_chunk(scale: float, state: np.ndarray, q, k, v, g, beta) -> np.ndarray:
+    """One call of the Gated DeltaNet recurrence (orc_gdn_chunk) over T tokens:
+    state [H, D, D] float64 (value dim, key dim) is updated in place; q, k, v
+    [T, H, D]; g (log decay) and beta [T, H]. Returns out [T, H, D] float64."""
+    assert state.dtype == np.float64 and state.flags["C_CONTIGUOUS"]
+    H, D, D2 = state.shape
+    assert D == D2
+    q, k, v = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+    g, beta = (np.ascontiguousarray(x, dtype=np.float64) for x in (g, beta))
+    T = q.shape[0]
+    assert q.shape == k.shape == v.shape == (T, H, D) and g.shape == beta.shape == (T, H)
+    out = np.empty((T, H, D), dtype=np.float64)
+    _check(lib().orc_gdn_chunk(H, D, T, scale, _ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                               _ptr(beta), _ptr(out)), "orc_gdn_chunk")
+    return out
+
+
+def gdn_inputs(w: Workload, stream: int, c: int, g_scale: float):
+    """Generated inputs of chunk c of a stream for the GDN block, as stored:
+    q, k, v [Lc, H, D] and g, beta [Lc, H], float64."""
+    from inputgen import fill_gates_host
+    cfg = cfg_for(w)
+    spec = spec_for(w)
+    q = input_block(cfg, spec, stream, c, 0)
+    k = input_block(cfg, spec, stream, c, 1)
+    v = input_block(cfg, spec, stream, c, 2)
+    g, beta = fill_gates_host(w, stream, c, g_scale)
+    return q, k, v, g.astype(np.float64), beta.astype(np.float64)
+
+
+def gdn_stream(w: Workload, stream: int, c: int, g_scale: float, scale: float, heads=None,
+               state: np.ndarray | None = None, c0: int = 0):
+    """Runs the GDN block over chunks c0..c of a stream from `state` (zero when
+    None) with the generated inputs; returns (out of chunk c [Lc, H', D],
+    state after chunk c [H', D, D]) for the heads `heads` (all when None)."""
+    hs = np.arange(w.H) if heads is None else np.asarray(heads)
+    if state is None:
+        state = np.zeros((len(hs), w.D, w.D), dtype=np.float64)
+    out = None
+    for ch in range(c0, c + 1):
+        q, k, v, g, beta = gdn_inputs(w, stream, ch, g_scale)
+        out = gdn_chunk(scale, state, q[:, hs], k[:, hs], v[:, hs], g[:, hs], beta[:, hs])
+    return out, state
 
 
 def num_threads() -> int:

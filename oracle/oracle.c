@@ -554,3 +554,71 @@ int32_t orc_bruteforce_rows(const orc_cfg* g, const ig_spec* sp, int64_t stream,
   free(Kr); free(Vr); free(Qr);
   return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Gated DeltaNet (GDN) block. SANA-Streaming, section "hybrid diffusion
+ * transformer": most blocks of that model use GDN linear attention, which
+ * folds the stream's history into a recurrent state of fixed size, updated
+ * as frames arrive; a GDN block keeps only its latest state between chunks.
+ * Section "system co-design": a fused kernel keeps that state on chip.
+ *
+ * The pages give neither the recurrence nor its gating or normalisation.
+ * Reading: the published gated delta rule (Yang, Kautz and Hatamizadeh,
+ * "Gated Delta Networks: Improving Mamba2 with Delta Rule", ICLR 2025) with
+ * its L2-normalised queries and keys, taken token by token in stream order
+ * (frame, row, column), per head:
+ *   k^ = k/|k|,  q^ = q/|q|                (a zero vector stays zero)
+ *   S  <- exp(g_t) S                        decay, g_t <= 0
+ *   S  <- S + beta_t (v_t - S k^_t) k^_t^T  delta-rule write
+ *   o_t = scale * S q^_t
+ * S has D rows (value dims) and D columns (key dims). Row i of S only ever
+ * meets v_t[i], so rows evolve independently.
+ * ------------------------------------------------------------------------- */
+static void l2_normalised(const double* x, int32_t D, double* out) {
+  double s = 0.0;
+  for (int32_t d = 0; d < D; ++d) s += x[d] * x[d];
+  const double inv = s > 0.0 ? 1.0 / sqrt(s) : 0.0;
+  for (int32_t d = 0; d < D; ++d) out[d] = x[d] * inv;
+}
+
+int32_t orc_gdn_chunk(int32_t H, int32_t D, int64_t T, double scale, double* state,
+                      const double* q, const double* k, const double* v, const double* g,
+                      const double* beta, double* out) {
+  if (H <= 0 || D <= 0 || T < 0 || !state) return -1;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !out)) return -1;
+  int32_t err = 0;
+#pragma omp parallel for schedule(dynamic)
+  for (int32_t h = 0; h < H; ++h) {
+    double* S = state + (size_t)h * D * D;
+    double* kh = (double*)malloc(sizeof(double) * (size_t)D * 2);
+    if (!kh) {
+#pragma omp atomic write
+      err = -1;
+      continue;
+    }
+    double* qh = kh + D;
+    for (int64_t t = 0; t < T; ++t) {
+      const size_t row = ((size_t)t * H + h) * D;
+      const size_t gi = (size_t)t * H + h;
+      l2_normalised(k + row, D, kh);
+      l2_normalised(q + row, D, qh);
+      const double alpha = exp(g[gi]);
+      for (size_t e = 0; e < (size_t)D * D; ++e) S[e] *= alpha;
+      for (int32_t i = 0; i < D; ++i) {
+        double* Si = S + (size_t)i * D;
+        double pred = 0.0;
+        for (int32_t j = 0; j < D; ++j) pred += Si[j] * kh[j];
+        const double u = beta[gi] * (v[row + i] - pred);
+        for (int32_t j = 0; j < D; ++j) Si[j] += u * kh[j];
+      }
+      for (int32_t i = 0; i < D; ++i) {
+        const double* Si = S + (size_t)i * D;
+        double o = 0.0;
+        for (int32_t j = 0; j < D; ++j) o += Si[j] * qh[j];
+        out[row + i] = scale * o;
+      }
+    }
+    free(kh);
+  }
+  return err;
+}

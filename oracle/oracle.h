@@ -93,6 +93,13 @@ int32_t orc_attend_rows_uncommitted(const orc_cfg* cfg, const ig_spec* sp_cache,
 int32_t orc_bruteforce_rows(const orc_cfg* cfg, const ig_spec* sp, int64_t stream,
                             int64_t c, int32_t n_rows, const int32_t* toks,
                             const int32_t* heads, double* out);
+/* Gated DeltaNet block, one call over T tokens of one stream, all heads (see
+ * oracle.c): state [H][D][D] (row i = value dim, column j = key dim) is read
+ * and updated in place; q, k, v, out [T][H][D]; g (log decay) and beta
+ * [T][H]. Returns 0, or -1 on a bad argument. */
+int32_t orc_gdn_chunk(int32_t H, int32_t D, int64_t T, double scale, double* state,
+                      const double* q, const double* k, const double* v, const double* g,
+                      const double* beta, double* out);
 int32_t orc_num_threads(void);
 
 #ifdef __cplusplus
