@@ -63,6 +63,10 @@ def parse():
     ap.add_argument("--eager", action="store_true", help="time eager launches, no CUDA graph")
     ap.add_argument("--chunks", type=int, default=0,
                     help="stream only this many chunks per stream (small profiling cases)")
+    ap.add_argument("--path", default="attention", choices=["attention", "gdn"],
+                    help="gdn: the Gated DeltaNet block (sa_gdn_chunk) on the same streams")
+    ap.add_argument("--gdn-g-scale", type=float, default=0.002,
+                    help="gdn: per-token log decay drawn in (-g_scale, 0)")
     return ap.parse_args()
 
 
@@ -202,6 +206,227 @@ def config_json(w, world):
                   " GB per step)"}
 
 
+# ------------------------------------------------------------------ GDN block
+GDN_METRIC = "GDN block: streamed chunks/s (gated delta rule state update + outputs)"
+FP32_LANES_PER_SM, SM_COUNT, SM_MAX_GHZ = 128, 148, 1.965
+
+
+def gdn_flops_per_token(D: int, ct: int = 64) -> float:
+    """Algorithmic FLOPs per token and head of the chunkwise gated delta rule
+    on sub-chunks of ct tokens: K S0^T, Q S0^T and the state update (2 D^2
+    each), the two lower-triangular Gram matrices and the two triangular
+    products with D columns (ct + 1) D each, and the triangular inverse
+    (ct^2 / 3). Counted once per head (the kernel's per-slice recomputation
+    is not algorithmic work)."""
+    return 6.0 * D * D + 4.0 * (ct + 1) * D + ct * ct / 3.0
+
+
+def gdn_oracle_sample(w, g_scale: float, n_tok: int = 256):
+    import numpy as np
+
+    import oracle as O
+    q, k, v, g, beta = O.gdn_inputs(w, 0, 0, g_scale)
+    st = np.zeros((w.H, w.D, w.D))
+    t0 = time.perf_counter()
+    O.gdn_chunk(1.0 / np.sqrt(w.D), st, q[:n_tok], k[:n_tok], v[:n_tok], g[:n_tok], beta[:n_tok])
+    dt = time.perf_counter() - t0
+    per_chunk = dt * w.Lc / n_tok
+    return {"value": 1.0 / per_chunk, "unit": "chunks/s", "cores": O.num_threads(),
+            "kind": "oracle",
+            "sample": f"{w.name}: the first {n_tok} of {w.Lc} tokens of one chunk, all {w.H} heads "
+                      f"(fp64 token-by-token recurrence, heads across threads), extrapolated "
+                      f"linearly to the chunk ({dt:.2f} s of CPU time)"}
+
+
+def gdn_config_json(w, world, g_scale):
+    return {"workload": w.name + "_gdn", "streams_per_gpu": w.B, "heads": w.H, "head_dim": w.D,
+            "tokens_per_chunk": w.Lc, "chunks_per_stream": w.n_chunks,
+            "g_scale": g_scale, "dtype_io": w.dtype, "state": "fp32 [B][H][D][D]",
+            "parallelism": f"independent streams per GPU x{world} (no collective)",
+            "l2": "inputs larger than L2 (every chunk of the step resident, "
+                  f"{3 * w.n_chunks * w.B * w.Lc * w.H * w.D * (2 if w.dtype == 'bf16' else 4) / 1e9:.1f}"
+                  " GB per step)"}
+
+
+def run_gdn(args, w, rank, world):
+    g_scale = args.gdn_g_scale
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per = []
+        for i in range(args.warmup + args.steps):
+            r = gdn_oracle_sample(w, g_scale, n_tok=64)
+            if i >= args.warmup:
+                per.append(1.0 / r["value"])
+        ms_step = 1000.0 * w.n_chunks * w.B * statistics.mean(per)
+        value = w.n_chunks * w.B / (ms_step / 1000.0)
+        print(json.dumps({
+            "metric": GDN_METRIC, "value": value, "unit": "chunks/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference", "config": gdn_config_json(w, world, g_scale),
+            "cpu_baseline": {"value": value, "unit": "chunks/s", "cores": r["cores"],
+                             "kind": "oracle", "sample": r["sample"]},
+            "e2e": {"value": value, "unit": "chunks/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import inputgen as IG
+    from rolling_kv_cache_sa_b200 import sa_gdn_chunk
+    from rolling_kv_cache_sa_b200.dist import aggregate_rate, max_over_ranks, rank_stream_ids
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    esz = 2 if w.dtype == "bf16" else 4
+    nC, B = w.n_chunks, w.B
+    shape = (nC, B, w.Lc, w.H, w.D)
+    q_all = torch.empty(shape, dtype=dt, device="cuda")
+    k_all, v_all, out_all = torch.empty_like(q_all), torch.empty_like(q_all), torch.empty_like(q_all)
+    g_all = torch.empty((nC, B, w.Lc, w.H), dtype=torch.float32, device="cuda")
+    b_all = torch.empty_like(g_all)
+    st = torch.cuda.current_stream().cuda_stream
+    sids = rank_stream_ids(rank, B)
+    for c in range(nC):
+        for t, buf in ((IG.Q, q_all), (IG.K, k_all), (IG.V, v_all)):
+            IG.fill_device(w, sids, [c] * B, t, buf[c].data_ptr(), st)
+        for bi, sid in enumerate(sids):
+            g, beta = IG.fill_gates_host(w, sid, c, g_scale)
+            g_all[c, bi].copy_(torch.from_numpy(g))
+            b_all[c, bi].copy_(torch.from_numpy(beta))
+    state = torch.zeros(B, w.H, w.D, w.D, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+
+    def run_step():
+        state.zero_()
+        for c in range(nC):
+            sa_gdn_chunk(state, q_all[c], k_all[c], v_all[c], g_all[c], b_all[c], out_all[c])
+
+    for _ in range(args.warmup):
+        run_step()
+    torch.cuda.synchronize()
+
+    def timed(fn, steps):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        e1.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), "cuda")
+
+    sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    # eager pass: CUDA events around every launch on the launch stream
+    eager_steps = max(1, min(args.steps, 10))
+    launch_ms = []
+    torch.cuda.synchronize()
+    for _ in range(eager_steps):
+        state.zero_()
+        evs = []
+        for c in range(nC):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sa_gdn_chunk(state, q_all[c], k_all[c], v_all[c], g_all[c], b_all[c], out_all[c])
+            e1.record()
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        launch_ms += [a.elapsed_time(b) for a, b in evs]
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap):
+        run_step()
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        graph.replay()
+    ms = timed(graph.replay, args.steps)
+    clocks = sampler.stop() if sampler else None
+    ms_step = ms / args.steps
+    chunks_per_step = nC * B
+    value = aggregate_rate(chunks_per_step * args.steps, world, ms)
+
+    flops_per_launch = gdn_flops_per_token(w.D) * w.Lc * w.H * B
+    avg_launch_s = statistics.mean(launch_ms) / 1000.0
+    achieved = flops_per_launch / avg_launch_s / 1e12
+    peak = FP32_LANES_PER_SM * SM_COUNT * 2 * SM_MAX_GHZ / 1e3
+    bytes_per_launch = B * (w.Lc * w.H * w.D * esz * 4 + w.Lc * w.H * 8 + 2 * w.H * w.D * w.D * 4)
+    hbm = peaks()[0]
+
+    # end to end through the public call: pinned host inputs copied in and
+    # outputs copied out every chunk, inside the timed region
+    qh = torch.empty(q_all.shape, dtype=dt, pin_memory=True)
+    kh, vh, oh = (torch.empty_like(qh, pin_memory=True) for _ in range(3))
+    gh = torch.empty(g_all.shape, dtype=torch.float32, pin_memory=True)
+    bh = torch.empty_like(gh, pin_memory=True)
+    qh.copy_(q_all), kh.copy_(k_all), vh.copy_(v_all), gh.copy_(g_all), bh.copy_(b_all)
+    dq, dk, dv, do = (torch.empty_like(q_all[0]) for _ in range(4))
+    dg, db = torch.empty_like(g_all[0]), torch.empty_like(b_all[0])
+
+    def run_step_host():
+        state.zero_()
+        for c in range(nC):
+            dq.copy_(qh[c], non_blocking=True)
+            dk.copy_(kh[c], non_blocking=True)
+            dv.copy_(vh[c], non_blocking=True)
+            dg.copy_(gh[c], non_blocking=True)
+            db.copy_(bh[c], non_blocking=True)
+            sa_gdn_chunk(state, dq, dk, dv, dg, db, do)
+            oh[c].copy_(do, non_blocking=True)
+
+    run_step_host()
+    e2e_steps = max(1, args.e2e_steps)
+    ems = timed(lambda: run_step_host(), e2e_steps)
+    e2e = {"value": aggregate_rate(chunks_per_step * e2e_steps, world, ems), "unit": "chunks/s",
+           "steps": e2e_steps,
+           "h2d_bytes_per_step": chunks_per_step * (3 * w.Lc * w.H * w.D * esz + 2 * w.Lc * w.H * 4),
+           "d2h_bytes_per_step": chunks_per_step * w.Lc * w.H * w.D * esz,
+           "api": "sa_gdn_chunk with every chunk's inputs copied from pinned host memory and its "
+                  "output copied back, in stream order, inside the timed region"}
+    cpu = gdn_oracle_sample(w, g_scale) if (rank == 0 and world == 1 and
+                                            not args.no_cpu_baseline) else None
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": GDN_METRIC, "value": value, "unit": "chunks/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded counter generator; Irwin-Hall N(0,1) q, k, v; uniform gates)",
+        "config": gdn_config_json(w, world, g_scale),
+        "ms_per_chunk": ms_step / chunks_per_step,
+        "launch_mode": "cuda graph of one step, replayed",
+        "roofline": {"bound": "alu", "kernel": f"gdn_chunk_kernel<{w.D}>",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak,
+                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP (FMA) x 1.965 GHz",
+                     "algorithmic_flops_per_launch": flops_per_launch,
+                     "hbm_bytes_per_launch": bytes_per_launch,
+                     "hbm_frac": bytes_per_launch / avg_launch_s / 1e9 / hbm,
+                     "duration": "mean of CUDA events around each launch on the launch stream, "
+                                 "eager pass", "traffic": None},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nC * args.steps, "clocks": clocks,
+        "launch_ms": {"mean": statistics.mean(launch_ms),
+                      "p50": float(np.percentile(launch_ms, 50)),
+                      "p99": float(np.percentile(launch_ms, 99))},
+    }), flush=True)
+
+
 # ------------------------------------------------------------------ GPU arm
 def main():
     args = parse()
@@ -219,6 +444,9 @@ def main():
     if args.cache:
         w = w.with_(cache=args.cache)
 
+    if args.path == "gdn":
+        run_gdn(args, w, rank, world)
+        return
     if args.impl == "reference":
         run_reference(args, w, rank, world)
         return

@@ -372,6 +372,49 @@ sa_status sa_sink_update(sa_cache* h, const void* k_new, const void* v_new, floa
 sa_status sa_wait_probe(uint64_t limit_ns, int64_t* waited_ns, sa_stream_t stream);
 
 /* Thread-local text of the last error; never NULL. */
+/*
+ * Gated DeltaNet (GDN) block: the linear-attention half of a hybrid streaming
+ * transformer (SANA-Streaming, sections "hybrid diffusion transformer" and
+ * "system co-design": most blocks keep a fixed-size recurrent state per head,
+ * updated as frames arrive, and cache only that state between chunks; a fused
+ * kernel keeps the state on chip). The pages give no recurrence; this call
+ * runs the published gated delta rule (Yang, Kautz and Hatamizadeh, "Gated
+ * Delta Networks", ICLR 2025) with L2-normalised q and k, token by token in
+ * the order given, per stream b and head h:
+ *     S <- exp(g_t) S (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = scale S q_t
+ * (k_t, q_t divided by their norms; a zero vector stays zero). S is D x D:
+ * row i = value dim, column j = key dim.
+ */
+typedef struct {
+  int32_t batch;     /* B streams, 1..SA_MAX_STREAMS */
+  int32_t heads;     /* H, 1..65535 */
+  int32_t head_dim;  /* D: 64 or 128 (query, key and value dims) */
+  int32_t dtype;     /* SA_F32 or SA_BF16: element type of q, k, v and out */
+  int64_t tokens;    /* T tokens of every active stream in this call, >= 0 */
+  float scale;       /* output scale, >= 0; 0 means 1/sqrt(D) */
+  int32_t pad_;
+} sa_gdn_config;
+
+/*
+ * Advances the state of every active stream over its next T tokens and
+ * writes their outputs. Device pointers, all owned by the caller:
+ *   state  [B][H][D][D] fp32, 16-byte aligned, read and written in place (the
+ *          block's whole memory between calls; zero it to start a stream);
+ *   q, k, v, out [B][T][H][D] in cfg->dtype (out may not alias the inputs);
+ *   g      [B][T][H] fp32, log decay of each token (<= 0; exp(g) multiplies S);
+ *   beta   [B][T][H] fp32, write strength of each token (in [0, 1] for a
+ *          contracting update; other values are computed as given).
+ * active: host array of B flags, NULL = all; an inactive stream's state and
+ * out rows are untouched. Arithmetic is fp32 with fp32 state; outputs are
+ * rounded once to cfg->dtype. Asynchronous on `stream`, graph-capturable.
+ * Errors: SA_ERR_INVALID_ARG (cfg, a NULL pointer with tokens > 0, alignment),
+ * SA_ERR_UNSUPPORTED (no compute capability 10.x device, or a size that does
+ * not fit), SA_ERR_CUDA (the launch failed).
+ */
+sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, const void* k,
+                       const void* v, const float* g, const float* beta, void* out,
+                       const uint8_t* active, sa_stream_t stream);
+
 const char* sa_last_error_string(void);
 
 int32_t sa_abi_version(void);

@@ -24,6 +24,7 @@ EXPORTED = (
     "sa_profile_launches", "sa_wait_probe", "sa_attend", "sa_cache_set_sink_mode",
     "sa_sink_update", "sa_append_attend_host_async", "sa_host_wait", "sa_cache_set_fp8_scales",
     "sa_cache_export_size", "sa_cache_export", "sa_cache_import", "sa_cache_get_fp8_scales",
+    "sa_gdn_chunk",
 )
 
 
@@ -35,6 +36,14 @@ class sa_config(ctypes.Structure):
         ("window_frames", ctypes.c_int32), ("rope_dims", ctypes.c_int32 * 3),
         ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float),
         ("dtype", ctypes.c_int32),
+    ]
+
+
+class sa_gdn_config(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("tokens", ctypes.c_int64), ("scale", ctypes.c_float),
+        ("pad_", ctypes.c_int32),
     ]
 
 
@@ -95,6 +104,7 @@ def lib() -> ctypes.CDLL:
         "sa_wait_probe": [ctypes.c_uint64, P(i64), vp],
         "sa_append_attend_noalloc": [P(sa_config), vp, vp, vp, P(i64), P(i64), vp, vp, vp, vp,
                                      vp, vp],
+        "sa_gdn_chunk": [P(sa_gdn_config), vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "sa_profile_end": [vp, P(ctypes.c_double), P(i32), P(ctypes.c_double), P(i32),
                            P(ctypes.c_double), P(i32)],
     }

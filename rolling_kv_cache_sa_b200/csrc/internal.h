@@ -96,6 +96,26 @@ struct AttnParams {
 // zero again.
 size_t attend_partials_bytes(int D, int num_sms, int64_t max_units);
 
+// Gated DeltaNet block (gdn.cu): T tokens of each listed stream; q, k, v, out
+// [B][T][H][D], g and beta [B][T][H], state [B][H][D][D] fp32 in place.
+struct GdnParams {
+  float* state;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  void* out;
+  int64_t T;
+  int32_t H;
+  float scale;
+  int32_t n_streams;
+  int32_t pad_;
+  int32_t stream_of[SA_MAX_STREAMS];
+};
+size_t gdn_smem_bytes(int D);
+cudaError_t launch_gdn(const GdnParams& p, int D, int dtype, cudaStream_t st);
+
 cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStream_t st);
 // Bounded-wait check (wait_probe.cu); synchronises `st` and returns the
 // device status word and the two warps' waiting times.

@@ -320,6 +320,66 @@ sa_status sa_wait_probe(uint64_t limit_ns, int64_t* waited_ns, sa_stream_t strea
   return SA_OK;
 }
 
+sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, const void* k,
+                       const void* v, const float* g, const float* beta, void* out,
+                       const uint8_t* active, sa_stream_t stream) {
+  if (!cfg) return fail(SA_ERR_INVALID_ARG, "config is NULL");
+  if (cfg->batch < 1 || cfg->batch > SA_MAX_STREAMS)
+    return fail(SA_ERR_INVALID_ARG, "batch must be in [1, %d], got %d", SA_MAX_STREAMS, cfg->batch);
+  if (cfg->heads < 1 || cfg->heads > 65535)
+    return fail(SA_ERR_INVALID_ARG, "heads must be in [1, 65535], got %d", cfg->heads);
+  if (cfg->head_dim != 64 && cfg->head_dim != 128)
+    return fail(SA_ERR_INVALID_ARG, "head_dim must be 64 or 128, got %d", cfg->head_dim);
+  if (cfg->dtype != SA_F32 && cfg->dtype != SA_BF16)
+    return fail(SA_ERR_INVALID_ARG, "dtype must be SA_F32 or SA_BF16");
+  if (cfg->tokens < 0) return fail(SA_ERR_INVALID_ARG, "tokens must be >= 0");
+  if (!(cfg->scale >= 0.f) || !std::isfinite(cfg->scale))
+    return fail(SA_ERR_INVALID_ARG, "scale must be finite and >= 0 (0 = 1/sqrt(D))");
+  const size_t esz = cfg->dtype == SA_F32 ? 4 : 2;
+  if ((double)cfg->batch * (double)cfg->tokens * cfg->heads * cfg->head_dim * esz > 9.0e18)
+    return fail(SA_ERR_UNSUPPORTED, "batch*tokens*heads*head_dim too large");
+  if (!state) return fail(SA_ERR_INVALID_ARG, "state is NULL");
+  if (reinterpret_cast<uintptr_t>(state) % 16)
+    return fail(SA_ERR_INVALID_ARG, "state must be 16-byte aligned");
+  if (cfg->tokens > 0) {
+    if (!q || !k || !v || !g || !beta || !out)
+      return fail(SA_ERR_INVALID_ARG, "q, k, v, g, beta and out must be non-NULL");
+    const uintptr_t ptrs[4] = {(uintptr_t)q, (uintptr_t)k, (uintptr_t)v, (uintptr_t)out};
+    for (uintptr_t a : ptrs)
+      if (a % esz) return fail(SA_ERR_INVALID_ARG, "q, k, v and out must be aligned to their element");
+    if ((uintptr_t)g % 4 || (uintptr_t)beta % 4)
+      return fail(SA_ERR_INVALID_ARG, "g and beta must be 4-byte aligned");
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SA_ERR_UNSUPPORTED, "no CUDA device: %s", cudaGetErrorString(e));
+  int major = 0;
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (major != 10)
+    return fail(SA_ERR_UNSUPPORTED, "device %d is sm_%d; this library runs on sm_100a (B200)", dev,
+                major * 10);
+  sa::GdnParams p;
+  memset(&p, 0, sizeof(p));
+  for (int b = 0; b < cfg->batch; ++b)
+    if (!active || active[b]) p.stream_of[p.n_streams++] = b;
+  if (p.n_streams == 0 || cfg->tokens == 0) return SA_OK;
+  p.state = state;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.g = g;
+  p.beta = beta;
+  p.out = out;
+  p.T = cfg->tokens;
+  p.H = cfg->heads;
+  p.scale = cfg->scale > 0.f ? cfg->scale : (float)(1.0 / sqrt((double)cfg->head_dim));
+  NvtxRange nv("sa_gdn_chunk");
+  e = sa::launch_gdn(p, cfg->head_dim, cfg->dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gdn launch");
+  return SA_OK;
+}
+
 const char* sa_last_error_string(void) { return g_last_error.c_str(); }
 
 sa_status sa_plan_chunk(const sa_config* cfg, int64_t frames_written, int64_t pos_base,

@@ -119,3 +119,52 @@ def test_planner_matches_oracle(C, Sn, W):
         sf = O.slot_frames(ocfg, c)
         occupied = [s for s, f in enumerate(sf) if f >= 0]
         assert occupied == list(range(pl.n_keys // w.F))
+
+
+def _gdn_cfg(**kw):
+    c = _lib.sa_gdn_config()
+    c.batch, c.heads, c.head_dim, c.dtype, c.tokens, c.scale = 2, 3, 128, _lib.SA_BF16, 64, 0.0
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("field,value", [("batch", 0), ("batch", 65), ("heads", 0),
+                                         ("head_dim", 96), ("dtype", 2), ("tokens", -1),
+                                         ("scale", -1.0), ("scale", float("inf"))])
+def test_gdn_chunk_validates_config(field, value):
+    """Argument checks run before any device call (no GPU needed)."""
+    c = _gdn_cfg(**{field: value})
+    buf = ctypes.create_string_buffer(1 << 12)
+    p = ctypes.cast(ctypes.addressof(buf) + (16 - ctypes.addressof(buf) % 16) % 16, ctypes.c_void_p)
+    st = _lib.lib().sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, None, None)
+    assert st == _lib.SA_ERR_INVALID_ARG
+    assert _lib.lib().sa_last_error_string()
+
+
+def test_gdn_chunk_validates_pointers():
+    L = _lib.lib()
+    c = _gdn_cfg()
+    assert L.sa_gdn_chunk(None, None, None, None, None, None, None, None, None, None) == \
+        _lib.SA_ERR_INVALID_ARG
+    buf = ctypes.create_string_buffer(1 << 12)
+    base = ctypes.addressof(buf) + (16 - ctypes.addressof(buf) % 16) % 16
+    p = ctypes.c_void_p(base)
+    assert L.sa_gdn_chunk(ctypes.byref(c), None, p, p, p, p, p, p, None, None) == \
+        _lib.SA_ERR_INVALID_ARG                      # state NULL
+    assert L.sa_gdn_chunk(ctypes.byref(c), ctypes.c_void_p(base + 4), p, p, p, p, p, p, None,
+                          None) == _lib.SA_ERR_INVALID_ARG   # state not 16-byte aligned
+    assert L.sa_gdn_chunk(ctypes.byref(c), p, p, None, p, p, p, p, None, None) == \
+        _lib.SA_ERR_INVALID_ARG                      # k NULL with tokens > 0
+    assert L.sa_gdn_chunk(ctypes.byref(c), p, ctypes.c_void_p(base + 1), p, p, p, p, p, None,
+                          None) == _lib.SA_ERR_INVALID_ARG   # q misaligned for bf16
+    assert b"aligned" in L.sa_last_error_string()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device refusal")
+def test_gdn_chunk_without_device_is_refused():
+    buf = ctypes.create_string_buffer(1 << 12)
+    p = ctypes.c_void_p(ctypes.addressof(buf) + (16 - ctypes.addressof(buf) % 16) % 16)
+    c = _gdn_cfg()
+    assert _lib.lib().sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, None, None) == \
+        _lib.SA_ERR_UNSUPPORTED
