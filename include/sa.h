@@ -400,7 +400,8 @@ typedef struct {
  * writes their outputs. Device pointers, all owned by the caller:
  *   state  [B][H][D][D] fp32, 16-byte aligned, read and written in place (the
  *          block's whole memory between calls; zero it to start a stream);
- *   q, k, v, out [B][T][H][D] in cfg->dtype (out may not alias the inputs);
+ *   q, k, v, out [B][T][H][D] in cfg->dtype (out may not alias the inputs;
+ *          q, k and v 16-byte aligned, out aligned to its element);
  *   g      [B][T][H] fp32, log decay of each token (<= 0; exp(g) multiplies S);
  *   beta   [B][T][H] fp32, write strength of each token (in [0, 1] for a
  *          contracting update; other values are computed as given).

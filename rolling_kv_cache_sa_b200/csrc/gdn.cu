@@ -49,7 +49,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Shared-memory layout in floats. Rows of K^, Q^ and S have pitch D + 4: a
 // multiple of 4 (16-byte aligned rows) whose 16-byte groups step by an odd
 // count, so float4 reads of consecutive rows fall in different bank groups.
-template <int D>
+// The staging area receives the next sub-chunk's raw q, k rows and value
+// slice (input element type) by cp.async while the current one is computed.
+template <int D, typename T>
 struct GdnSmem {
   static constexpr int KP = D + 4;
   static constexpr int kh = 0;                    // [64][KP] normalised keys
@@ -64,8 +66,10 @@ struct GdnSmem {
   static constexpr int gs = uv + kCt * kVp;       // [64] in-warp prefix sums of g log2(e)
   static constexpr int bs = gs + kCt;             // [64] beta
   static constexpr int ws = bs + kCt;             // [64] e^(G_last - G_t)
-  static constexpr int total = ws + kCt;
-  static constexpr size_t bytes = (size_t)total * sizeof(float);
+  static constexpr int stage = (ws + kCt + 3) / 4 * 4;   // raw staging (bytes from here)
+  static constexpr int kStageK = kCt * D * (int)sizeof(T);        // bytes of 64 raw rows
+  static constexpr int kStageV = kCt * kDvs * (int)sizeof(T);     // bytes of 64 value slices
+  static constexpr size_t bytes = (size_t)stage * sizeof(float) + 2 * kStageK + kStageV;
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -84,10 +88,32 @@ __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
   return fmaf(a.w, b.w, acc);
 }
 
-__device__ __forceinline__ float ld_in(const float* p, size_t i) { return __ldg(p + i); }
-__device__ __forceinline__ float ld_in(const __nv_bfloat16* p, size_t i) {
-  return __bfloat162float(p[i]);
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// Four consecutive input elements (16 bytes of fp32 or 8 of bf16) as floats.
+__device__ __forceinline__ float4 ld_raw4(const float* p) { return ld4(p); }
+__device__ __forceinline__ float4 ld_raw4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+}
+// Two consecutive input elements as floats.
+__device__ __forceinline__ float2 ld_raw2(const float* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+__device__ __forceinline__ float2 ld_raw2(const __nv_bfloat16* p) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ void st_out(float* p, size_t i, float x) { p[i] = x; }
 __device__ __forceinline__ void st_out(__nv_bfloat16* p, size_t i, float x) {
   p[i] = __float2bfloat16_rn(x);
@@ -95,10 +121,11 @@ __device__ __forceinline__ void st_out(__nv_bfloat16* p, size_t i, float x) {
 
 template <int D, typename T>
 __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_constant__ GdnParams p) {
-  using L = GdnSmem<D>;
+  using L = GdnSmem<D, T>;
   constexpr int KP = L::KP;
-  constexpr int NE = D / 32;   // elements of a row per lane
-  constexpr int NJ = D / 32;   // float4 groups of state per thread
+  constexpr int NJ = D / 32;                         // float4 groups of state per thread
+  constexpr int kRow16 = D * (int)sizeof(T) / 16;    // 16-byte pieces of a raw row
+  constexpr int kV16 = kDvs * (int)sizeof(T) / 16;   // 16-byte pieces of a value slice
   extern __shared__ __align__(16) float sm[];
   float* Kh = sm + L::kh;
   float* Qh = sm + L::qh;
@@ -112,6 +139,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
   float* Gs = sm + L::gs;
   float* Bs = sm + L::bs;
   float* Ws = sm + L::ws;
+  unsigned char* stg = reinterpret_cast<unsigned char*>(sm + L::stage);
+  T* Kraw = reinterpret_cast<T*>(stg);                       // [64][D]
+  T* Qraw = reinterpret_cast<T*>(stg + L::kStageK);          // [64][D]
+  T* Vraw = reinterpret_cast<T*>(stg + 2 * L::kStageK);      // [64][32]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int slice = blockIdx.x, h = blockIdx.y, b = p.stream_of[blockIdx.z];
@@ -127,6 +158,37 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
   const int vcol = slice * kDvs;
   float* Sg = p.state + (((size_t)b * H + h) * D + vcol) * D;
 
+  // Issues the copies of sub-chunk [t0, t0 + 64) into the staging area (rows
+  // past the end are not copied; the consumer treats them as zero) and
+  // returns the gates of token t0 + tid for threads tid < 64.
+  auto prefetch = [&](int64_t t0, float& gl, float& bl) {
+    const int n = (int)(Tn - t0 < kCt ? Tn - t0 : kCt);
+    for (int c = tid; c < kCt * kRow16; c += kGdnThreads) {
+      const int r = c / kRow16, piece = c % kRow16;
+      if (r < n) {
+        const size_t off = bh0 + (size_t)(t0 + r) * tok_stride;
+        cp_async16(reinterpret_cast<unsigned char*>(Kraw + r * D) + piece * 16,
+                   reinterpret_cast<const unsigned char*>(k + off) + piece * 16);
+        cp_async16(reinterpret_cast<unsigned char*>(Qraw + r * D) + piece * 16,
+                   reinterpret_cast<const unsigned char*>(q + off) + piece * 16);
+      }
+    }
+    for (int c = tid; c < kCt * kV16; c += kGdnThreads) {
+      const int r = c / kV16, piece = c % kV16;
+      if (r < n) {
+        const size_t off = bh0 + (size_t)(t0 + r) * tok_stride + vcol;
+        cp_async16(reinterpret_cast<unsigned char*>(Vraw + r * kDvs) + piece * 16,
+                   reinterpret_cast<const unsigned char*>(v + off) + piece * 16);
+      }
+    }
+    cp_async_commit();
+    if (tid < kCt) {
+      const bool ok = tid < n;
+      gl = ok ? p.g[g0 + (size_t)(t0 + tid) * H] : 0.f;
+      bl = ok ? p.beta[g0 + (size_t)(t0 + tid) * H] : 0.f;
+    }
+  };
+
   // Cumulative log2 decay through token t of the sub-chunk (warp 1's prefix
   // sums lack warp 0's total, added here).
   auto gcum = [&](int t) -> float { return Gs[t] + (t >= 32 ? Gs[31] : 0.f); };
@@ -140,40 +202,20 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
     sreg[m] = *reinterpret_cast<const float4*>(Sg + (size_t)uc * D + uj + 32 * m);
     st4(St + uc * KP + uj + 32 * m, sreg[m]);
   }
+  // Tokens and state rows of the products with D columns (right-hand side,
+  // U, outputs): tokens tw + 16a (a < 4), rows cw + 16bb (bb < 2).
+  const int tw = warp * 2 + (lane >> 4);
+  const int cw = lane & 15;
+
+  float gnext = 0.f, bnext = 0.f;
+  prefetch(0, gnext, bnext);
 
   for (int64_t t0 = 0; t0 < Tn; t0 += kCt) {
     const int n = (int)(Tn - t0 < kCt ? Tn - t0 : kCt);
-
-    // ---- normalised key and query rows, the value slice, the gates
-    for (int r = warp; r < kCt; r += 8) {
-      float kx[NE], qx[NE];
-      float sk = 0.f, sq = 0.f;
-      const size_t off = bh0 + (size_t)(t0 + r) * tok_stride;
-#pragma unroll
-      for (int e = 0; e < NE; ++e) {
-        kx[e] = r < n ? ld_in(k, off + lane + 32 * e) : 0.f;
-        qx[e] = r < n ? ld_in(q, off + lane + 32 * e) : 0.f;
-        sk = fmaf(kx[e], kx[e], sk);
-        sq = fmaf(qx[e], qx[e], sq);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        sk += __shfl_xor_sync(0xffffffffu, sk, o);
-        sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      }
-      const float ik = sk > 0.f ? rsqrtf(sk) : 0.f;
-      const float iq = sq > 0.f ? rsqrtf(sq) : 0.f;
-#pragma unroll
-      for (int e = 0; e < NE; ++e) {
-        Kh[r * KP + lane + 32 * e] = kx[e] * ik;
-        Qh[r * KP + lane + 32 * e] = qx[e] * iq;
-      }
-      Rv[r * kVp + lane] = r < n ? ld_in(v, off + vcol + lane) : 0.f;
-    }
-    if (tid < kCt) {   // warps 0 and 1
-      const bool ok = tid < n;
-      float gl = ok ? p.g[g0 + (size_t)(t0 + tid) * H] * kLog2e : 0.f;
-      Bs[tid] = ok ? p.beta[g0 + (size_t)(t0 + tid) * H] : 0.f;
+    cp_async_wait_all();
+    if (tid < kCt) {   // warps 0 and 1: gates of this sub-chunk, prefix sums
+      float gl = gnext * kLog2e;
+      Bs[tid] = bnext;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, gl, o);
@@ -182,6 +224,43 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
       Gs[tid] = gl;
     }
     __syncthreads();
+
+    // ---- normalised key and query rows, the value slice (rows past n are 0)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = warp + 8 * i;
+      float4 kx = make_float4(0.f, 0.f, 0.f, 0.f), qx = kx;
+      if (r < n) {
+        if constexpr (D == 128) {
+          kx = ld_raw4(Kraw + r * D + 4 * lane);
+          qx = ld_raw4(Qraw + r * D + 4 * lane);
+        } else {
+          const float2 k2 = ld_raw2(Kraw + r * D + 2 * lane);
+          const float2 q2 = ld_raw2(Qraw + r * D + 2 * lane);
+          kx = make_float4(k2.x, k2.y, 0.f, 0.f);
+          qx = make_float4(q2.x, q2.y, 0.f, 0.f);
+        }
+      }
+      float sk = dot4(kx, kx, 0.f), sq = dot4(qx, qx, 0.f);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      }
+      const float ik = sk > 0.f ? rsqrtf(sk) : 0.f;
+      const float iq = sq > 0.f ? rsqrtf(sq) : 0.f;
+      if constexpr (D == 128) {
+        st4(Kh + r * KP + 4 * lane, make_float4(kx.x * ik, kx.y * ik, kx.z * ik, kx.w * ik));
+        st4(Qh + r * KP + 4 * lane, make_float4(qx.x * iq, qx.y * iq, qx.z * iq, qx.w * iq));
+      } else {
+        *reinterpret_cast<float2*>(Kh + r * KP + 2 * lane) = make_float2(kx.x * ik, kx.y * ik);
+        *reinterpret_cast<float2*>(Qh + r * KP + 2 * lane) = make_float2(qx.x * iq, qx.y * iq);
+      }
+      Rv[r * kVp + lane] = r < n ? to_f(Vraw[r * kDvs + lane]) : 0.f;
+    }
+    __syncthreads();
+    // the staging area is free again: fetch the next sub-chunk behind this one
+    if (t0 + kCt < Tn) prefetch(t0 + kCt, gnext, bnext);
 
     // ---- Gram matrices on the lower triangle -> L and P. Thread (ty, tx)
     // takes rows ty + 16a and columns tx + 16b, b <= a (the pairs a < b lie
@@ -228,31 +307,38 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
           Pm[t * kLp + s] = pv;
         }
     }
-    // ---- K^ S0^T and Q^ S0^T for this CTA's rows: thread (warp, lane) takes
-    // tokens warp + 8a and state row lane. The right-hand side
+    // ---- K^ S0^T and Q^ S0^T for this CTA's rows. The right-hand side
     // beta_t (v_t - e^(G_t) (S0 k_t)) replaces v in Rv; the inter-chunk part of
-    // the output stays in registers.
-    float oin[8];
+    // the output, scale e^(G_t) (S0 q_t), stays in registers.
+    float oin[4][2];
     {
-      float aks[8], aqs[8];
+      float aks[4][2], aqs[4][2];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) aks[a] = aqs[a] = 0.f;
-      const float* srow = St + lane * KP;
+      for (int a = 0; a < 4; ++a) aks[a][0] = aks[a][1] = aqs[a][0] = aqs[a][1] = 0.f;
 #pragma unroll 2
       for (int d = 0; d < D; d += 4) {
-        const float4 s4 = ld4(srow + d);
+        const float4 s0 = ld4(St + cw * KP + d);
+        const float4 s1 = ld4(St + (cw + 16) * KP + d);
 #pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          aks[a] = dot4(ld4(Kh + (warp + 8 * a) * KP + d), s4, aks[a]);
-          aqs[a] = dot4(ld4(Qh + (warp + 8 * a) * KP + d), s4, aqs[a]);
+        for (int a = 0; a < 4; ++a) {
+          const float4 k4 = ld4(Kh + (tw + 16 * a) * KP + d);
+          const float4 q4 = ld4(Qh + (tw + 16 * a) * KP + d);
+          aks[a][0] = dot4(k4, s0, aks[a][0]);
+          aks[a][1] = dot4(k4, s1, aks[a][1]);
+          aqs[a][0] = dot4(q4, s0, aqs[a][0]);
+          aqs[a][1] = dot4(q4, s1, aqs[a][1]);
         }
       }
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const int t = warp + 8 * a;
+      for (int a = 0; a < 4; ++a) {
+        const int t = tw + 16 * a;
         const float gam = ex2f(gcum(t));
-        Rv[t * kVp + lane] = Bs[t] * (Rv[t * kVp + lane] - gam * aks[a]);
-        oin[a] = p.scale * gam * aqs[a];
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int c = cw + 16 * bb;
+          Rv[t * kVp + c] = Bs[t] * (Rv[t * kVp + c] - gam * aks[a][bb]);
+          oin[a][bb] = p.scale * gam * aqs[a][bb];
+        }
       }
     }
     __syncthreads();
@@ -266,7 +352,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
       for (int t = 0; t < 16; ++t) {
         float acc = 0.f;
 #pragma unroll
-        for (int s = 0; s < t; ++s) acc = fmaf(Lm[(r0 + t) * kLp + r0 + s], x[s], acc);
+        for (int s2 = 0; s2 < t; ++s2) acc = fmaf(Lm[(r0 + t) * kLp + r0 + s2], x[s2], acc);
         x[t] = t < j ? 0.f : (t == j ? 1.f : -acc);
       }
 #pragma unroll
@@ -279,76 +365,109 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
 
     // ---- merge to 32 x 32 blocks (rows r0+16.., columns r0.., r0 = 0, 32):
     // X = L21 T11, then T21 = -T22 X
-    for (int e = tid; e < 512; e += kGdnThreads) {
+#pragma unroll
+    for (int e0 = 0; e0 < 512; e0 += kGdnThreads) {
+      const int e = e0 + tid;
       const int pp = e >> 8, i = (e >> 4) & 15, j = e & 15, r0 = pp * 32;
       float acc = 0.f;
-      for (int s = j; s < 16; ++s)
-        acc = fmaf(Lm[(r0 + 16 + i) * kLp + r0 + s], Tm[(r0 + s) * kLp + r0 + j], acc);
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2)
+        if (s2 >= j)
+          acc = fmaf(Lm[(r0 + 16 + i) * kLp + r0 + s2], Tm[(r0 + s2) * kLp + r0 + j], acc);
       Xm[pp * 272 + i * 17 + j] = acc;
     }
     __syncthreads();
-    for (int e = tid; e < 512; e += kGdnThreads) {
+#pragma unroll
+    for (int e0 = 0; e0 < 512; e0 += kGdnThreads) {
+      const int e = e0 + tid;
       const int pp = e >> 8, i = (e >> 4) & 15, j = e & 15, r0 = pp * 32;
       float acc = 0.f;
-      for (int s = 0; s <= i; ++s)
-        acc = fmaf(Tm[(r0 + 16 + i) * kLp + r0 + 16 + s], Xm[pp * 272 + s * 17 + j], acc);
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2)
+        if (s2 <= i)
+          acc = fmaf(Tm[(r0 + 16 + i) * kLp + r0 + 16 + s2], Xm[pp * 272 + s2 * 17 + j], acc);
       Tm[(r0 + 16 + i) * kLp + r0 + j] = -acc;
     }
     __syncthreads();
     // ---- merge to the full 64 x 64 inverse (rows 32.., columns 0..31)
-    for (int e = tid; e < 1024; e += kGdnThreads) {
+#pragma unroll
+    for (int e0 = 0; e0 < 1024; e0 += kGdnThreads) {
+      const int e = e0 + tid;
       const int i = e >> 5, j = e & 31;
       float acc = 0.f;
-      for (int s = j; s < 32; ++s) acc = fmaf(Lm[(32 + i) * kLp + s], Tm[s * kLp + j], acc);
+#pragma unroll
+      for (int s2 = 0; s2 < 32; ++s2)
+        if (s2 >= j) acc = fmaf(Lm[(32 + i) * kLp + s2], Tm[s2 * kLp + j], acc);
       Xm[i * 33 + j] = acc;
     }
     __syncthreads();
-    for (int e = tid; e < 1024; e += kGdnThreads) {
+#pragma unroll
+    for (int e0 = 0; e0 < 1024; e0 += kGdnThreads) {
+      const int e = e0 + tid;
       const int i = e >> 5, j = e & 31;
       float acc = 0.f;
-      for (int s = 0; s <= i; ++s) acc = fmaf(Tm[(32 + i) * kLp + 32 + s], Xm[s * 33 + j], acc);
+#pragma unroll
+      for (int s2 = 0; s2 < 32; ++s2)
+        if (s2 <= i) acc = fmaf(Tm[(32 + i) * kLp + 32 + s2], Xm[s2 * 33 + j], acc);
       Tm[(32 + i) * kLp + j] = -acc;
     }
     __syncthreads();
 
-    // ---- corrected values U = (I + L)^-1 RHS (tokens warp + 8a, row lane)
+    // ---- corrected values U = (I + L)^-1 RHS. Rows of RHS past n are zero,
+    // so the sums run over all 64 tokens.
     {
-      float acc[8];
+      float acc[4][2];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) acc[a] = 0.f;
-      for (int s = 0; s < n; ++s) {
-        const float r = Rv[s * kVp + lane];
+      for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0.f;
+#pragma unroll 8
+      for (int s2 = 0; s2 < kCt; ++s2) {
+        const float r0 = Rv[s2 * kVp + cw];
+        const float r1 = Rv[s2 * kVp + cw + 16];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const int t = warp + 8 * a;
-          if (s <= t) acc[a] = fmaf(Tm[t * kLp + s], r, acc[a]);
+        for (int a = 0; a < 4; ++a) {
+          const int t = tw + 16 * a;
+          const float tv = s2 <= t ? Tm[t * kLp + s2] : 0.f;
+          acc[a][0] = fmaf(tv, r0, acc[a][0]);
+          acc[a][1] = fmaf(tv, r1, acc[a][1]);
         }
       }
 #pragma unroll
-      for (int a = 0; a < 8; ++a) Uv[(warp + 8 * a) * kVp + lane] = acc[a];
+      for (int a = 0; a < 4; ++a) {
+        Uv[(tw + 16 * a) * kVp + cw] = acc[a][0];
+        Uv[(tw + 16 * a) * kVp + cw + 16] = acc[a][1];
+      }
     }
     __syncthreads();
 
     // ---- outputs: inter-chunk part + intra-chunk part P U
     {
-      float acc[8];
+      float acc[4][2];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) acc[a] = oin[a];
-      for (int s = 0; s < n; ++s) {
-        const float u = Uv[s * kVp + lane];
+      for (int a = 0; a < 4; ++a) acc[a][0] = oin[a][0], acc[a][1] = oin[a][1];
+#pragma unroll 8
+      for (int s2 = 0; s2 < kCt; ++s2) {
+        const float u0 = Uv[s2 * kVp + cw];
+        const float u1 = Uv[s2 * kVp + cw + 16];
 #pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const int t = warp + 8 * a;
-          if (s <= t) acc[a] = fmaf(Pm[t * kLp + s], u, acc[a]);
+        for (int a = 0; a < 4; ++a) {
+          const int t = tw + 16 * a;
+          const float pv = s2 <= t ? Pm[t * kLp + s2] : 0.f;
+          acc[a][0] = fmaf(pv, u0, acc[a][0]);
+          acc[a][1] = fmaf(pv, u1, acc[a][1]);
         }
       }
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        const int t = warp + 8 * a;
-        if (t < n) st_out(out, bh0 + (size_t)(t0 + t) * tok_stride + vcol + lane, acc[a]);
+      for (int a = 0; a < 4; ++a) {
+        const int t = tw + 16 * a;
+        if (t < n) {
+          const size_t o = bh0 + (size_t)(t0 + t) * tok_stride + vcol + cw;
+          st_out(out, o, acc[a][0]);
+          st_out(out, o + 16, acc[a][1]);
+        }
       }
     }
     // ---- state: S = e^(G_last) S0 + sum_t e^(G_last - G_t) u_t k_t^T
+    // (u and k are zero past n)
     {
       const float dec = ex2f(gcum(kCt - 1));
 #pragma unroll
@@ -358,7 +477,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
         sreg[m].z *= dec;
         sreg[m].w *= dec;
       }
-      for (int t = 0; t < n; ++t) {
+#pragma unroll 8
+      for (int t = 0; t < kCt; ++t) {
         const float uw = Uv[t * kVp + uc] * Ws[t];
 #pragma unroll
         for (int m = 0; m < NJ; ++m) {
@@ -381,7 +501,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
 
 template <int D, typename T>
 cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
-  constexpr size_t smem = GdnSmem<D>::bytes;
+  constexpr size_t smem = GdnSmem<D, T>::bytes;
   static unsigned configured = 0;   // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -398,7 +518,10 @@ cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
 
 }  // namespace
 
-size_t gdn_smem_bytes(int D) { return D == 64 ? GdnSmem<64>::bytes : GdnSmem<128>::bytes; }
+size_t gdn_smem_bytes(int D, int dtype) {
+  if (D == 64) return dtype == SA_BF16 ? GdnSmem<64, __nv_bfloat16>::bytes : GdnSmem<64, float>::bytes;
+  return dtype == SA_BF16 ? GdnSmem<128, __nv_bfloat16>::bytes : GdnSmem<128, float>::bytes;
+}
 
 cudaError_t launch_gdn(const GdnParams& p, int D, int dtype, cudaStream_t st) {
   if (p.n_streams <= 0 || p.T <= 0) return cudaSuccess;

@@ -113,7 +113,7 @@ struct GdnParams {
   int32_t pad_;
   int32_t stream_of[SA_MAX_STREAMS];
 };
-size_t gdn_smem_bytes(int D);
+size_t gdn_smem_bytes(int D, int dtype);
 cudaError_t launch_gdn(const GdnParams& p, int D, int dtype, cudaStream_t st);
 
 cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStream_t st);

@@ -344,9 +344,10 @@ sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, co
   if (cfg->tokens > 0) {
     if (!q || !k || !v || !g || !beta || !out)
       return fail(SA_ERR_INVALID_ARG, "q, k, v, g, beta and out must be non-NULL");
-    const uintptr_t ptrs[4] = {(uintptr_t)q, (uintptr_t)k, (uintptr_t)v, (uintptr_t)out};
+    const uintptr_t ptrs[3] = {(uintptr_t)q, (uintptr_t)k, (uintptr_t)v};
     for (uintptr_t a : ptrs)
-      if (a % esz) return fail(SA_ERR_INVALID_ARG, "q, k, v and out must be aligned to their element");
+      if (a % 16) return fail(SA_ERR_INVALID_ARG, "q, k and v must be 16-byte aligned");
+    if ((uintptr_t)out % esz) return fail(SA_ERR_INVALID_ARG, "out must be aligned to its element");
     if ((uintptr_t)g % 4 || (uintptr_t)beta % 4)
       return fail(SA_ERR_INVALID_ARG, "g and beta must be 4-byte aligned");
   }
