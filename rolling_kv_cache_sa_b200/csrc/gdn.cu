@@ -42,13 +42,16 @@ namespace {
 constexpr int kCt = 64;         // tokens per sub-chunk
 constexpr int kDvs = 32;        // state rows (value dims) per CTA
 constexpr int kGdnThreads = 256;
-constexpr int kLp = kCt + 1;    // row pitch of the 64 x 64 matrices
-constexpr int kVp = kDvs + 1;   // row pitch of the 64 x 32 matrices
+constexpr int kLp = kCt + 4;    // row pitch of the 64 x 64 matrices (16-byte rows)
+constexpr int kVp = kDvs + 4;   // row pitch of the 64 x 32 matrices (16-byte rows)
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Shared-memory layout in floats. Rows of K^, Q^ and S have pitch D + 4: a
+// Shared-memory layout in floats. Rows of K^ and Q^ have pitch D + 4: a
 // multiple of 4 (16-byte aligned rows) whose 16-byte groups step by an odd
 // count, so float4 reads of consecutive rows fall in different bank groups.
+// The state slice has pitch D with its 16-byte groups XOR-swizzled by
+// (row / 4) mod 8, so float4 reads of rows 4x + i (x = 0..7) are conflict
+// free. The merge scratch shares the storage of U (never live together).
 // The staging area receives the next sub-chunk's raw q, k rows and value
 // slice (input element type) by cp.async while the current one is computed.
 template <int D, typename T>
@@ -56,13 +59,13 @@ struct GdnSmem {
   static constexpr int KP = D + 4;
   static constexpr int kh = 0;                    // [64][KP] normalised keys
   static constexpr int qh = kh + kCt * KP;        // [64][KP] normalised queries
-  static constexpr int st = qh + kCt * KP;        // [32][KP] state slice S0
-  static constexpr int lm = st + kDvs * KP;       // [64][65] L (strictly lower)
-  static constexpr int pm = lm + kCt * kLp;       // [64][65] scale e^(G_t-G_s) q_t.k_s (s <= t)
-  static constexpr int tm = pm + kCt * kLp;       // [64][65] (I + L)^-1 (lower)
-  static constexpr int xm = tm + kCt * kLp;       // [32][33] merge scratch
-  static constexpr int rv = xm + 32 * 33;         // [64][33] v slice, then the right-hand side
-  static constexpr int uv = rv + kCt * kVp;       // [64][33] corrected values u
+  static constexpr int st = qh + kCt * KP;        // [32][D] state slice S0 (swizzled)
+  static constexpr int lm = st + kDvs * D;        // [64][68] L (strictly lower)
+  static constexpr int pm = lm + kCt * kLp;       // [64][68] scale e^(G_t-G_s) q_t.k_s (s <= t)
+  static constexpr int tm = pm + kCt * kLp;       // [64][68] (I + L)^-1 (lower)
+  static constexpr int rv = tm + kCt * kLp;       // [64][36] v slice, right-hand side, then
+                                                  //          u_t e^(G_last - G_t)
+  static constexpr int uv = rv + kCt * kVp;       // [64][36] corrected values u; merge scratch
   static constexpr int gs = uv + kCt * kVp;       // [64] in-warp prefix sums of g log2(e)
   static constexpr int bs = gs + kCt;             // [64] beta
   static constexpr int ws = bs + kCt;             // [64] e^(G_last - G_t)
@@ -133,7 +136,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
   float* Lm = sm + L::lm;
   float* Pm = sm + L::pm;
   float* Tm = sm + L::tm;
-  float* Xm = sm + L::xm;
+  float* Xm = sm + L::uv;   // [32][33] merge scratch (before U is written)
   float* Rv = sm + L::rv;
   float* Uv = sm + L::uv;
   float* Gs = sm + L::gs;
@@ -193,6 +196,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
   // sums lack warp 0's total, added here).
   auto gcum = [&](int t) -> float { return Gs[t] + (t >= 32 ? Gs[31] : 0.f); };
 
+  // Offset of (row r, column col) of the state slice, col a multiple of 4.
+  auto st_off = [](int r, int col) -> int {
+    return r * D + (((col >> 2) ^ ((r >> 2) & 7)) << 2);
+  };
   // State rows this thread updates: row uc, columns uj + 32 m (+0..3).
   const int uc = warp * 4 + (lane >> 3);
   const int uj = 4 * (lane & 7);
@@ -200,12 +207,12 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
 #pragma unroll
   for (int m = 0; m < NJ; ++m) {
     sreg[m] = *reinterpret_cast<const float4*>(Sg + (size_t)uc * D + uj + 32 * m);
-    st4(St + uc * KP + uj + 32 * m, sreg[m]);
+    st4(St + st_off(uc, uj + 32 * m), sreg[m]);
   }
-  // Tokens and state rows of the products with D columns (right-hand side,
-  // U, outputs): tokens tw + 16a (a < 4), rows cw + 16bb (bb < 2).
-  const int tw = warp * 2 + (lane >> 4);
-  const int cw = lane & 15;
+  // Tokens and state rows of the products with 32 state rows (right-hand
+  // side, U, outputs): tokens tq + 32a (a < 2), rows cq .. cq + 3.
+  const int tq = warp * 4 + (lane >> 3);
+  const int cq = 4 * (lane & 7);
 
   float gnext = 0.f, bnext = 0.f;
   prefetch(0, gnext, bnext);
@@ -310,35 +317,42 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
     // ---- K^ S0^T and Q^ S0^T for this CTA's rows. The right-hand side
     // beta_t (v_t - e^(G_t) (S0 k_t)) replaces v in Rv; the inter-chunk part of
     // the output, scale e^(G_t) (S0 q_t), stays in registers.
-    float oin[4][2];
+    float oin[2][4];
     {
-      float aks[4][2], aqs[4][2];
+      float aks[2][4], aqs[2][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) aks[a][0] = aks[a][1] = aqs[a][0] = aqs[a][1] = 0.f;
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) aks[a][i] = aqs[a][i] = 0.f;
 #pragma unroll 2
       for (int d = 0; d < D; d += 4) {
-        const float4 s0 = ld4(St + cw * KP + d);
-        const float4 s1 = ld4(St + (cw + 16) * KP + d);
+        float4 sr[4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const float4 k4 = ld4(Kh + (tw + 16 * a) * KP + d);
-          const float4 q4 = ld4(Qh + (tw + 16 * a) * KP + d);
-          aks[a][0] = dot4(k4, s0, aks[a][0]);
-          aks[a][1] = dot4(k4, s1, aks[a][1]);
-          aqs[a][0] = dot4(q4, s0, aqs[a][0]);
-          aqs[a][1] = dot4(q4, s1, aqs[a][1]);
+        for (int i = 0; i < 4; ++i) sr[i] = ld4(St + st_off(cq + i, d));
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          const float4 k4 = ld4(Kh + (tq + 32 * a) * KP + d);
+          const float4 q4 = ld4(Qh + (tq + 32 * a) * KP + d);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            aks[a][i] = dot4(k4, sr[i], aks[a][i]);
+            aqs[a][i] = dot4(q4, sr[i], aqs[a][i]);
+          }
         }
       }
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const int t = tw + 16 * a;
+      for (int a = 0; a < 2; ++a) {
+        const int t = tq + 32 * a;
         const float gam = ex2f(gcum(t));
+        const float bt = Bs[t];
+        float4 r = ld4(Rv + t * kVp + cq);
+        r.x = bt * (r.x - gam * aks[a][0]);
+        r.y = bt * (r.y - gam * aks[a][1]);
+        r.z = bt * (r.z - gam * aks[a][2]);
+        r.w = bt * (r.w - gam * aks[a][3]);
+        st4(Rv + t * kVp + cq, r);
 #pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const int c = cw + 16 * bb;
-          Rv[t * kVp + c] = Bs[t] * (Rv[t * kVp + c] - gam * aks[a][bb]);
-          oin[a][bb] = p.scale * gam * aqs[a][bb];
-        }
+        for (int i = 0; i < 4; ++i) oin[a][i] = p.scale * gam * aqs[a][i];
       }
     }
     __syncthreads();
@@ -389,84 +403,121 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
       Tm[(r0 + 16 + i) * kLp + r0 + j] = -acc;
     }
     __syncthreads();
-    // ---- merge to the full 64 x 64 inverse (rows 32.., columns 0..31)
+    // ---- merge to the full 64 x 64 inverse (rows 32.., columns 0..31): warp
+    // w takes rows 4w .. 4w+3 of the 32 x 32 block, lane j its column j
+    {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int j = lane;
 #pragma unroll
-    for (int e0 = 0; e0 < 1024; e0 += kGdnThreads) {
-      const int e = e0 + tid;
-      const int i = e >> 5, j = e & 31;
-      float acc = 0.f;
+      for (int s4 = 0; s4 < 32; s4 += 4) {
+        float4 l4[4];
 #pragma unroll
-      for (int s2 = 0; s2 < 32; ++s2)
-        if (s2 >= j) acc = fmaf(Lm[(32 + i) * kLp + s2], Tm[s2 * kLp + j], acc);
-      Xm[i * 33 + j] = acc;
+        for (int r = 0; r < 4; ++r) l4[r] = ld4(Lm + (32 + warp * 4 + r) * kLp + s4);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float tv = s4 + u >= j ? Tm[(s4 + u) * kLp + j] : 0.f;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const float lv = u == 0 ? l4[r].x : u == 1 ? l4[r].y : u == 2 ? l4[r].z : l4[r].w;
+            acc[r] = fmaf(lv, tv, acc[r]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) Xm[(warp * 4 + r) * 33 + j] = acc[r];
     }
     __syncthreads();
+    {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int j = lane;
 #pragma unroll
-    for (int e0 = 0; e0 < 1024; e0 += kGdnThreads) {
-      const int e = e0 + tid;
-      const int i = e >> 5, j = e & 31;
-      float acc = 0.f;
+      for (int s4 = 0; s4 < 32; s4 += 4) {
+        float4 t4[4];
 #pragma unroll
-      for (int s2 = 0; s2 < 32; ++s2)
-        if (s2 <= i) acc = fmaf(Tm[(32 + i) * kLp + 32 + s2], Xm[s2 * 33 + j], acc);
-      Tm[(32 + i) * kLp + j] = -acc;
+        for (int r = 0; r < 4; ++r) t4[r] = ld4(Tm + (32 + warp * 4 + r) * kLp + 32 + s4);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float xv = Xm[(s4 + u) * 33 + j];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const float tv = u == 0 ? t4[r].x : u == 1 ? t4[r].y : u == 2 ? t4[r].z : t4[r].w;
+            if (s4 + u <= warp * 4 + r) acc[r] = fmaf(tv, xv, acc[r]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) Tm[(32 + warp * 4 + r) * kLp + j] = -acc[r];
     }
     __syncthreads();
 
     // ---- corrected values U = (I + L)^-1 RHS. Rows of RHS past n are zero,
     // so the sums run over all 64 tokens.
+    float uacc[2][4];
     {
-      float acc[4][2];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0.f;
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) uacc[a][i] = 0.f;
 #pragma unroll 8
       for (int s2 = 0; s2 < kCt; ++s2) {
-        const float r0 = Rv[s2 * kVp + cw];
-        const float r1 = Rv[s2 * kVp + cw + 16];
+        const float4 r4 = ld4(Rv + s2 * kVp + cq);
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const int t = tw + 16 * a;
+        for (int a = 0; a < 2; ++a) {
+          const int t = tq + 32 * a;
           const float tv = s2 <= t ? Tm[t * kLp + s2] : 0.f;
-          acc[a][0] = fmaf(tv, r0, acc[a][0]);
-          acc[a][1] = fmaf(tv, r1, acc[a][1]);
+          uacc[a][0] = fmaf(tv, r4.x, uacc[a][0]);
+          uacc[a][1] = fmaf(tv, r4.y, uacc[a][1]);
+          uacc[a][2] = fmaf(tv, r4.z, uacc[a][2]);
+          uacc[a][3] = fmaf(tv, r4.w, uacc[a][3]);
         }
       }
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        Uv[(tw + 16 * a) * kVp + cw] = acc[a][0];
-        Uv[(tw + 16 * a) * kVp + cw + 16] = acc[a][1];
-      }
+      for (int a = 0; a < 2; ++a)
+        st4(Uv + (tq + 32 * a) * kVp + cq,
+            make_float4(uacc[a][0], uacc[a][1], uacc[a][2], uacc[a][3]));
     }
     __syncthreads();
 
-    // ---- outputs: inter-chunk part + intra-chunk part P U
+    // ---- u_t e^(G_last - G_t) replaces the right-hand side (all of it has
+    // been read); outputs: inter-chunk part + intra-chunk part P U
     {
-      float acc[4][2];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) acc[a][0] = oin[a][0], acc[a][1] = oin[a][1];
+      for (int a = 0; a < 2; ++a) {
+        const int t = tq + 32 * a;
+        const float w = Ws[t];
+        st4(Rv + t * kVp + cq, make_float4(uacc[a][0] * w, uacc[a][1] * w, uacc[a][2] * w,
+                                           uacc[a][3] * w));
+      }
+      float acc[2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[a][i] = oin[a][i];
 #pragma unroll 8
       for (int s2 = 0; s2 < kCt; ++s2) {
-        const float u0 = Uv[s2 * kVp + cw];
-        const float u1 = Uv[s2 * kVp + cw + 16];
+        const float4 u4 = ld4(Uv + s2 * kVp + cq);
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const int t = tw + 16 * a;
+        for (int a = 0; a < 2; ++a) {
+          const int t = tq + 32 * a;
           const float pv = s2 <= t ? Pm[t * kLp + s2] : 0.f;
-          acc[a][0] = fmaf(pv, u0, acc[a][0]);
-          acc[a][1] = fmaf(pv, u1, acc[a][1]);
+          acc[a][0] = fmaf(pv, u4.x, acc[a][0]);
+          acc[a][1] = fmaf(pv, u4.y, acc[a][1]);
+          acc[a][2] = fmaf(pv, u4.z, acc[a][2]);
+          acc[a][3] = fmaf(pv, u4.w, acc[a][3]);
         }
       }
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const int t = tw + 16 * a;
+      for (int a = 0; a < 2; ++a) {
+        const int t = tq + 32 * a;
         if (t < n) {
-          const size_t o = bh0 + (size_t)(t0 + t) * tok_stride + vcol + cw;
-          st_out(out, o, acc[a][0]);
-          st_out(out, o + 16, acc[a][1]);
+          const size_t o = bh0 + (size_t)(t0 + t) * tok_stride + vcol + cq;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) st_out(out, o + i, acc[a][i]);
         }
       }
     }
-    // ---- state: S = e^(G_last) S0 + sum_t e^(G_last - G_t) u_t k_t^T
+    __syncthreads();
+    // ---- state: S = e^(G_last) S0 + sum_t (u_t e^(G_last - G_t)) k_t^T
     // (u and k are zero past n)
     {
       const float dec = ex2f(gcum(kCt - 1));
@@ -479,7 +530,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
       }
 #pragma unroll 8
       for (int t = 0; t < kCt; ++t) {
-        const float uw = Uv[t * kVp + uc] * Ws[t];
+        const float uw = Rv[t * kVp + uc];
 #pragma unroll
         for (int m = 0; m < NJ; ++m) {
           const float4 k4 = ld4(Kh + t * KP + uj + 32 * m);
@@ -490,7 +541,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
         }
       }
 #pragma unroll
-      for (int m = 0; m < NJ; ++m) st4(St + uc * KP + uj + 32 * m, sreg[m]);
+      for (int m = 0; m < NJ; ++m) st4(St + st_off(uc, uj + 32 * m), sreg[m]);
     }
     __syncthreads();
   }
