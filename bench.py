@@ -15,6 +15,10 @@ the max over ranks.
 
 --impl reference times the fp64 CPU oracle (the reference implementation of
 this repository) on the host cores, on a bounded sample of the same workload.
+
+--path gdn measures the Gated DeltaNet block (sa_gdn_chunk) on the same
+stream shape instead: one step = 64 calls of 2,048 tokens from a zero state;
+its roofline is the fp32 FMA peak of the CUDA cores it runs on.
 """
 from __future__ import annotations
 

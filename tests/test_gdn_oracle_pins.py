@@ -196,3 +196,61 @@ def test_bad_arguments(bad):
     rc = L.orc_gdn_chunk(H, 4, 1, 1.0, sp, x.ctypes.data, x.ctypes.data, x.ctypes.data,
                          gg.ctypes.data, gg.ctypes.data, x.ctypes.data)
     assert rc == -1
+
+
+def _tri_inv_blocked(L):
+    """(I + L)^-1 for strictly lower-triangular L (64 x 64): 16 x 16 diagonal
+    blocks by forward substitution, then two merges with
+    [A 0; C B]^-1 = [A^-1 0; -B^-1 C A^-1  B^-1]."""
+    n = L.shape[0]
+    T = np.zeros_like(L)
+    for b0 in range(0, n, 16):
+        for j in range(16):
+            x = np.zeros(16)
+            x[j] = 1.0
+            for t in range(j + 1, 16):
+                x[t] = -L[b0 + t, b0:b0 + t] @ x[:t]
+            T[b0:b0 + 16, b0 + j] = x
+    for w in (16, 32):
+        for b0 in range(0, n, 2 * w):
+            T11 = T[b0:b0 + w, b0:b0 + w]
+            T22 = T[b0 + w:b0 + 2 * w, b0 + w:b0 + 2 * w]
+            T[b0 + w:b0 + 2 * w, b0:b0 + w] = -T22 @ (L[b0 + w:b0 + 2 * w, b0:b0 + w] @ T11)
+    return T
+
+
+def _chunkwise(scale, S, q, k, v, g, beta, ct=64):
+    """The chunkwise (WY) form of the gated delta rule on sub-chunks of ct
+    tokens, one head: (I + L) U = diag(beta)(V - diag(e^G) K S^T), outputs and
+    end state by triangular products. Ragged tail rows are zero."""
+    Tn, D = q.shape
+    out = np.zeros_like(q)
+    for t0 in range(0, Tn, ct):
+        n = min(ct, Tn - t0)
+        K = np.zeros((ct, D)); Q = np.zeros((ct, D)); V = np.zeros((ct, S.shape[0]))
+        gg = np.zeros(ct); bb = np.zeros(ct)
+        K[:n], Q[:n], V[:n] = _unit(k[t0:t0 + n]), _unit(q[t0:t0 + n]), v[t0:t0 + n]
+        gg[:n], bb[:n] = g[t0:t0 + n], beta[t0:t0 + n]
+        G = np.cumsum(gg)
+        E = np.exp(G[:, None] - G[None, :])
+        L = np.tril(bb[:, None] * E * (K @ K.T), -1)
+        P = np.tril(scale * E * (Q @ K.T), 0)
+        U = _tri_inv_blocked(L) @ (bb[:, None] * (V - np.exp(G)[:, None] * (K @ S.T)))
+        out[t0:t0 + n] = (scale * np.exp(G)[:, None] * (Q @ S.T) + P @ U)[:n]
+        S = np.exp(G[-1]) * S + (U * np.exp(G[-1] - G)[:, None]).T @ K
+    return out, S
+
+
+@pytest.mark.parametrize("T,D,g_scale", [(150, 16, 0.3), (64, 32, 0.01), (200, 8, 2.0),
+                                         (130, 64, 0.002)])
+def test_chunkwise_form_equals_recurrence(T, D, g_scale):
+    """The algebra the GPU kernel runs (chunkwise WY form with a blocked
+    triangular inverse, ragged last sub-chunk) reproduces the token-by-token
+    recurrence of the oracle."""
+    q, k, v, g, beta = _rand(T, 1, D, g_scale)
+    S0 = 0.3 * RNG.standard_normal((1, D, D))
+    st = S0.copy()
+    ref = O.gdn_chunk(0.5, st, q, k, v, g, beta)
+    o, S = _chunkwise(0.5, S0[0].copy(), q[:, 0], k[:, 0], v[:, 0], g[:, 0], beta[:, 0])
+    np.testing.assert_allclose(o, ref[:, 0], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(S, st[0], atol=1e-12, rtol=0)
