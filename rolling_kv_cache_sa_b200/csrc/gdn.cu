@@ -126,7 +126,6 @@ template <int D, typename T>
 __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_constant__ GdnParams p) {
   using L = GdnSmem<D, T>;
   constexpr int KP = L::KP;
-  constexpr int NJ = D / 32;                         // float4 groups of state per thread
   constexpr int kRow16 = D * (int)sizeof(T) / 16;    // 16-byte pieces of a raw row
   constexpr int kV16 = kDvs * (int)sizeof(T) / 16;   // 16-byte pieces of a value slice
   extern __shared__ __align__(16) float sm[];
@@ -198,17 +197,21 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
 
   // Offset of (row r, column col) of the state slice, col a multiple of 4.
   auto st_off = [](int r, int col) -> int {
-    return r * D + (((col >> 2) ^ ((r >> 2) & 7)) << 2);
+    return r * D + ((((col >> 2) ^ ((r >> 2) & 7)) << 2) | (col & 3));
   };
-  // State rows this thread updates: row uc, columns uj + 32 m (+0..3).
-  const int uc = warp * 4 + (lane >> 3);
-  const int uj = 4 * (lane & 7);
-  float4 sreg[NJ];
+  // State block this thread updates: rows 4 warp + i (i < 4), columns
+  // NC lane .. NC lane + NC - 1 (NC = D / 32 = 4 or 2).
+  constexpr int NC = D / 32;
+  const int ur = warp * 4;
+  const int ucol = NC * lane;
+  float sreg[4][NC];
 #pragma unroll
-  for (int m = 0; m < NJ; ++m) {
-    sreg[m] = *reinterpret_cast<const float4*>(Sg + (size_t)uc * D + uj + 32 * m);
-    st4(St + st_off(uc, uj + 32 * m), sreg[m]);
-  }
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      sreg[i][c] = Sg[(size_t)(ur + i) * D + ucol + c];
+      St[st_off(ur + i, ucol + c)] = sreg[i][c];
+    }
   // Tokens and state rows of the products with 32 state rows (right-hand
   // side, U, outputs): tokens tq + 32a (a < 2), rows cq .. cq + 3.
   const int tq = warp * 4 + (lane >> 3);
@@ -522,32 +525,39 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
     {
       const float dec = ex2f(gcum(kCt - 1));
 #pragma unroll
-      for (int m = 0; m < NJ; ++m) {
-        sreg[m].x *= dec;
-        sreg[m].y *= dec;
-        sreg[m].z *= dec;
-        sreg[m].w *= dec;
-      }
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < NC; ++c) sreg[i][c] *= dec;
 #pragma unroll 8
       for (int t = 0; t < kCt; ++t) {
-        const float uw = Rv[t * kVp + uc];
+        const float4 uw = ld4(Rv + t * kVp + ur);
+        float kv[NC];
+        if constexpr (NC == 4) {
+          const float4 k4 = ld4(Kh + t * KP + ucol);
+          kv[0] = k4.x, kv[1] = k4.y, kv[2] = k4.z, kv[3] = k4.w;
+        } else {
+          const float2 k2 = *reinterpret_cast<const float2*>(Kh + t * KP + ucol);
+          kv[0] = k2.x, kv[1] = k2.y;
+        }
 #pragma unroll
-        for (int m = 0; m < NJ; ++m) {
-          const float4 k4 = ld4(Kh + t * KP + uj + 32 * m);
-          sreg[m].x = fmaf(uw, k4.x, sreg[m].x);
-          sreg[m].y = fmaf(uw, k4.y, sreg[m].y);
-          sreg[m].z = fmaf(uw, k4.z, sreg[m].z);
-          sreg[m].w = fmaf(uw, k4.w, sreg[m].w);
+        for (int c = 0; c < NC; ++c) {
+          sreg[0][c] = fmaf(uw.x, kv[c], sreg[0][c]);
+          sreg[1][c] = fmaf(uw.y, kv[c], sreg[1][c]);
+          sreg[2][c] = fmaf(uw.z, kv[c], sreg[2][c]);
+          sreg[3][c] = fmaf(uw.w, kv[c], sreg[3][c]);
         }
       }
 #pragma unroll
-      for (int m = 0; m < NJ; ++m) st4(St + st_off(uc, uj + 32 * m), sreg[m]);
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < NC; ++c) St[st_off(ur + i, ucol + c)] = sreg[i][c];
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int m = 0; m < NJ; ++m)
-    *reinterpret_cast<float4*>(Sg + (size_t)uc * D + uj + 32 * m) = sreg[m];
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < NC; ++c) Sg[(size_t)(ur + i) * D + ucol + c] = sreg[i][c];
 }
 
 template <int D, typename T>
