@@ -195,7 +195,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
   // sums lack warp 0's total, added here).
   auto gcum = [&](int t) -> float { return Gs[t] + (t >= 32 ? Gs[31] : 0.f); };
 
-  // Offset of (row r, column col) of the state slice, col a multiple of 4.
+  // Offset of (row r, column col) of the state slice: 16-byte group col / 4
+  // is stored at group (col / 4) xor ((r / 4) mod 8) of row r.
   auto st_off = [](int r, int col) -> int {
     return r * D + ((((col >> 2) ^ ((r >> 2) & 7)) << 2) | (col & 3));
   };
