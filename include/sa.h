@@ -404,17 +404,33 @@ typedef struct {
  *          q, k and v 16-byte aligned, out aligned to its element);
  *   g      [B][T][H] fp32, log decay of each token (<= 0; exp(g) multiplies S);
  *   beta   [B][T][H] fp32, write strength of each token (in [0, 1] for a
- *          contracting update; other values are computed as given).
+ *          contracting update; other values are computed as given);
+ *   workspace  scratch of workspace_bytes >= sa_gdn_workspace_size(cfg),
+ *          16-byte aligned; contents need not be kept between calls. The call
+ *          runs two kernels: one computes, for every 64-token block, the
+ *          triangular inverse and the masked q.k matrix of the chunkwise form
+ *          into the workspace; the other walks the blocks in order and
+ *          updates the state.
  * active: host array of B flags, NULL = all; an inactive stream's state and
  * out rows are untouched. Arithmetic is fp32 with fp32 state; outputs are
  * rounded once to cfg->dtype. Asynchronous on `stream`, graph-capturable.
- * Errors: SA_ERR_INVALID_ARG (cfg, a NULL pointer with tokens > 0, alignment),
- * SA_ERR_UNSUPPORTED (no compute capability 10.x device, or a size that does
- * not fit), SA_ERR_CUDA (the launch failed).
+ * Errors: SA_ERR_INVALID_ARG (cfg, a NULL pointer with tokens > 0, alignment,
+ * a workspace smaller than sa_gdn_workspace_size), SA_ERR_UNSUPPORTED (no
+ * compute capability 10.x device, or a size that does not fit), SA_ERR_CUDA
+ * (the launch failed).
  */
 sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, const void* k,
                        const void* v, const float* g, const float* beta, void* out,
-                       const uint8_t* active, sa_stream_t stream);
+                       void* workspace, size_t workspace_bytes, const uint8_t* active,
+                       sa_stream_t stream);
+
+/*
+ * Bytes of the device workspace sa_gdn_chunk needs for cfg: 32 KiB per
+ * (stream, head, started 64-token block of the call), i.e.
+ * batch * heads * ceil(tokens / 64) * 32768.
+ * Errors: SA_ERR_INVALID_ARG (cfg invalid or bytes NULL), SA_ERR_UNSUPPORTED.
+ */
+sa_status sa_gdn_workspace_size(const sa_gdn_config* cfg, size_t* bytes);
 
 const char* sa_last_error_string(void);
 

@@ -98,6 +98,8 @@ size_t attend_partials_bytes(int D, int num_sms, int64_t max_units);
 
 // Gated DeltaNet block (gdn.cu): T tokens of each listed stream; q, k, v, out
 // [B][T][H][D], g and beta [B][T][H], state [B][H][D][D] fp32 in place.
+// workspace: T and P of every (listed stream, head, 64-token sub-chunk),
+// gdn_workspace_bytes(n_streams, H, T) bytes, 16-byte aligned.
 struct GdnParams {
   float* state;
   const void* q;
@@ -106,13 +108,15 @@ struct GdnParams {
   const float* g;
   const float* beta;
   void* out;
+  float* workspace;
   int64_t T;
   int32_t H;
   float scale;
   int32_t n_streams;
-  int32_t pad_;
+  int32_t n_sub;       // ceil(T / 64)
   int32_t stream_of[SA_MAX_STREAMS];
 };
+size_t gdn_workspace_bytes(int B, int H, int64_t T);
 size_t gdn_smem_bytes(int D, int dtype);
 cudaError_t launch_gdn(const GdnParams& p, int D, int dtype, cudaStream_t st);
 

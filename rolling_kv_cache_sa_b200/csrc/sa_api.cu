@@ -320,9 +320,8 @@ sa_status sa_wait_probe(uint64_t limit_ns, int64_t* waited_ns, sa_stream_t strea
   return SA_OK;
 }
 
-sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, const void* k,
-                       const void* v, const float* g, const float* beta, void* out,
-                       const uint8_t* active, sa_stream_t stream) {
+namespace {
+sa_status validate_gdn_config(const sa_gdn_config* cfg) {
   if (!cfg) return fail(SA_ERR_INVALID_ARG, "config is NULL");
   if (cfg->batch < 1 || cfg->batch > SA_MAX_STREAMS)
     return fail(SA_ERR_INVALID_ARG, "batch must be in [1, %d], got %d", SA_MAX_STREAMS, cfg->batch);
@@ -338,6 +337,27 @@ sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, co
   const size_t esz = cfg->dtype == SA_F32 ? 4 : 2;
   if ((double)cfg->batch * (double)cfg->tokens * cfg->heads * cfg->head_dim * esz > 9.0e18)
     return fail(SA_ERR_UNSUPPORTED, "batch*tokens*heads*head_dim too large");
+  if ((cfg->tokens + 63) / 64 > 65535)
+    return fail(SA_ERR_UNSUPPORTED, "tokens must be at most 65535 * 64 per call");
+  return SA_OK;
+}
+}  // namespace
+
+sa_status sa_gdn_workspace_size(const sa_gdn_config* cfg, size_t* bytes) {
+  sa_status st = validate_gdn_config(cfg);
+  if (st != SA_OK) return st;
+  if (!bytes) return fail(SA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = sa::gdn_workspace_bytes(cfg->batch, cfg->heads, cfg->tokens);
+  return SA_OK;
+}
+
+sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, const void* k,
+                       const void* v, const float* g, const float* beta, void* out,
+                       void* workspace, size_t workspace_bytes, const uint8_t* active,
+                       sa_stream_t stream) {
+  sa_status vst = validate_gdn_config(cfg);
+  if (vst != SA_OK) return vst;
+  const size_t esz = cfg->dtype == SA_F32 ? 4 : 2;
   if (!state) return fail(SA_ERR_INVALID_ARG, "state is NULL");
   if (reinterpret_cast<uintptr_t>(state) % 16)
     return fail(SA_ERR_INVALID_ARG, "state must be 16-byte aligned");
@@ -350,6 +370,12 @@ sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, co
     if ((uintptr_t)out % esz) return fail(SA_ERR_INVALID_ARG, "out must be aligned to its element");
     if ((uintptr_t)g % 4 || (uintptr_t)beta % 4)
       return fail(SA_ERR_INVALID_ARG, "g and beta must be 4-byte aligned");
+    const size_t need = sa::gdn_workspace_bytes(cfg->batch, cfg->heads, cfg->tokens);
+    if (!workspace || (uintptr_t)workspace % 16)
+      return fail(SA_ERR_INVALID_ARG, "workspace must be non-NULL and 16-byte aligned");
+    if (workspace_bytes < need)
+      return fail(SA_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed (sa_gdn_workspace_size)",
+                  workspace_bytes, need);
   }
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -372,7 +398,9 @@ sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, co
   p.g = g;
   p.beta = beta;
   p.out = out;
+  p.workspace = static_cast<float*>(workspace);
   p.T = cfg->tokens;
+  p.n_sub = (int32_t)((cfg->tokens + 63) / 64);
   p.H = cfg->heads;
   p.scale = cfg->scale > 0.f ? cfg->scale : (float)(1.0 / sqrt((double)cfg->head_dim));
   NvtxRange nv("sa_gdn_chunk");

@@ -137,28 +137,43 @@ def test_gdn_chunk_validates_config(field, value):
     c = _gdn_cfg(**{field: value})
     buf = ctypes.create_string_buffer(1 << 12)
     p = ctypes.cast(ctypes.addressof(buf) + (16 - ctypes.addressof(buf) % 16) % 16, ctypes.c_void_p)
-    st = _lib.lib().sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, None, None)
+    st = _lib.lib().sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, p, 1 << 30, None, None)
     assert st == _lib.SA_ERR_INVALID_ARG
     assert _lib.lib().sa_last_error_string()
+    n = ctypes.c_size_t()
+    assert _lib.lib().sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == \
+        _lib.SA_ERR_INVALID_ARG
 
 
 def test_gdn_chunk_validates_pointers():
     L = _lib.lib()
     c = _gdn_cfg()
-    assert L.sa_gdn_chunk(None, None, None, None, None, None, None, None, None, None) == \
-        _lib.SA_ERR_INVALID_ARG
+    assert L.sa_gdn_chunk(None, None, None, None, None, None, None, None, None, 0, None,
+                          None) == _lib.SA_ERR_INVALID_ARG
     buf = ctypes.create_string_buffer(1 << 12)
     base = ctypes.addressof(buf) + (16 - ctypes.addressof(buf) % 16) % 16
     p = ctypes.c_void_p(base)
-    assert L.sa_gdn_chunk(ctypes.byref(c), None, p, p, p, p, p, p, None, None) == \
+    big = 1 << 30
+    assert L.sa_gdn_chunk(ctypes.byref(c), None, p, p, p, p, p, p, p, big, None, None) == \
         _lib.SA_ERR_INVALID_ARG                      # state NULL
-    assert L.sa_gdn_chunk(ctypes.byref(c), ctypes.c_void_p(base + 4), p, p, p, p, p, p, None,
-                          None) == _lib.SA_ERR_INVALID_ARG   # state not 16-byte aligned
-    assert L.sa_gdn_chunk(ctypes.byref(c), p, p, None, p, p, p, p, None, None) == \
+    assert L.sa_gdn_chunk(ctypes.byref(c), ctypes.c_void_p(base + 4), p, p, p, p, p, p, p, big,
+                          None, None) == _lib.SA_ERR_INVALID_ARG   # state not 16-byte aligned
+    assert L.sa_gdn_chunk(ctypes.byref(c), p, p, None, p, p, p, p, p, big, None, None) == \
         _lib.SA_ERR_INVALID_ARG                      # k NULL with tokens > 0
-    assert L.sa_gdn_chunk(ctypes.byref(c), p, ctypes.c_void_p(base + 1), p, p, p, p, p, None,
-                          None) == _lib.SA_ERR_INVALID_ARG   # q misaligned for bf16
+    assert L.sa_gdn_chunk(ctypes.byref(c), p, ctypes.c_void_p(base + 1), p, p, p, p, p, p, big,
+                          None, None) == _lib.SA_ERR_INVALID_ARG   # q misaligned for bf16
     assert b"aligned" in L.sa_last_error_string()
+    assert L.sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, None, big, None, None) == \
+        _lib.SA_ERR_INVALID_ARG                      # workspace NULL
+    n = ctypes.c_size_t()
+    assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
+    assert n.value == 2 * 3 * 1 * 32768              # B * H * ceil(64 / 64) * 32 KiB
+    c.tokens = 65
+    assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
+    assert n.value == 2 * 3 * 2 * 32768
+    assert L.sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, p, n.value - 16, None,
+                          None) == _lib.SA_ERR_INVALID_ARG   # workspace too small
+    assert b"workspace" in L.sa_last_error_string()
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device refusal")
@@ -166,5 +181,5 @@ def test_gdn_chunk_without_device_is_refused():
     buf = ctypes.create_string_buffer(1 << 12)
     p = ctypes.c_void_p(ctypes.addressof(buf) + (16 - ctypes.addressof(buf) % 16) % 16)
     c = _gdn_cfg()
-    assert _lib.lib().sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, None, None) == \
-        _lib.SA_ERR_UNSUPPORTED
+    assert _lib.lib().sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, p, 1 << 30, None,
+                                   None) == _lib.SA_ERR_UNSUPPORTED
