@@ -183,3 +183,21 @@ def test_gdn_chunk_without_device_is_refused():
     c = _gdn_cfg()
     assert _lib.lib().sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, p, 1 << 30, None,
                                    None) == _lib.SA_ERR_UNSUPPORTED
+
+
+def test_gdn_binding_checks_shapes_before_the_call():
+    """The Python binding refuses mismatched tensors before reaching the library."""
+    from rolling_kv_cache_sa_b200 import sa_gdn_chunk
+    B, T, H, D = 2, 5, 3, 64
+    q = torch.zeros(B, T, H, D)
+    ok = dict(state=torch.zeros(B, H, D, D), k=torch.zeros_like(q), v=torch.zeros_like(q),
+              g=torch.zeros(B, T, H), beta=torch.zeros(B, T, H), out=torch.zeros_like(q))
+    bad = [("state", torch.zeros(B, H, D, D + 1)), ("k", torch.zeros(B, T, H, D + 1)),
+           ("v", torch.zeros(B, T, H, D, dtype=torch.bfloat16)), ("g", torch.zeros(B, T, H + 1)),
+           ("beta", torch.zeros(B, T, H, dtype=torch.float64)),
+           ("out", torch.zeros(B, T, H, D).transpose(0, 1).contiguous().transpose(0, 1))]
+    for name, t in bad:
+        args = dict(ok, **{name: t})
+        with pytest.raises(ValueError, match=name):
+            sa_gdn_chunk(args["state"], q, args["k"], args["v"], args["g"], args["beta"],
+                         args["out"])
