@@ -408,9 +408,9 @@ typedef struct {
  *   workspace  scratch of workspace_bytes >= sa_gdn_workspace_size(cfg),
  *          16-byte aligned; contents need not be kept between calls. The call
  *          runs two kernels: one computes, for every 64-token block, the
- *          triangular inverse and the masked q.k matrix of the chunkwise form
- *          into the workspace; the other walks the blocks in order and
- *          updates the state.
+ *          triangular inverse of the chunkwise form and its product with the
+ *          decay-masked q.k matrix into the workspace; the other walks the
+ *          blocks in order and updates the state.
  * active: host array of B flags, NULL = all; an inactive stream's state and
  * out rows are untouched. Arithmetic is fp32 with fp32 state; outputs are
  * rounded once to cfg->dtype. Asynchronous on `stream`, graph-capturable.

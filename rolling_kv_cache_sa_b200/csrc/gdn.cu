@@ -29,7 +29,9 @@
 // Two kernels per call:
 //  * gdn_prep_kernel: one CTA per (stream, head, sub-chunk), all independent.
 //    It computes what depends only on K, Q, g and beta -- T = (I + L)^-1 and
-//    scale * P -- and writes both (64 x 64 fp32 each) to the workspace.
+//    M = scale P T -- and writes both (64 x 64 fp32 each) to the workspace.
+//    With U = T RHS, the intra-chunk part of the outputs is P U = M RHS, so the
+//    sequential pass gets U and the outputs from one sweep over RHS.
 //  * gdn_chunk_kernel: one CTA per (stream, head, 32 value rows of the state).
 //    Rows of S evolve independently, so a CTA owns its 32 x D slice of the
 //    state for the whole call (in registers, with a copy in shared memory for
@@ -81,10 +83,9 @@ struct GdnSmem {
   static constexpr int qh = kh + kCt * KP;        // [64][KP] normalised queries
   static constexpr int st = qh + kCt * KP;        // [32][D] state slice S0 (swizzled)
   static constexpr int tm = st + kDvs * D;        // [64][68] (I + L)^-1 (lower)
-  static constexpr int pm = tm + kCt * kLp;       // [64][68] scale P (lower)
-  static constexpr int rv = pm + kCt * kLp;       // [64][36] v slice, right-hand side, then
-                                                  //          u_t e^(G_last - G_t)
-  static constexpr int uv = rv + kCt * kVp;       // [64][36] corrected values u
+  static constexpr int pm = tm + kCt * kLp;       // [64][68] M = scale P T (lower)
+  static constexpr int rv = pm + kCt * kLp;       // [64][36] v slice, then the right-hand side
+  static constexpr int uv = rv + kCt * kVp;       // [64][36] u_t e^(G_last - G_t)
   static constexpr int gs = uv + kCt * kVp;       // [64] in-warp prefix sums of g log2(e)
   static constexpr int bs = gs + kCt;             // [64] beta
   static constexpr int ws = bs + kCt;             // [64] e^(G_last - G_t)
@@ -193,8 +194,8 @@ __device__ __forceinline__ void gate_scan(float g, float beta, float* Gs, float*
   Gs[tid] = gl;
 }
 
-// One CTA per (stream, head, sub-chunk): T = (I + L)^-1 and scale * P of the
-// sub-chunk into the workspace, both [64][64] row-major, zero above the
+// One CTA per (stream, head, sub-chunk): T = (I + L)^-1 and M = scale P T of
+// the sub-chunk into the workspace, both [64][64] row-major, zero above the
 // diagonal.
 template <int D, typename T>
 __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_constant__ GdnParams p) {
@@ -368,12 +369,51 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_c
     }
     __syncthreads();
 
+  // ---- M = P T (lower triangular; L is no longer needed, M takes its place).
+  // The outputs' intra-chunk part is P U = P T RHS = M RHS. Thread (ty, tx)
+  // takes rows ty + 16a and columns tx + 16b, b <= a.
+  {
+    float* Mm = Lm;
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[10];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int r = 0; r < kCt; ++r) {
+      float pv[4], tv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const int t = ty + 16 * a, s2 = tx + 16 * a;
+        pv[a] = r <= t ? Pm[t * kLp + r] : 0.f;
+        tv[a] = r >= s2 ? Tm[r * kLp + s2] : 0.f;
+      }
+      int i = 0;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb <= a; ++bb, ++i) acc[i] = fmaf(pv[a], tv[bb], acc[i]);
+    }
+    int i = 0;   // (the last reads of L were in the merges, before the barrier above)
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const int t = ty + 16 * a, s2 = tx + 16 * bb;
+        float mv = 0.f;
+        if (bb <= a) {
+          if (s2 <= t) mv = acc[i];
+          ++i;
+        }
+        Mm[t * kLp + s2] = mv;
+      }
+  }
+  __syncthreads();
 
-  // ---- T and P to the workspace, zero above the diagonal
+  // ---- T and M to the workspace, zero above the diagonal
   float* dst = p.workspace + (((size_t)z * H + h) * (size_t)p.n_sub + (size_t)j) * kTpFloats;
   for (int e = tid; e < 2 * kCt * (kCt / 4); e += kGdnThreads) {
     const int mat = e / (kCt * (kCt / 4)), row = (e / (kCt / 4)) % kCt, c4 = (e % (kCt / 4)) * 4;
-    float4 x = ld4((mat ? Pm : Tm) + row * kLp + c4);
+    float4 x = ld4((mat ? Lm : Tm) + row * kLp + c4);
     if (c4 + 0 > row) x.x = 0.f;
     if (c4 + 1 > row) x.y = 0.f;
     if (c4 + 2 > row) x.z = 0.f;
@@ -392,7 +432,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
   float* Kh = sm + L::kh;
   float* Qh = sm + L::qh;
   float* St = sm + L::st;
-  float* Pm = sm + L::pm;
+  float* Mm = sm + L::pm;   // M = P T
   float* Tm = sm + L::tm;
   float* Rv = sm + L::rv;
   float* Uv = sm + L::uv;
@@ -450,14 +490,14 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
     }
   };
 
-  // Issues the copies of T and scale * P of sub-chunk j from the workspace
-  // (written by gdn_prep_kernel) into Tm and Pm.
+  // Issues the copies of T and M = scale P T of sub-chunk j from the
+  // workspace (written by gdn_prep_kernel) into Tm and Mm.
   const float* wsp = p.workspace + ((size_t)blockIdx.z * H + h) * (size_t)p.n_sub * kTpFloats;
   auto prefetch_tp = [&](int64_t j) {
     const float* src = wsp + (size_t)j * kTpFloats;
     for (int c = tid; c < 2 * kCt * (kCt / 4); c += kGdnThreads) {
       const int mat = c / (kCt * (kCt / 4)), row = (c / (kCt / 4)) % kCt, c4 = (c % (kCt / 4)) * 4;
-      cp_async16((mat ? Pm : Tm) + row * kLp + c4, src + mat * kCt * kCt + row * kCt + c4);
+      cp_async16((mat ? Mm : Tm) + row * kLp + c4, src + mat * kCt * kCt + row * kCt + c4);
     }
     cp_async_commit();
   };
@@ -554,14 +594,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
     if (tid < kCt) Ws[tid] = ex2f(gcum(kCt - 1) - gcum(tid));   // end-state weights
     __syncthreads();
 
-    // ---- corrected values U = (I + L)^-1 RHS. Rows of RHS past n are zero,
-    // so the sums run over all 64 tokens.
-    float uacc[2][4];
+    // ---- one pass over the right-hand side: U = T RHS (the corrected values)
+    // and the outputs' intra-chunk part P U = M RHS. Rows of RHS past n are
+    // zero, so the sums run over all 64 tokens. u_t e^(G_last - G_t) goes to
+    // Uv for the state update.
     {
+      float uacc[2][4], acc[2][4];
 #pragma unroll
       for (int a = 0; a < 2; ++a)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) uacc[a][i] = 0.f;
+        for (int i = 0; i < 4; ++i) uacc[a][i] = 0.f, acc[a][i] = oin[a][i];
 #pragma unroll 8
       for (int s2 = 0; s2 < kCt; ++s2) {
         const float4 r4 = ld4(Rv + s2 * kVp + cq);
@@ -569,50 +611,23 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
         for (int a = 0; a < 2; ++a) {
           const int t = tq + 32 * a;
           const float tv = s2 <= t ? Tm[t * kLp + s2] : 0.f;
+          const float mv = s2 <= t ? Mm[t * kLp + s2] : 0.f;
           uacc[a][0] = fmaf(tv, r4.x, uacc[a][0]);
           uacc[a][1] = fmaf(tv, r4.y, uacc[a][1]);
           uacc[a][2] = fmaf(tv, r4.z, uacc[a][2]);
           uacc[a][3] = fmaf(tv, r4.w, uacc[a][3]);
+          acc[a][0] = fmaf(mv, r4.x, acc[a][0]);
+          acc[a][1] = fmaf(mv, r4.y, acc[a][1]);
+          acc[a][2] = fmaf(mv, r4.z, acc[a][2]);
+          acc[a][3] = fmaf(mv, r4.w, acc[a][3]);
         }
       }
-#pragma unroll
-      for (int a = 0; a < 2; ++a)
-        st4(Uv + (tq + 32 * a) * kVp + cq,
-            make_float4(uacc[a][0], uacc[a][1], uacc[a][2], uacc[a][3]));
-    }
-    __syncthreads();
-
-    // ---- u_t e^(G_last - G_t) replaces the right-hand side (all of it has
-    // been read); outputs: inter-chunk part + intra-chunk part P U
-    {
 #pragma unroll
       for (int a = 0; a < 2; ++a) {
         const int t = tq + 32 * a;
         const float w = Ws[t];
-        st4(Rv + t * kVp + cq, make_float4(uacc[a][0] * w, uacc[a][1] * w, uacc[a][2] * w,
+        st4(Uv + t * kVp + cq, make_float4(uacc[a][0] * w, uacc[a][1] * w, uacc[a][2] * w,
                                            uacc[a][3] * w));
-      }
-      float acc[2][4];
-#pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[a][i] = oin[a][i];
-#pragma unroll 8
-      for (int s2 = 0; s2 < kCt; ++s2) {
-        const float4 u4 = ld4(Uv + s2 * kVp + cq);
-#pragma unroll
-        for (int a = 0; a < 2; ++a) {
-          const int t = tq + 32 * a;
-          const float pv = s2 <= t ? Pm[t * kLp + s2] : 0.f;
-          acc[a][0] = fmaf(pv, u4.x, acc[a][0]);
-          acc[a][1] = fmaf(pv, u4.y, acc[a][1]);
-          acc[a][2] = fmaf(pv, u4.z, acc[a][2]);
-          acc[a][3] = fmaf(pv, u4.w, acc[a][3]);
-        }
-      }
-#pragma unroll
-      for (int a = 0; a < 2; ++a) {
-        const int t = tq + 32 * a;
         if (t < n) {
           const size_t o = bh0 + (size_t)(t0 + t) * tok_stride + vcol + cq;
 #pragma unroll
@@ -621,7 +636,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
       }
     }
     __syncthreads();
-    // T and P of this sub-chunk have been read: fetch the next sub-chunk's
+    // T and M of this sub-chunk have been read: fetch the next sub-chunk's
     if (t0 + kCt < Tn) prefetch_tp(t0 / kCt + 1);
     // ---- state: S = e^(G_last) S0 + sum_t (u_t e^(G_last - G_t)) k_t^T
     // (u and k are zero past n)
@@ -633,7 +648,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
         for (int c = 0; c < NC; ++c) sreg[i][c] *= dec;
 #pragma unroll 8
       for (int t = 0; t < kCt; ++t) {
-        const float4 uw = ld4(Rv + t * kVp + ur);
+        const float4 uw = ld4(Uv + t * kVp + ur);
         float kv[NC];
         if constexpr (NC == 4) {
           const float4 k4 = ld4(Kh + t * KP + ucol);
