@@ -1,4 +1,5 @@
-"""ctypes wrapper of the fp64 C oracle (oracle.c).
+"""ctypes wrapper of the fp64 C oracle (oracle.c): the rolling-cache attention
+path and the GDN block's gated delta rule.
 
 TEST INFRASTRUCTURE ONLY: imported by the tests, the smoke check and the
 benchmark's CPU-baseline leg; never by the product path. It shares no code

@@ -1,6 +1,7 @@
 /*
  * oracle.h -- plain, slow, fp64 CPU oracle of per-chunk block-causal attention
- * over a rolling (sink + sliding window) KV cache with 3D RoPE and refresh.
+ * over a rolling (sink + sliding window) KV cache with 3D RoPE and refresh,
+ * and of the gated delta rule of the hybrid model's GDN blocks (orc_gdn_chunk).
  *
  * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the
  * benchmark's CPU-baseline leg may load this library. It shares no code with
@@ -15,6 +16,8 @@
  *    attend to a sliding local window plus a persistent sink chunk, i.e. a
  *    bounded context with constant memory.
  *  - StreamDiT (abstract): window attention over a moving buffer of frames.
+ *  - SANA-Streaming (sections "hybrid diffusion transformer", "system
+ *    co-design"): the GDN blocks' recurrent state (see orc_gdn_chunk).
  * The pages print no formula; the numeric definition below (ring geometry,
  * 3D RoPE bands, rebase offset, dtype rounding) is the reading stated beside
  * each function.
