@@ -2,15 +2,16 @@
 
 The oracle (orc_gdn_chunk) runs the gated delta rule token by token; the
 kernel runs its chunkwise form in fp32. Tolerances:
-  * fp32 inputs and outputs: max abs 2e-4 on outputs and on the state. The
-    kernel's fp32 error per sub-chunk is a few ulps of values |S|, |o| <~ 4
-    through dot products of <= 128 terms and a 64 x 64 triangular inverse;
-    over the tens of sub-chunks a call spans, with the decay damping older
-    errors, that stays well under 2e-4.
+  * fp32 inputs and outputs: max abs 1e-4 on outputs and on the state, the
+    bar the fp32 attention path is held to. The kernel's fp32 error per
+    sub-chunk is a few ulps (2^-24 relative) of values |S|, |o| <~ 4 through
+    dot products of <= 128 terms and a 64 x 64 triangular inverse, about
+    1e-6; the decay damps older errors, so it does not grow over a stream
+    (a 32-call stream is checked without re-synchronising with the oracle).
   * bf16 inputs and outputs: the same fp32 arithmetic on the same (bf16)
     input values, then one rounding of o to bf16 (relative 2^-9): the
     attention bar, max abs 2e-2 and mean abs 2e-3 on outputs; the fp32 state
-    within 2e-4.
+    within 1e-4.
 """
 from __future__ import annotations
 
@@ -24,9 +25,9 @@ from inputgen.workloads import P512, Workload
 
 pytestmark = pytest.mark.gpu
 
-F32_MAX = 2e-4
+F32_MAX = 1e-4
 BF16_MAX, BF16_MEAN = 2e-2, 2e-3
-STATE_MAX = 2e-4
+STATE_MAX = 1e-4
 
 
 def _gdn():
