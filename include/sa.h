@@ -277,6 +277,13 @@ sa_status sa_profile_end(sa_cache* h, double* append_ms, int32_t* n_append, doub
  *                    chunk. k_raw may be NULL when S = 0.
  *   frames_written : host array [B], read and advanced by C per active stream.
  *   pos_base       : host array [B], the streams' RoPE position bases (read).
+ *                    There is no allocation-free RoPE refresh: the keys
+ *                    already stored keep the positions they were written
+ *                    with, so a stream's pos_base must stay the value it had
+ *                    at its first chunk (0 for a new stream). Changing it
+ *                    between calls shifts new keys against stored ones and
+ *                    silently changes every score; streams that need periodic
+ *                    refreshes must use a cache handle (sa_rope_refresh).
  *   q, k, v, out, active, stream : as for sa_append_attend.
  * Scratch: a file-scope static device array of 16 MiB (rotated queries
  * B*H*C*F*D elements, the spatial RoPE tables and a status word), present on
@@ -287,13 +294,23 @@ sa_status sa_profile_end(sa_cache* h, double* append_ms, int32_t* n_append, doub
  * scratch array, which keeps the last call's contents: calls whose work
  * overlaps on the GPU (other streams, other host threads) race and must be
  * serialised by the caller. Enqueues work on `stream` and never synchronises;
- * calls no allocator. A bounded-wait expiry is recorded in the scratch status
- * word only (not reported).
+ * calls no allocator. A bounded-wait expiry is not returned by the call (it
+ * happens later, on the GPU): it sets a sticky status word in the scratch,
+ * which sa_noalloc_device_status reports and clears.
  */
 sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cache, void* v_cache,
                                    void* k_raw, int64_t* frames_written, const int64_t* pos_base,
                                    const void* q, const void* k, const void* v, void* out,
                                    const uint8_t* active, sa_stream_t stream);
+
+/* Device status of the allocation-free entry on the current device (no
+ * counterpart on the pages; the analogue of sa_get_device_status for callers
+ * without a handle). Synchronises `stream`, reads the status word in the
+ * static scratch and clears it. Returns SA_ERR_DEVICE_TIMEOUT if a bounded
+ * wait of any sa_append_attend_noalloc call on this device gave up since the
+ * last read (the outputs and cache rows of those calls are not valid),
+ * SA_OK otherwise, SA_ERR_CUDA on a CUDA error. Allocates nothing. */
+sa_status sa_noalloc_device_status(sa_stream_t stream);
 
 /* Number of kernels the handle launched since sa_profile_begin (host count). */
 sa_status sa_profile_launches(const sa_cache* h, int64_t* launches);

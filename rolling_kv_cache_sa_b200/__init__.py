@@ -12,6 +12,6 @@ from .cache import (  # noqa: F401
     sa_get_device_status, sa_plan_chunk, sa_profile_begin, sa_profile_end, sa_profile_launches, sa_refresh_delta,
     sa_rope_refresh, sa_stream_state, sa_wait_probe, sa_attend, sa_cache_set_sink_mode,
     sa_sink_update, sa_append_attend_host_async, sa_host_wait, sa_cache_set_fp8_scales,
-    sa_cache_export, sa_cache_import, sa_cache_get_fp8_scales,
+    sa_cache_export, sa_cache_import, sa_cache_get_fp8_scales, sa_noalloc_device_status,
 )
 from .gdn import GDNState, gdn_workspace, sa_gdn_chunk, sa_gdn_workspace_size  # noqa: F401

@@ -24,7 +24,7 @@ EXPORTED = (
     "sa_profile_launches", "sa_wait_probe", "sa_attend", "sa_cache_set_sink_mode",
     "sa_sink_update", "sa_append_attend_host_async", "sa_host_wait", "sa_cache_set_fp8_scales",
     "sa_cache_export_size", "sa_cache_export", "sa_cache_import", "sa_cache_get_fp8_scales",
-    "sa_gdn_chunk", "sa_gdn_workspace_size",
+    "sa_gdn_chunk", "sa_gdn_workspace_size", "sa_noalloc_device_status",
 )
 
 
@@ -107,6 +107,7 @@ def lib() -> ctypes.CDLL:
         "sa_gdn_chunk": [P(sa_gdn_config), vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp,
                          vp],
         "sa_gdn_workspace_size": [P(sa_gdn_config), P(ctypes.c_size_t)],
+        "sa_noalloc_device_status": [vp],
         "sa_profile_end": [vp, P(ctypes.c_double), P(i32), P(ctypes.c_double), P(i32),
                            P(ctypes.c_double), P(i32)],
     }

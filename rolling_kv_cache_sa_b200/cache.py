@@ -195,18 +195,59 @@ def sa_profile_launches(h: int) -> int:
     return n.value
 
 
+def _need(t, name: str, shape, dtype, device):
+    if not isinstance(t, torch.Tensor) or t.device != device or t.dtype != dtype or \
+            not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        got = (f"{tuple(t.shape)} {t.dtype} on {t.device}"
+               f"{'' if t.is_contiguous() else ', not contiguous'}"
+               if isinstance(t, torch.Tensor) else type(t).__name__)
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on "
+                         f"{device}; got {got}")
+
+
 def sa_append_attend_noalloc(cfg: sa_config, k_cache: torch.Tensor, v_cache: torch.Tensor,
                              k_raw: Optional[torch.Tensor], frames_written, pos_base,
                              q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                              active=None, stream: Optional[torch.cuda.Stream] = None):
     """Allocation-free append + attention over caller-owned cache buffers.
     frames_written / pos_base: ctypes int64 arrays of length B (host);
-    frames_written is advanced in place."""
+    frames_written is advanced in place; pos_base must stay at each stream's
+    first value (there is no allocation-free refresh).
+
+    The library cannot check the sizes of the buffers it is given, so they
+    are checked here before the call: k_cache and v_cache [B, H, (S+W+C)*F, D],
+    k_raw [B, H, S*F, D] (when S > 0), q, k, v and out [B, C*F, H, D], all
+    contiguous, of the configuration's dtype and on the current device."""
+    if cfg.dtype == SA_BF16_E4M3:
+        raise ValueError("the allocation-free entry runs SA_F32 and SA_BF16 caches")
+    B, H, D = cfg.batch, cfg.heads, cfg.head_dim
+    F = cfg.frame_h * cfg.frame_w
+    Lc = cfg.chunk_frames * F
+    ntok = (cfg.sink_frames + cfg.window_frames + cfg.chunk_frames) * F
+    dt = torch.float32 if cfg.dtype == SA_F32 else torch.bfloat16
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _need(k_cache, "k_cache", (B, H, ntok, D), dt, dev)
+    _need(v_cache, "v_cache", (B, H, ntok, D), dt, dev)
+    if cfg.sink_frames > 0:
+        _need(k_raw, "k_raw", (B, H, cfg.sink_frames * F, D), dt, dev)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, n, (B, Lc, H, D), dt, dev)
+    if len(frames_written) != B or len(pos_base) != B:
+        raise ValueError(f"frames_written and pos_base must hold {B} entries")
+    if active is not None and len(active) != B:
+        raise ValueError(f"active must hold {B} entries")
     check(lib().sa_append_attend_noalloc(
         ctypes.byref(cfg), k_cache.data_ptr(), v_cache.data_ptr(),
-        k_raw.data_ptr() if k_raw is not None else None, frames_written, pos_base,
-        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _mask(active, cfg.batch),
-        _stream_ptr(stream)), "sa_append_attend_noalloc")
+        k_raw.data_ptr() if (k_raw is not None and cfg.sink_frames > 0) else None,
+        frames_written, pos_base, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+        _mask(active, cfg.batch), _stream_ptr(stream)), "sa_append_attend_noalloc")
+
+
+def sa_noalloc_device_status(stream: Optional[torch.cuda.Stream] = None):
+    """Raises SAError(SA_ERR_DEVICE_TIMEOUT) if a bounded wait of an
+    allocation-free call on the current device gave up since the last read;
+    synchronises the stream and clears the word."""
+    check(lib().sa_noalloc_device_status(_stream_ptr(stream)), "sa_noalloc_device_status")
 
 
 def sa_wait_probe(limit_ns: int, stream: Optional[torch.cuda.Stream] = None):

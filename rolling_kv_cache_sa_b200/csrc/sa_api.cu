@@ -1160,8 +1160,9 @@ sa_status sa_profile_end(sa_cache* h, double* append_ms, int32_t* n_append, doub
 // until the process exits. The first call on a device looks its address up
 // (cudaGetSymbolAddress with that device current), so that first call should
 // come before any stream capture. All calls share the array and it keeps the
-// last call's contents: the status word is cleared by each call, and calls
-// whose work overlaps on the GPU race.
+// last call's contents: the status word is sticky (a call whose bounded wait
+// gave up sets it; only sa_noalloc_device_status reads and clears it), and
+// calls whose work overlaps on the GPU race.
 // ---------------------------------------------------------------------------
 #include <mutex>
 
@@ -1278,9 +1279,8 @@ extern "C" sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cach
       return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // every call shares the scratch: the status word must start at zero
-  e = cudaMemsetAsync(d_status, 0, sizeof(int), s);
-  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  // the status word starts at zero (static storage) and is cleared only by
+  // sa_noalloc_device_status, so an expired wait stays visible until read
   if (c.frame_h * dh2 + c.frame_w * dw2 > 0) {
     noalloc_tables_kernel<<<std::max(1, nsm), 256, 0, s>>>(
         htab, wtab, c.frame_h, c.frame_w, dh2, dw2, c.rope_dims[1], c.rope_dims[2],
@@ -1339,5 +1339,26 @@ extern "C" sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cach
                          : sa::launch_attend_simt_f32(ap, c.head_dim, s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   for (int b : act) frames_written[b] += C;
+  return SA_OK;
+}
+
+extern "C" sa_status sa_noalloc_device_status(sa_stream_t stream) {
+  void* scratch = nullptr;
+  sa_status st = noalloc_scratch(&scratch);
+  if (st != SA_OK) return st;
+  int* d_status = static_cast<int*>(scratch);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, d_status, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word != 0) {
+    e = cudaMemsetAsync(d_status, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+    return fail(SA_ERR_DEVICE_TIMEOUT,
+                "a bounded device wait of an allocation-free call gave up (status %d); the "
+                "outputs and caches those calls wrote are not valid", word);
+  }
   return SA_OK;
 }
