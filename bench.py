@@ -71,6 +71,10 @@ def parse():
                     help="gdn: the Gated DeltaNet block (sa_gdn_chunk) on the same streams")
     ap.add_argument("--gdn-g-scale", type=float, default=0.002,
                     help="gdn: per-token log decay drawn in (-g_scale, 0)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other configurations' per_config entries")
+    ap.add_argument("--per-config-steps", type=int, default=3,
+                    help="timed steps per other configuration")
     return ap.parse_args()
 
 
@@ -438,16 +442,303 @@ def run_gdn(args, w, rank, world):
 
 
 # ------------------------------------------------------------------ GPU arm
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16 (spec sheet; fp8 twice that)
+NOMINAL_HBM_GBS = 8000.0      # B200 HBM3e (spec sheet, ~8 TB/s)
+
+# The other configurations reported in per_config (the headline line is the
+# 512p one). The long-stress case streams 10,000 chunks per stream (1.5e16
+# FLOP): it is timed on a window of 64 global steps once every stream is
+# active and its ring is full, a window that holds each stream's refresh at
+# local chunk 256 (stream b refreshes at global step 256 + start_b <= 298).
+STRESS_WINDOW = (240, 304)
+
+
+def _config_alias():
+    from inputgen.workloads import ALL
+    return {f"C{i + 1}": wl.name for i, wl in enumerate(ALL)}
+
+
+def measure_attention(w, args, rank, world, local, *, steps, warmup, window=None,
+                      use_graph=True, eager_steps=None, latency=False, e2e=False):
+    """Times the attention hot path on workload w (one step = global steps
+    [g0, g1) of w's schedule, from an empty cache unless a window is given:
+    then steps [0, g0) run untimed first to reach the window's cache state).
+    Returns the raw figures; `use_graph` replays one captured step."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import inputgen as IG
+    from rolling_kv_cache_sa_b200 import SACache, attention_flops, config_for, sa_plan_chunk
+    from rolling_kv_cache_sa_b200.dist import aggregate_rate, max_over_ranks, rank_stream_ids
+    from rolling_kv_cache_sa_b200.session import StreamSession
+
+    cfg = config_for(w)
+    cache = SACache(cfg)
+    sess = StreamSession(cache, w.refresh_period)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    g0, g1 = window if window else (0, w.n_steps)
+    nT = g1 - g0
+    shape = (nT, w.B, w.Lc, w.H, w.D)
+    q_all = torch.empty(shape, dtype=dt, device="cuda")
+    k_all, v_all, out_all = torch.empty_like(q_all), torch.empty_like(q_all), torch.empty_like(q_all)
+    st = torch.cuda.current_stream().cuda_stream
+    stream_ids = rank_stream_ids(rank, w.B)  # distinct streams per rank
+    actives, step_flops, chunks_per_step = [], 0.0, 0
+    for i, g in enumerate(range(g0, g1)):
+        chunks = w.local_chunks(g)
+        actives.append([c >= 0 for c in chunks])
+        for t, buf in ((IG.Q, q_all), (IG.K, k_all), (IG.V, v_all)):
+            IG.fill_device(w, stream_ids, chunks, t, buf[i].data_ptr(), st)
+        for c in chunks:
+            if c >= 0:
+                chunks_per_step += 1
+                # algorithmic FLOPs: 4 * Lc * n_keys * D * H per stream-chunk
+                step_flops += attention_flops(cfg, sa_plan_chunk(cfg, c * w.C, 0).n_keys)
+    torch.cuda.synchronize()
+    esz = 2 if w.dtype == "bf16" else 4
+    cesz = 1 if w.cache == "e4m3" else esz  # cache element bytes
+    append_bytes_per_chunk = 3 * w.Lc * w.H * w.D * (esz + cesz)  # read q,k,v; write q',k',v
+
+    def run_prefix():
+        # untimed: bring the cache to the window's state (the data of these
+        # steps does not enter the timed window's work, only its positions)
+        cache.reset()
+        for g in range(g0):
+            chunks = w.local_chunks(g)
+            act = [c >= 0 for c in chunks]
+            if any(act):
+                sess.step(q_all[g % nT], k_all[g % nT], v_all[g % nT], out_all[g % nT], act)
+
+    def run_step():
+        if not window:
+            cache.reset()
+        for i in range(nT):
+            sess.step(q_all[i], k_all[i], v_all[i], out_all[i], actives[i])
+
+    def timed(fn, n, prefix=None):
+        total = 0.0
+        for _ in range(n if prefix else 1):
+            if prefix:
+                prefix()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(1 if prefix else n):
+                fn()
+            e1.record()
+            e1.synchronize()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        return max_over_ranks(total, "cuda")
+
+    for _ in range(warmup):
+        if window:
+            run_prefix()
+        run_step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    # eager: every library call issued from Python; the library's per-launch
+    # CUDA events (on the launch stream) time each kernel
+    n_eager = eager_steps if eager_steps else (steps if not use_graph else max(1, min(steps, 20)))
+    if window:
+        # the prefix runs outside the profiled and timed region
+        tot, launches_total = 0.0, 0
+        prof = {"append": [0.0, 0], "attend": [0.0, 0], "refresh": [0.0, 0]}
+        for _ in range(n_eager):
+            run_prefix()
+            torch.cuda.synchronize()
+            cache.profile_begin()
+            tot += timed(run_step, 1)
+            launches_total += cache.profile_launches()
+            pe = cache.profile_end()
+            for k_ in prof:
+                prof[k_][0] += pe[k_][0]
+                prof[k_][1] += pe[k_][1]
+        ms_eager = tot
+        prof = {k_: tuple(v_) for k_, v_ in prof.items()}
+        launches_per_step = launches_total / n_eager
+    else:
+        cache.profile_begin()
+        ms_eager = timed(run_step, n_eager)
+        launches_per_step = cache.profile_launches() / n_eager
+        prof = cache.profile_end()
+
+    graph = None
+    if not use_graph:
+        ms, n_timed = ms_eager, n_eager
+    else:
+        # one whole step captured once (every hot call of the library is
+        # capturable: no synchronisation, parameters by value) and replayed
+        # with profiling off, so the graph holds kernel nodes only
+        if window:
+            run_prefix()
+            torch.cuda.synchronize()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            run_step()
+        torch.cuda.synchronize()
+        for _ in range(warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        ms, n_timed = timed(graph.replay, steps), steps
+    clocks = sampler.stop() if sampler else None
+
+    res = {"w": w, "cache": cache, "sess": sess, "graph": graph, "q_all": q_all, "k_all": k_all,
+           "v_all": v_all, "out_all": out_all, "actives": actives, "dt": dt, "esz": esz,
+           "nT": nT, "window": window, "run_prefix": run_prefix, "run_step": run_step}
+    res["chunks_per_step"] = chunks_per_step
+    res["step_flops"] = step_flops
+    res["ms_step"] = ms / n_timed
+    res["value"] = aggregate_rate(chunks_per_step * n_timed, world, ms)
+    res["ms_eager"] = ms_eager / n_eager
+    res["eager_value"] = chunks_per_step * world / (res["ms_eager"] / 1000.0)
+    res["launches"] = int(round(launches_per_step * n_timed))
+    res["timed_steps"] = n_timed
+    res["clocks"] = clocks
+    att_ms, att_n = prof["attend"]
+    app_ms, app_n = prof["append"]
+    ref_ms, _ = prof["refresh"]
+    res["kernel_ms_per_step"] = {"attend": att_ms / n_eager, "append": app_ms / n_eager,
+                                 "refresh": ref_ms / n_eager}
+    res["att_launches_per_step"] = att_n / n_eager
+    res["att_avg_s"] = att_ms / 1000.0 / max(att_n, 1)
+    res["att_flops_per_launch"] = step_flops * n_eager / max(att_n, 1)
+    res["achieved"] = res["att_flops_per_launch"] / res["att_avg_s"] / 1e12 if att_n else None
+    res["append_bytes_per_launch"] = append_bytes_per_chunk * chunks_per_step * n_eager / max(app_n, 1)
+    res["append_gbs"] = (append_bytes_per_chunk * chunks_per_step * n_eager / (app_ms / 1000.0) / 1e9
+                         if app_n and app_ms > 0 else None)
+
+    if latency:
+        # per-call latency: two eager steps, CUDA events around each call
+        # (device time of the call's kernels on the launch stream, refresh
+        # included when due)
+        lat = []
+        for _ in range(2):
+            if window:
+                run_prefix()
+            else:
+                cache.reset()
+            evs = []
+            for i in range(nT):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                sess.step(q_all[i], k_all[i], v_all[i], out_all[i], actives[i])
+                e1.record()
+                evs.append((e0, e1))
+            torch.cuda.synchronize()
+            lat += [a.elapsed_time(b) for a, b in evs]
+        res["call_latency"] = {
+            "p50_ms": float(np.percentile(lat, 50)), "p99_ms": float(np.percentile(lat, 99)),
+            "calls": len(lat),
+            "what": "device time per step call (append + attention, refresh when due), eager, "
+                    "CUDA events on the launch stream"}
+
+    if e2e and not window:
+        qh = torch.empty(q_all.shape, dtype=dt, pin_memory=True)
+        kh = torch.empty_like(qh, pin_memory=True)
+        vh = torch.empty_like(qh, pin_memory=True)
+        oh = torch.empty_like(qh, pin_memory=True)
+        qh.copy_(q_all)
+        kh.copy_(k_all)
+        vh.copy_(v_all)
+
+        def run_step_host():
+            # every call is queued: copies of one chunk overlap the compute of
+            # another in the library's pipeline; waited for at the end
+            cache.reset()
+            for i in range(nT):
+                sess.step_host_async(qh[i], kh[i], vh[i], oh[i], actives[i])
+
+        run_step_host()
+        cache.host_wait()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.e2e_steps):
+            run_step_host()
+        cache.host_wait()  # the last copy-out has landed before the closing event
+        e1.record()
+        e1.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1), "cuda")
+        per_chunk_in = 3 * w.Lc * w.H * w.D * esz
+        res["e2e"] = {"value": aggregate_rate(chunks_per_step * args.e2e_steps, world, ems),
+                      "unit": "chunks/s", "steps": args.e2e_steps,
+                      "h2d_bytes_per_step": per_chunk_in * chunks_per_step,
+                      "d2h_bytes_per_step": w.Lc * w.H * w.D * esz * chunks_per_step,
+                      "api": "sa_append_attend_host_async (pinned host buffers; the copy-in, "
+                             "compute and copy-out of consecutive chunks overlap; every copy is "
+                             "inside the timed region)"}
+    return res
+
+
+def release(res):
+    import torch
+    res["graph"] = None
+    res["cache"].close()
+    for k in ("q_all", "k_all", "v_all", "out_all"):
+        res[k] = None
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def fractions(res, f8=False, tc=True):
+    """Attention and append figures of a measurement against the measured
+    and nominal peaks. The attention kernel is timed per launch (CUDA events
+    around each launch over a short eager pass), i.e. in bursts: the burst
+    peak is the denominator of `frac`; the sustained figure is kept beside it."""
+    hbm, pk_burst, pk_sust, pk_src = peaks()
+    mul = 2.0 if f8 else 1.0  # fp8 contraction: the bf16 peaks x the nominal 2x
+    a = res["achieved"]
+    out = {"attention_tflops": a,
+           "attention_frac_of_burst": a / (mul * pk_burst) if (a and tc) else None,
+           "attention_frac_of_sustained": a / (mul * pk_sust) if (a and tc) else None,
+           "attention_frac_of_nominal": a / (mul * NOMINAL_BF16_TFLOPS) if (a and tc) else None,
+           "append_gbs": res["append_gbs"],
+           "append_frac_of_hbm": res["append_gbs"] / hbm if res["append_gbs"] else None,
+           "append_frac_of_nominal": (res["append_gbs"] / NOMINAL_HBM_GBS
+                                      if res["append_gbs"] else None),
+           "peak_source": pk_src}
+    return out
+
+
+def per_config_entry(res, note):
+    w = res["w"]
+    f8 = w.cache == "e4m3"
+    fr = fractions(res, f8=f8, tc=w.dtype == "bf16")
+    return {"workload": w.name, "value": res["value"], "unit": "chunks/s",
+            "ms_per_step": res["ms_step"], "chunks_per_step": res["chunks_per_step"],
+            "timed_steps": res["timed_steps"],
+            "launch_mode": "cuda graph of one step, replayed" if res["graph"] is not None
+            else "eager",
+            "step": note, "config": config_json(w, 1),
+            "attention_tflops": fr["attention_tflops"],
+            "attention_frac_of_burst": fr["attention_frac_of_burst"],
+            "attention_frac_of_nominal": fr["attention_frac_of_nominal"],
+            "append_gbs": fr["append_gbs"], "append_frac_of_hbm": fr["append_frac_of_hbm"],
+            "kernel_ms_per_step": res["kernel_ms_per_step"],
+            "attention_launches_per_step": res["att_launches_per_step"],
+            "gpu_launches": res["launches"], "clocks": res["clocks"]}
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    from inputgen.workloads import ALL, BY_NAME
-    # C1..C5: the five configurations in order (tiny fp32, 512p, 480x832 ragged,
-    # 1280x704, long-stream stress)
-    aliases = {f"C{i + 1}": wl.name for i, wl in enumerate(ALL)}
+    from inputgen.workloads import BY_NAME
+    aliases = _config_alias()
     w = BY_NAME[aliases.get(args.workload, args.workload)]
     if args.chunks:
         w = w.with_(n_chunks=args.chunks)
@@ -464,179 +755,52 @@ def main():
     import torch
     import torch.distributed as dist
 
-    import inputgen as IG
-    from rolling_kv_cache_sa_b200 import SACache, attention_flops, config_for, sa_plan_chunk
-    from rolling_kv_cache_sa_b200.dist import aggregate_rate, max_over_ranks, rank_stream_ids
-    from rolling_kv_cache_sa_b200.session import StreamSession
-
     torch.cuda.set_device(local)
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
 
-    cfg = config_for(w)
-    cache = SACache(cfg)
-    sess = StreamSession(cache, w.refresh_period)
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    n_steps_g = w.n_steps
-    shape = (n_steps_g, w.B, w.Lc, w.H, w.D)
-    q_all = torch.empty(shape, dtype=dt, device="cuda")
-    k_all = torch.empty_like(q_all)
-    v_all = torch.empty_like(q_all)
-    out_all = torch.empty_like(q_all)
-    st = torch.cuda.current_stream().cuda_stream
-    stream_ids = rank_stream_ids(rank, w.B)  # distinct streams per rank
-    actives = []
-    for g in range(n_steps_g):
-        chunks = w.local_chunks(g)
-        actives.append([c >= 0 for c in chunks])
-        for t, buf in ((IG.Q, q_all), (IG.K, k_all), (IG.V, v_all)):
-            IG.fill_device(w, stream_ids, chunks, t, buf[g].data_ptr(), st)
-    torch.cuda.synchronize()
-
-    chunks_per_step = sum(sum(a) for a in actives)
-    # algorithmic attention FLOPs of one step: 4 * Lc * n_keys * D * H per stream-chunk
-    step_flops = 0.0
-    for c in range(w.n_chunks):
-        step_flops += w.B * attention_flops(cfg, sa_plan_chunk(cfg, c * w.C, 0).n_keys)
-    esz = 2 if w.dtype == "bf16" else 4
-    cesz = 1 if w.cache == "e4m3" else esz  # cache element bytes
-    append_bytes_per_chunk = 3 * w.Lc * w.H * w.D * (esz + cesz)  # read q,k,v; write q',k',v
-
-    def run_step():
-        cache.reset()
-        for g in range(n_steps_g):
-            sess.step(q_all[g], k_all[g], v_all[g], out_all[g], actives[g])
-
-    for _ in range(args.warmup):
-        run_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-
-    def timed(fn, steps):
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(steps):
-            fn()
-        e1.record()
-        e1.synchronize()
-        torch.cuda.synchronize()
-        return max_over_ranks(e0.elapsed_time(e1), "cuda")
-
-    # eager: every library call issued from Python, one launch at a time; the
-    # library's per-launch CUDA events (on the launch stream) time each kernel
-    sampler = ClockSampler(gpu_id_for(local)) if rank == 0 else None
-    if sampler:
-        sampler.start()
-        time.sleep(0.3)
-    eager_steps = args.steps if args.eager else max(1, min(args.steps, 20))
-    cache.profile_begin()
-    ms_eager = timed(run_step, eager_steps)
-    launches_per_step = cache.profile_launches() / eager_steps
-    prof = cache.profile_end()
-    prof_steps = eager_steps
-
-    # graph: one whole step captured once (every hot call of the library is
-    # capturable: no synchronisation, parameters by value) and replayed with
-    # profiling off, so the graph holds kernel nodes only
-    graph = None
-    if args.eager:
-        ms = ms_eager
-    else:
-        cap = torch.cuda.Stream()
-        cap.wait_stream(torch.cuda.current_stream())
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=cap):
-            run_step()
-        torch.cuda.synchronize()
-        for _ in range(args.warmup):
-            graph.replay()
-        torch.cuda.synchronize()
-        ms = timed(graph.replay, args.steps)
-    clocks = sampler.stop() if sampler else None
-    launches = int(round(launches_per_step * args.steps))
-
-    # per-call latency: two eager steps, CUDA events around each call (device
-    # time of the call's kernels on the launch stream, refresh included when due)
-    lat = []
-    for _ in range(2):
-        cache.reset()
-        evs = []
-        for g in range(n_steps_g):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            sess.step(q_all[g], k_all[g], v_all[g], out_all[g], actives[g])
-            e1.record()
-            evs.append((e0, e1))
-        torch.cuda.synchronize()
-        lat += [a.elapsed_time(b) for a, b in evs]
-    import numpy as np
-    call_latency = {"p50_ms": float(np.percentile(lat, 50)), "p99_ms": float(np.percentile(lat, 99)),
-                    "calls": len(lat),
-                    "what": "device time per step call (append + attention, refresh when due), "
-                            "eager, CUDA events on the launch stream"}
-    ms_eager /= eager_steps
-    cache.reset()
-    ms_step = ms / args.steps
-    value = aggregate_rate(chunks_per_step * args.steps, world, ms)
-
-    hbm, pk_burst, pk_sust, pk_src = peaks()
+    res = measure_attention(w, args, rank, world, local, steps=args.steps, warmup=args.warmup,
+                            use_graph=not args.eager, latency=True, e2e=not args.no_e2e)
     f8 = w.cache == "e4m3"
-    if f8:  # fp8 contraction: the measured bf16 peaks x the nominal 2x (4.5 / 2.25 PFLOP/s)
-        pk_burst, pk_sust = 2.0 * pk_burst, 2.0 * pk_sust
-    att_ms, att_n = prof["attend"]
-    app_ms, app_n = prof["append"]
-    ref_ms, ref_n = prof["refresh"]
-    att_flops_per_launch = step_flops * prof_steps / max(att_n, 1)
-    att_avg_s = att_ms / 1000.0 / max(att_n, 1)
-    achieved = att_flops_per_launch / att_avg_s / 1e12
-    # append bytes: every active (stream, chunk) of the profiled steps
-    append_gbs = (append_bytes_per_chunk * chunks_per_step * prof_steps / (app_ms / 1000.0) / 1e9
-                  if app_n and app_ms > 0 else None)
+    fr = fractions(res, f8=f8)
+    e2e = res.get("e2e")
+    ms_step = res["ms_step"]
+    release(res)
 
-    e2e = None
-    if not args.no_e2e:
-        qh = torch.empty(q_all.shape, dtype=dt, pin_memory=True)
-        kh = torch.empty_like(qh, pin_memory=True)
-        vh = torch.empty_like(qh, pin_memory=True)
-        oh = torch.empty_like(qh, pin_memory=True)
-        qh.copy_(q_all)
-        kh.copy_(k_all)
-        vh.copy_(v_all)
-
-        def run_step_host():
-            # every call is queued: copies of one chunk overlap the compute of
-            # another in the library's pipeline; waited for at the end
-            cache.reset()
-            for g in range(n_steps_g):
-                sess.step_host_async(qh[g], kh[g], vh[g], oh[g], actives[g])
-
-        run_step_host()
-        cache.host_wait()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(args.e2e_steps):
-            run_step_host()
-        cache.host_wait()  # the last copy-out has landed before the closing event
-        e1.record()
-        e1.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1), "cuda")
-        per_chunk_in = 3 * w.Lc * w.H * w.D * esz
-        e2e = {"value": aggregate_rate(chunks_per_step * args.e2e_steps, world, ems),
-               "unit": "chunks/s", "steps": args.e2e_steps,
-               "h2d_bytes_per_step": per_chunk_in * chunks_per_step,
-               "d2h_bytes_per_step": w.Lc * w.H * w.D * esz * chunks_per_step,
-               "api": "sa_append_attend_host_async (pinned host buffers; the copy-in, "
-                      "compute and copy-out of consecutive chunks overlap; every copy is "
-                      "inside the timed region)"}
+    # the other configurations of the metric, a few timed steps each
+    per_config = None
+    if not args.no_per_config and not args.chunks:
+        per_config = {}
+        from inputgen.workloads import ALL
+        for i, wc in enumerate(ALL):
+            alias = f"C{i + 1}"
+            if wc.name == w.name:
+                continue
+            if f8:
+                if wc.dtype != "bf16":
+                    continue
+                wc = wc.with_(cache="e4m3")
+            k_steps = max(1, min(args.steps, args.per_config_steps))
+            if wc.name == "long_stress_b8_10000":
+                r = measure_attention(wc, args, rank, world, local, steps=k_steps,
+                                      warmup=1, window=STRESS_WINDOW, use_graph=False,
+                                      eager_steps=k_steps)
+                note = (f"global steps {STRESS_WINDOW[0]}..{STRESS_WINDOW[1] - 1} of the "
+                        f"10,000-chunk schedule (all 8 streams active, rings full, each stream's "
+                        f"refresh at its local chunk 256 inside); steps 0..{STRESS_WINDOW[0] - 1} "
+                        f"run untimed before each timed window; eager issue")
+            else:
+                r = measure_attention(wc, args, rank, world, local, steps=k_steps,
+                                      warmup=min(args.warmup, 2), use_graph=True,
+                                      eager_steps=k_steps)
+                note = (f"the whole schedule ({wc.n_steps} global steps, {wc.n_chunks} chunks per "
+                        f"stream) from an empty cache")
+            per_config[alias] = per_config_entry(r, note)
+            release(r)
+        per_config["C2" if not f8 else "C2_e4m3"] = {"workload": w.name,
+                                                    "see": "the line's own value and roofline"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -646,37 +810,42 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
-        cache.close()
         return
-    att_tflops_step = step_flops / (ms_step / 1000.0) / 1e12
+    hbm, pk_burst, pk_sust, pk_src = peaks()
+    mul = 2.0 if f8 else 1.0
+    att_tflops_step = res["step_flops"] / (ms_step / 1000.0) / 1e12
     line = {
-        "metric": METRIC, "value": value, "unit": "chunks/s", "n_gpus": world,
+        "metric": METRIC, "value": res["value"], "unit": "chunks/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3" if f8 else "bf16",
+        "dtype": "e4m3" if f8 else ("bf16" if w.dtype == "bf16" else "f32"),
         "data": "synthetic (seeded counter generator; Irwin-Hall N(0,1) inputs)",
         "config": config_json(w, world),
-        "ms_per_chunk": ms_step / chunks_per_step,
+        "ms_per_chunk": ms_step / res["chunks_per_step"],
         "attention_tflops_whole_step": att_tflops_step,
-        "attention_frac_of_peak_whole_step": att_tflops_step / pk_sust,
-        "append_gbs": append_gbs,
-        "append_frac_of_hbm": (append_gbs / hbm) if append_gbs else None,
-        "kernel_ms_per_step": {"attend": att_ms / prof_steps, "append": app_ms / prof_steps,
-                               "refresh": ref_ms / prof_steps},
-        "call_latency": call_latency,
-        "launch_mode": "cuda graph of one step, replayed" if graph is not None else "eager",
-        "eager_chunks_per_s": chunks_per_step * world / (ms_eager / 1000.0),
-        "eager_ms_per_step": ms_eager,
-        # the kernel is timed inside long back-to-back stepping (the eager
-        # pass and the replays run continuously under the power cap), so the
-        # denominator is the sustained bf16 figure; the burst one is kept too
+        "attention_frac_of_burst_whole_step": att_tflops_step / (mul * pk_burst),
+        "attention_frac_of_nominal": fr["attention_frac_of_nominal"],
+        "append_gbs": fr["append_gbs"],
+        "append_frac_of_hbm": fr["append_frac_of_hbm"],
+        "append_frac_of_nominal": fr["append_frac_of_nominal"],
+        "kernel_ms_per_step": res["kernel_ms_per_step"],
+        "call_latency": res.get("call_latency"),
+        "launch_mode": "eager" if args.eager else "cuda graph of one step, replayed",
+        "eager_chunks_per_s": res["eager_value"],
+        "eager_ms_per_step": res["ms_eager"],
+        # the kernel is timed per launch (CUDA events around each launch of
+        # a short eager pass), so the burst peak is the denominator; the
+        # sustained (power-capped, seconds-long GEMM loop) figure is kept
         "roofline": {"bound": "tensor",
                      "kernel": "attend_tc_kernel<128, e4m3>" if f8 else "attend_tc_kernel<128>",
-                     "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
-                     "frac": achieved / pk_sust,
-                     "peak_source": (f"{pk_src} bf16 sustained x 2 (fp8 nominal ratio)" if f8 else
-                                     f"{pk_src} bf16 sustained (timed inside long stepping)"),
-                     "frac_of_burst": achieved / pk_burst,
+                     "achieved": res["achieved"], "peak": mul * pk_burst, "unit": "TFLOP/s",
+                     "frac": res["achieved"] / (mul * pk_burst),
+                     "peak_source": (f"{pk_src} bf16 burst x 2 (fp8 nominal ratio)" if f8 else
+                                     f"{pk_src} bf16 burst (kernel timed per launch)"),
+                     "frac_of_sustained": res["achieved"] / (mul * pk_sust),
+                     "frac_of_nominal": res["achieved"] / (mul * NOMINAL_BF16_TFLOPS),
+                     "nominal_peak": mul * NOMINAL_BF16_TFLOPS,
+                     "algorithmic_flops_per_launch": res["att_flops_per_launch"],
                      "duration": "mean of the library's CUDA events around each launch, on "
                                  "its launch stream, over the eager timed pass",
                      "traffic": PROFILED_TRAFFIC.get(attend_source_hash() + ("/e4m3" if f8 else "")),
@@ -684,16 +853,14 @@ def main():
                                       "(7168 keys, cold L2); algorithmic minimum 63 MB (e4m3 "
                                       "Q', K', V in, bf16 O out)") if f8 else
                                      ("ncu dram read+write bytes of one steady-state launch "
-                                      "(7168 keys, cold L2); algorithmic minimum 113 MB; the "
-                                      "excess is split-unit fp32 partials written and read "
-                                      "back and K/V re-reads past L2")},
+                                      "(7168 keys, cold L2); algorithmic minimum 113 MB")},
+        "per_config": per_config,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": launches,
-        "clocks": clocks,
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
     }
     print(json.dumps(line), flush=True)
-    cache.close()
 
 
 if __name__ == "__main__":
