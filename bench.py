@@ -18,7 +18,8 @@ this repository) on the host cores, on a bounded sample of the same workload.
 
 --path gdn measures the Gated DeltaNet block (sa_gdn_chunk) on the same
 stream shape instead: one step = 64 calls of 2,048 tokens from a zero state;
-its roofline is the fp32 FMA peak of the CUDA cores it runs on.
+its roofline is the bf16 tensor peak (D = 128: the sequential pass runs on
+the tensor cores), the fp32 FMA peak for D = 64.
 """
 from __future__ import annotations
 
@@ -373,10 +374,18 @@ def run_gdn(args, w, rank, world):
     flops_per_launch = gdn_flops_per_token(w.D) * w.Lc * w.H * B
     avg_launch_s = statistics.mean(launch_ms) / 1000.0
     achieved = flops_per_launch / avg_launch_s / 1e12
-    peak = FP32_LANES_PER_SM * SM_COUNT * 2 * SM_MAX_GHZ / 1e3
+    alu_peak = FP32_LANES_PER_SM * SM_COUNT * 2 * SM_MAX_GHZ / 1e3
+    tc = w.D == 128  # the sequential pass runs on the tensor cores (bf16 split products)
+    hbm_pk, bf16_burst, _, pk_src = peaks()
+    peak = bf16_burst if tc else alu_peak
+    n_sub = (w.Lc + 63) // 64
+    # tensor-core FLOPs the sequential pass issues per call: per (head, 64-token
+    # block) K^S^T and Q^S^T (2 x 128 x D x D), T and M times the right-hand side
+    # (2 x 128 x 64 x D) and the state update (2 x D x 64 x D), three split terms each
+    issued = 3.0 * (2 * 128 * w.D * w.D + 2 * 128 * 64 * w.D + 2 * w.D * 64 * w.D) * n_sub * w.H * B
     bytes_per_launch = B * (w.Lc * w.H * w.D * esz * 4 + w.Lc * w.H * 8 + 2 * w.H * w.D * w.D * 4)
-    # (the workspace of T and P, 32 KiB per 64 tokens and head, is written and
-    # read back through L2 and is not algorithmic traffic)
+    # (the workspace of the prep kernel's per-block output is written and read
+    # back, mostly through L2, and is not algorithmic traffic)
     hbm = peaks()[0]
 
     # end to end through the public call: pinned host inputs copied in and
@@ -424,11 +433,17 @@ def run_gdn(args, w, rank, world):
         "config": gdn_config_json(w, world, g_scale),
         "ms_per_chunk": ms_step / chunks_per_step,
         "launch_mode": "cuda graph of one step, replayed",
-        "roofline": {"bound": "alu",
-                     "kernel": f"gdn_prep_kernel<{w.D}> + gdn_chunk_kernel<{w.D}> (one call)",
+        "roofline": {"bound": "tensor" if tc else "alu",
+                     "kernel": (f"gdn_prep_kernel<{w.D}> + gdn_tc_kernel (one call)" if tc else
+                                f"gdn_prep_kernel<{w.D}> + gdn_chunk_kernel<{w.D}> (one call)"),
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
-                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP (FMA) x 1.965 GHz",
+                     "peak_source": (f"{pk_src} bf16 burst (the sequential pass issues bf16 "
+                                     f"tensor-core MMAs)" if tc else
+                                     "derived: 148 SMs x 128 fp32 lanes x 2 FLOP (FMA) x 1.965 GHz"),
+                     "frac_of_fp32_alu_peak": achieved / alu_peak,
+                     "issued_tensor_flops_per_launch": issued if tc else 0.0,
+                     "issued_tensor_tflops": (issued / avg_launch_s / 1e12) if tc else 0.0,
                      "algorithmic_flops_per_launch": flops_per_launch,
                      "hbm_bytes_per_launch": bytes_per_launch,
                      "hbm_frac": bytes_per_launch / avg_launch_s / 1e9 / hbm,

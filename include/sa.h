@@ -59,7 +59,8 @@ typedef enum {
   SA_ERR_OOM = 3,            /* device or pinned-host allocation failed */
   SA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
   SA_ERR_STATE = 5,          /* call not valid in the handle's current state */
-  SA_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up on a bounded wait (see sa_get_device_status) */
+  SA_ERR_DEVICE_TIMEOUT = 6, /* a kernel gave up on a bounded wait (see sa_get_device_status) */
+  SA_ERR_DEVICE_BOUNDS = 7   /* debug build: a kernel's index check failed (sa_debug_bounds_status) */
 } sa_status;
 
 /* SA_F32, SA_BF16: q, k, v, out and the cache in that type.
@@ -312,6 +313,27 @@ sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cache, void* v_
  * SA_OK otherwise, SA_ERR_CUDA on a CUDA error. Allocates nothing. */
 sa_status sa_noalloc_device_status(sa_stream_t stream);
 
+/*
+ * Debug build (libsa_debug.so, compiled with -DSA_DEBUG_BOUNDS; no passage on
+ * the pages: robustness of this implementation, the in-kernel stand-in for a
+ * memory checker). Every index a kernel computes into a buffer -- cache rows
+ * of appended frames, raw-sink rows, ring and sink rows of a refresh, query
+ * and key/value tile coordinates, partial-result slots and arrival counters
+ * of split attention units, GDN workspace blocks and state slices -- is
+ * range-checked before the access. A failed check skips the access (a load
+ * reads zero, a tile coordinate is clamped to 0) and sets a bit in a device
+ * word of the kernel's source file; no trap, no fault, the kernel ends.
+ * sa_debug_bounds_status synchronises `stream`, reads and clears those words
+ * on the current device, and returns SA_ERR_DEVICE_BOUNDS (the words in the
+ * error text: file and site bits) if any bit was set, SA_OK otherwise. In the
+ * normal build (libsa.so) the checks are compiled out and both calls return
+ * SA_ERR_UNSUPPORTED. sa_debug_bounds_selftest enqueues one kernel on
+ * `stream` that records a failed check at site 31 of the attention file's
+ * word without any memory access, so a test can see the recording path work.
+ */
+sa_status sa_debug_bounds_status(sa_stream_t stream);
+sa_status sa_debug_bounds_selftest(sa_stream_t stream);
+
 /* Number of kernels the handle launched since sa_profile_begin (host count). */
 sa_status sa_profile_launches(const sa_cache* h, int64_t* launches);
 
@@ -418,19 +440,29 @@ typedef struct {
  *   state  [B][H][D][D] fp32, 16-byte aligned, read and written in place (the
  *          block's whole memory between calls; zero it to start a stream);
  *   q, k, v, out [B][T][H][D] in cfg->dtype (out may not alias the inputs;
- *          q, k and v 16-byte aligned, out aligned to its element);
+ *          all four 16-byte aligned);
  *   g      [B][T][H] fp32, log decay of each token (<= 0; exp(g) multiplies S);
  *   beta   [B][T][H] fp32, write strength of each token (in [0, 1] for a
  *          contracting update; other values are computed as given);
  *   workspace  scratch of workspace_bytes >= sa_gdn_workspace_size(cfg),
- *          16-byte aligned; contents need not be kept between calls. The call
- *          runs two kernels: one computes, for every 64-token block, the
- *          triangular inverse of the chunkwise form and its product with the
- *          decay-masked q.k matrix into the workspace; the other walks the
- *          blocks in order and updates the state.
+ *          16-byte aligned; contents need not be kept between calls. Its
+ *          first 1 KiB holds the call's device status word
+ *          (sa_gdn_device_status). The call runs two kernels: one computes,
+ *          for every 64-token block and all blocks in parallel, the normalised
+ *          keys and queries, the triangular inverse T of the chunkwise form
+ *          and M = scale P T (P the decay-masked q.k matrix) into the
+ *          workspace; the other walks the blocks in order and updates the
+ *          state.
+ * Precision. D = 64: fp32 arithmetic on the CUDA cores. D = 128: the
+ * sequential pass runs its contractions (K S^T, Q S^T, T and M times the
+ * right-hand side, the state update) on the tensor cores as three-term split
+ * products of bf16 operands (x = hi + lo, a.b ~ a_hi.b_hi + a_hi.b_lo +
+ * a_lo.b_hi, fp32 accumulation: about 2^-16 relative per product, within
+ * 1e-4 of the fp64 recurrence on the outputs and the state), with the state
+ * in tensor memory for the whole call; everything else is fp32.
  * active: host array of B flags, NULL = all; an inactive stream's state and
- * out rows are untouched. Arithmetic is fp32 with fp32 state; outputs are
- * rounded once to cfg->dtype. Asynchronous on `stream`, graph-capturable.
+ * out rows are untouched. The state is fp32; outputs are rounded once to
+ * cfg->dtype. Asynchronous on `stream`, graph-capturable.
  * Errors: SA_ERR_INVALID_ARG (cfg, a NULL pointer with tokens > 0, alignment,
  * a workspace smaller than sa_gdn_workspace_size), SA_ERR_UNSUPPORTED (no
  * compute capability 10.x device, or a size that does not fit), SA_ERR_CUDA
@@ -442,12 +474,24 @@ sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, co
                        sa_stream_t stream);
 
 /*
- * Bytes of the device workspace sa_gdn_chunk needs for cfg: 32 KiB per
- * (stream, head, started 64-token block of the call), i.e.
- * batch * heads * ceil(tokens / 64) * 32768.
+ * Bytes of the device workspace sa_gdn_chunk needs for cfg: a 1 KiB header
+ * plus, per (stream, head, started 64-token block of the call), 96 KiB for
+ * D = 128 (the operand images of the tensor-core pass) or 32 KiB for D = 64,
+ * i.e. 1024 + batch * heads * ceil(tokens / 64) * (98304 or 32768).
  * Errors: SA_ERR_INVALID_ARG (cfg invalid or bytes NULL), SA_ERR_UNSUPPORTED.
  */
 sa_status sa_gdn_workspace_size(const sa_gdn_config* cfg, size_t* bytes);
+
+/*
+ * Device status of the last sa_gdn_chunk call that used `workspace` (no
+ * passage on the pages: robustness of this implementation). Synchronises
+ * `stream` and reads the status word the call's kernels keep in the
+ * workspace header (cleared by each call's first kernel). Returns
+ * SA_ERR_DEVICE_TIMEOUT if a bounded wait of the tensor-core pass gave up
+ * (the call's outputs and state are not valid), SA_OK otherwise,
+ * SA_ERR_INVALID_ARG for a NULL or unaligned workspace, SA_ERR_CUDA.
+ */
+sa_status sa_gdn_device_status(const void* workspace, sa_stream_t stream);
 
 const char* sa_last_error_string(void);
 

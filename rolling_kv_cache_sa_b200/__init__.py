@@ -14,4 +14,5 @@ from .cache import (  # noqa: F401
     sa_sink_update, sa_append_attend_host_async, sa_host_wait, sa_cache_set_fp8_scales,
     sa_cache_export, sa_cache_import, sa_cache_get_fp8_scales, sa_noalloc_device_status,
 )
-from .gdn import GDNState, gdn_workspace, sa_gdn_chunk, sa_gdn_workspace_size  # noqa: F401
+from .gdn import (GDNState, gdn_workspace, sa_gdn_chunk, sa_gdn_device_status,  # noqa: F401
+                  sa_gdn_workspace_size)

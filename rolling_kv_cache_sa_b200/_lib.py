@@ -5,12 +5,16 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsa.so")
+# SA_LIBRARY_VARIANT=debug loads the debug build (index checks in every kernel,
+# sa_debug_bounds_status); anything else the normal build
+LIB_PATH = os.path.join(_HERE, "libsa_debug.so" if os.environ.get("SA_LIBRARY_VARIANT") == "debug"
+                        else "libsa.so")
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_OOM, SA_ERR_CUDA, SA_ERR_STATE, \
-    SA_ERR_DEVICE_TIMEOUT = range(7)
+    SA_ERR_DEVICE_TIMEOUT, SA_ERR_DEVICE_BOUNDS = range(8)
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_OOM",
-                4: "SA_ERR_CUDA", 5: "SA_ERR_STATE", 6: "SA_ERR_DEVICE_TIMEOUT"}
+                4: "SA_ERR_CUDA", 5: "SA_ERR_STATE", 6: "SA_ERR_DEVICE_TIMEOUT",
+                7: "SA_ERR_DEVICE_BOUNDS"}
 SA_F32, SA_BF16, SA_BF16_E4M3 = 0, 1, 2
 SA_SINK_SHIFT, SA_SINK_REPIN = 0, 1
 SA_MAX_CHUNK_FRAMES = 32
@@ -25,6 +29,7 @@ EXPORTED = (
     "sa_sink_update", "sa_append_attend_host_async", "sa_host_wait", "sa_cache_set_fp8_scales",
     "sa_cache_export_size", "sa_cache_export", "sa_cache_import", "sa_cache_get_fp8_scales",
     "sa_gdn_chunk", "sa_gdn_workspace_size", "sa_noalloc_device_status",
+    "sa_debug_bounds_status", "sa_debug_bounds_selftest", "sa_gdn_device_status",
 )
 
 
@@ -108,6 +113,9 @@ def lib() -> ctypes.CDLL:
                          vp],
         "sa_gdn_workspace_size": [P(sa_gdn_config), P(ctypes.c_size_t)],
         "sa_noalloc_device_status": [vp],
+        "sa_debug_bounds_status": [vp],
+        "sa_debug_bounds_selftest": [vp],
+        "sa_gdn_device_status": [vp, vp],
         "sa_profile_end": [vp, P(ctypes.c_double), P(i32), P(ctypes.c_double), P(i32),
                            P(ctypes.c_double), P(i32)],
     }

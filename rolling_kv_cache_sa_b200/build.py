@@ -6,6 +6,8 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsa.so")
+# the debug build: every computed buffer index is range-checked in the kernels
+DEBUG_LIB = os.path.join(HERE, "libsa_debug.so")
 
 NVCC_FLAGS = ["-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
               "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
@@ -23,22 +25,34 @@ def deps():
 
 
 def is_stale() -> bool:
-    if not os.path.exists(LIB):
-        return True
-    t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(s) > t for s in deps())
+    for lib in (LIB, DEBUG_LIB):
+        if not os.path.exists(lib):
+            return True
+        t = os.path.getmtime(lib)
+        if any(os.path.getmtime(s) > t for s in deps()):
+            return True
+    return False
 
 
 def build(verbose: bool = False) -> str:
-    cmd = ["nvcc", *NVCC_FLAGS, *sources(), "-o", LIB, "-lcuda", "-ldl"]
+    """Builds libsa.so and the debug build libsa_debug.so (-DSA_DEBUG_BOUNDS)
+    side by side; returns the path of libsa.so."""
+    cmds = [["nvcc", *NVCC_FLAGS, *sources(), "-o", LIB, "-lcuda", "-ldl"],
+            ["nvcc", *NVCC_FLAGS, "-DSA_DEBUG_BOUNDS", *sources(), "-o", DEBUG_LIB, "-lcuda",
+             "-ldl"]]
     if verbose:
-        print(" ".join(cmd))
-    r = subprocess.run(cmd, capture_output=True, text=True)
+        for c in cmds:
+            print(" ".join(c))
+    procs = [subprocess.Popen(c, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+             for c in cmds]
+    outs = [pr.communicate() for pr in procs]
     log = os.path.join(HERE, "build.log")
     with open(log, "w") as f:
-        f.write(r.stdout + r.stderr)
-    if r.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + r.stderr[-6000:])
+        for (o, e) in outs:
+            f.write(o + e)
+    for pr, (o, e) in zip(procs, outs):
+        if pr.returncode != 0:
+            raise RuntimeError("nvcc failed:\n" + e[-6000:])
     return LIB
 
 

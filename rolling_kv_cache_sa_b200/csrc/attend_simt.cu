@@ -10,6 +10,11 @@
 #include "internal.h"
 
 namespace sa {
+
+// debug build: the bounds word of this file (sites: 0 stream / key prefix of
+// a (stream, head), 1 output row)
+SA_DEFINE_BOUNDS_WORD(bounds_word_attend_simt)
+
 namespace {
 
 constexpr int kRows = 16;  // query rows per block
@@ -29,6 +34,8 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(const __grid_constant_
   const int row0 = blockIdx.x * kRows;
   const int n_keys = p.n_keys[a];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // (block-uniform: the whole block leaves before any barrier)
+  if (!SA_BOUNDS(b >= 0 && b < p.batch && n_keys >= 0 && n_keys <= p.ntok, 0)) return;
   const int64_t bh = (int64_t)b * p.H + h;
   const float* q = static_cast<const float*>(p.q_ws) + bh * p.Lc * D;
   const float* kc = static_cast<const float*>(p.k_cache) + bh * p.ntok * D;
@@ -92,6 +99,7 @@ __global__ void __launch_bounds__(256) attend_simt_kernel(const __grid_constant_
   for (int rr = 0; rr < 2; ++rr) {
     const int tok = row0 + warp * 2 + rr;
     if (tok >= p.Lc) continue;
+    if (!SA_BOUNDS(h < p.H, 1)) continue;
     const float inv = 1.f / l[rr];
     float* dst = out + (((int64_t)b * p.Lc + tok) * p.H + h) * D;
 #pragma unroll

@@ -40,21 +40,51 @@
 #include "ptx.cuh"
 
 namespace sa {
+
+// debug build: the bounds word of this file (sites: 0 query tile coordinate,
+// 1 key/value tile coordinate, 2 output row, 3 partial-result slot written,
+// 4 arrival counter, 5 partial-result slot read by a merge, 31 self-test)
+SA_DEFINE_BOUNDS_WORD(bounds_word_attend_tc)
+
 namespace {
 
 constexpr int BM = 128;                  // query rows per tile
 constexpr int BN = 128;                  // keys per tile
 constexpr uint32_t PANEL = 128u * 128u;  // one 128-row x 128-byte swizzled panel
 constexpr uint64_t kTimeoutNs = 1000000000ull;
-constexpr int kThreads = 320;
+// 10 warps (producer, MMA issuer, two softmax warpgroups; 168 registers each
+// thread) or, with SA_ATTN_WARPS12, 12 warps in three warpgroups whose
+// registers are redistributed with setmaxnreg: the producer/MMA warpgroup
+// gives up registers to the two softmax warpgroups (launch 384 x 168 =
+// 128 x kRegLow + 256 x kRegHigh, so the increase always finds its registers).
+#ifndef SA_ATTN_WARPS12
+#define SA_ATTN_WARPS12 0
+#endif
+constexpr bool kWarps12 = SA_ATTN_WARPS12 != 0;
+constexpr int kThreads = kWarps12 ? 384 : 320;
+constexpr int kFirstSoftmaxWarp = kWarps12 ? 4 : 2;
+constexpr int kRegLaunch = 168, kRegLow = 96, kRegHigh = 200;
+static_assert(128 * kRegLow + 256 * kRegHigh <= 384 * kRegLaunch, "register split exceeds the launch");
 constexpr int kMaxCtas = 256;
+#ifndef SA_ATTN_HYBRID
+#define SA_ATTN_HYBRID 1
+#endif
+constexpr bool kHybrid = SA_ATTN_HYBRID != 0;
+#ifndef SA_ATTN_ROTATE
+#define SA_ATTN_ROTATE 1
+#endif
+constexpr bool kRotate = SA_ATTN_ROTATE != 0;
 
 struct TcParams {
   int32_t H, Lc, n_q_tiles, n_pairs;
   int32_t n_streams, grid, split, units_per_stream;
   float scale_log2;
-  int32_t pad_;
+  int32_t batch;      // B (bounds checks)
+  int64_t ntok;       // cache rows per (stream, head) (bounds checks)
   int64_t total;      // key tiles over all units
+  int32_t full;       // split mode: whole units per CTA taken first (0: pure stream-K)
+  int32_t pad2_;
+  int64_t t1;         // split mode: first key tile of the units split between CTAs
   void* out;          // [B][Lc][H][D] bf16
   float4* part_o;     // [slots][2][D/4][128] fp32 (row-contiguous per column quad)
   float2* part_ml;    // [slots][2][128] (m in log2 units, l)
@@ -81,14 +111,24 @@ __host__ __device__ inline int64_t unit_tile_offset(const TcParams& p, int64_t u
   return p.prefix[a] + (u - (int64_t)a * p.units_per_stream) * p.nkv[a];
 }
 
-__host__ __device__ inline void cta_range(const TcParams& p, int c, int64_t& r0, int64_t& r1) {
+// The key tiles CTA c takes in split mode, [r0, r1): an equal share of the
+// tiles from t1 on (the units split between CTAs). With full > 0 the CTA
+// first takes the whole units [c * full, (c + 1) * full) (tiles [w0, w1)),
+// so only the last units are split and their pieces all run at the end of
+// the launch, close together in time. Without a partials buffer, ranges
+// snap to whole units (w0 = w1).
+__host__ __device__ inline void cta_range(const TcParams& p, int c, int64_t& r0, int64_t& r1,
+                                          int64_t& w0, int64_t& w1) {
   if (p.split) {
-    r0 = p.total * c / p.grid;
-    r1 = p.total * (c + 1) / p.grid;
+    w0 = unit_tile_offset(p, (int64_t)c * p.full);
+    w1 = unit_tile_offset(p, (int64_t)(c + 1) * p.full);
+    r0 = p.t1 + (p.total - p.t1) * c / p.grid;
+    r1 = p.t1 + (p.total - p.t1) * (c + 1) / p.grid;
   } else {
     const int64_t U = (int64_t)p.n_streams * p.units_per_stream;
     r0 = unit_tile_offset(p, U * c / p.grid);
     r1 = unit_tile_offset(p, U * (c + 1) / p.grid);
+    w0 = w1 = 0;
   }
 }
 
@@ -115,30 +155,81 @@ __host__ __device__ inline Seg make_seg(const TcParams& p, int64_t t, int64_t r1
   return s;
 }
 
-// CTA whose range holds key tile t (split mode)
+// The order in which a CTA takes its segments: first its whole units [w0, w1)
+// (split mode with full > 0), then its share [r0, r1) of the split units.
+// When r0 falls inside a unit (the head piece of a unit the previous CTA
+// began) and nothing else comes first, that piece goes after the rest of the
+// share, so both pieces of a unit split between CTAs c and c + 1 end near
+// the same time and the last one merges the partials while they are in L2.
+// Every role of the CTA walks the same cursor, so they agree on the order.
+struct SegCursor {
+  int64_t t, stop;   // current range
+  int64_t nx0, nx1;  // next range
+  int64_t nz0, nz1;  // the one after it
+  __device__ void init(const TcParams& p, int64_t r0, int64_t r1, int64_t w0, int64_t w1) {
+    int64_t h_end = r0;
+    if (kRotate && w0 >= w1 && r0 < r1) {
+      const Seg h = make_seg(p, r0, r1);
+      if (h.lo > 0 && h.t_end < r1) h_end = h.t_end;
+    }
+    t = w0;
+    stop = w1;
+    nx0 = h_end;
+    nx1 = r1;
+    nz0 = r0;
+    nz1 = h_end;
+  }
+  __device__ bool next(const TcParams& p, Seg& s) {
+    while (t >= stop) {
+      if (nx0 >= nx1 && nz0 >= nz1) return false;
+      t = nx0;
+      stop = nx1;
+      nx0 = nz0;
+      nx1 = nz1;
+      nz0 = nz1 = 0;
+    }
+    s = make_seg(p, t, stop);
+    t = s.t_end;
+    return true;
+  }
+};
+
+// CTA whose split share holds key tile t (t >= t1; split mode)
 __device__ inline int cta_of(const TcParams& p, int64_t t) {
-  int c = (int)(t * p.grid / p.total);
-  while (c + 1 < p.grid && p.total * (c + 1) / p.grid <= t) ++c;
-  while (c > 0 && p.total * c / p.grid > t) --c;
+  const int64_t n = p.total - p.t1, x = t - p.t1;
+  int c = (int)(x * p.grid / n);
+  while (c + 1 < p.grid && n * (c + 1) / p.grid <= x) ++c;
+  while (c > 0 && n * c / p.grid > x) --c;
   return c;
 }
 
 // Partial slot of the piece that CTA c holds of the unit starting at tile us:
-// slot 2c for a CTA's first segment, 2c + 1 for a later one.
+// slot 2c for the piece that starts c's split share, 2c + 1 for the one that
+// ends it.
 __device__ inline int piece_slot(const TcParams& p, int c, int c_first, int64_t us) {
-  return 2 * c + ((c == c_first && p.total * c / p.grid != us) ? 1 : 0);
+  return 2 * c + ((c == c_first && p.t1 + (p.total - p.t1) * c / p.grid != us) ? 1 : 0);
 }
 
 // Merge of one query row of a split unit from the partial results of its
 // pieces (CTAs c0..c1): O = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,
 // stored as bf16 to dst (nullptr: a padding row past Lc, nothing stored).
-// Kept out of line so the softmax loop's register allocation does not see it.
+// The other pieces' partials were written long before and are usually out of
+// L2, so every line of this row is first prefetched into L2 (one memory
+// latency for all of them instead of one per piece and column chunk); two
+// pieces -- the only case at the workload sizes, where a CTA's range is longer
+// than a unit -- are then read together. Kept out of line so the softmax
+// loop's register allocation does not see it.
 template <int HD>
 __device__ __noinline__ void merge_row(const TcParams& p, int ti, int row, int c0, int c1,
                                        int64_t us, __nv_bfloat16* dst) {
   float M = -INFINITY;
   for (int c = c0; c <= c1; ++c) {
     const int sl = piece_slot(p, c, c0, us);
+    if (!SA_BOUNDS(sl >= 0 && sl < 2 * p.grid, 5)) return;
+    const float4* src = p.part_o + ((int64_t)sl * 2 + ti) * (HD / 4) * BM + row;
+#pragma unroll
+    for (int g4 = 0; g4 < HD / 4; ++g4)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(src + g4 * BM));
     M = fmaxf(M, __ldcg(p.part_ml + ((int64_t)sl * 2 + ti) * BM + row).x);
   }
   float Ls = 0.f;
@@ -149,6 +240,33 @@ __device__ __noinline__ void merge_row(const TcParams& p, int ti, int row, int c
   }
   const float inv = 1.f / Ls;
   if (!dst) return;
+  if (c1 == c0 + 1) {
+    const int s0 = piece_slot(p, c0, c0, us), s1 = piece_slot(p, c1, c0, us);
+    const float w0 = ptx::ex2(__ldcg(p.part_ml + ((int64_t)s0 * 2 + ti) * BM + row).x - M) * inv;
+    const float w1 = ptx::ex2(__ldcg(p.part_ml + ((int64_t)s1 * 2 + ti) * BM + row).x - M) * inv;
+    const float4* a0 = p.part_o + ((int64_t)s0 * 2 + ti) * (HD / 4) * BM + row;
+    const float4* a1 = p.part_o + ((int64_t)s1 * 2 + ti) * (HD / 4) * BM + row;
+#pragma unroll 1
+    for (int cc = 0; cc < HD / 32; ++cc) {
+      float4 x0[8], x1[8];
+#pragma unroll
+      for (int g4 = 0; g4 < 8; ++g4) {
+        x0[g4] = __ldcg(a0 + (cc * 8 + g4) * BM);
+        x1[g4] = __ldcg(a1 + (cc * 8 + g4) * BM);
+      }
+#pragma unroll
+      for (int g8 = 0; g8 < 4; ++g8) {
+        const float4 u0 = x0[2 * g8], u1 = x0[2 * g8 + 1], v0 = x1[2 * g8], v1 = x1[2 * g8 + 1];
+        uint4 o;
+        o.x = ptx::pack_bf16x2(fmaf(w0, u0.x, w1 * v0.x), fmaf(w0, u0.y, w1 * v0.y));
+        o.y = ptx::pack_bf16x2(fmaf(w0, u0.z, w1 * v0.z), fmaf(w0, u0.w, w1 * v0.w));
+        o.z = ptx::pack_bf16x2(fmaf(w0, u1.x, w1 * v1.x), fmaf(w0, u1.y, w1 * v1.y));
+        o.w = ptx::pack_bf16x2(fmaf(w0, u1.z, w1 * v1.z), fmaf(w0, u1.w, w1 * v1.w));
+        *reinterpret_cast<uint4*>(dst + cc * 32 + g8 * 8) = o;
+      }
+    }
+    return;
+  }
 #pragma unroll 1
   for (int cc = 0; cc < HD / 32; ++cc) {
     float acc[32];
@@ -206,6 +324,56 @@ struct Layout {
   static constexpr uint32_t bytes = misc + 16;
   static_assert(bytes <= 232448, "exceeds 227 KB of shared memory per CTA");
 };
+
+// 2^x of two floats on the FMA pipe instead of the MUFU unit, by the range
+// reduction of Cody and Waite (1980): x = n + f with n = round(x) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with constant term 1, fitted
+// here by a minimax linear program on [-1/2, 1/2] (relative error 1.0e-4,
+// below the 2^-9 of the bf16 rounding that P then goes through); 2^n is
+// added to the exponent field. round(x) comes from adding 1.5 * 2^23 (the
+// sum's low mantissa bits hold n), so no conversion instruction is used.
+// x is clamped to -120 first (masked columns are -inf), which keeps the
+// exponent field positive; 2^-120 instead of 0 is negligible against the
+// row's largest term (>= 2^-8).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c1 = 0x1.62f5fap-1f, c2 = 0x1.f00c4cp-3f, c3 = 0x1.c2a21ap-5f;
+  x.x = fmaxf(x.x, -120.f);
+  x.y = fmaxf(x.y, -120.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));            // kRound + n
+  const float2 r = __ffma2_rn(t, make_float2(-1.f, -1.f), make_float2(kRound, kRound));  // -n
+  const float2 f = __fadd2_rn(x, r);                                      // exact
+  float2 pf = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  pf = __ffma2_rn(pf, f, make_float2(c1, c1));
+  pf = __ffma2_rn(pf, f, make_float2(1.f, 1.f));
+  return make_float2(__uint_as_float(__float_as_uint(pf.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(pf.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Pairs of a 32-score group whose exponentials run on the FMA pipe: kPoly of
+// the 16, spread evenly (pair e when (e * kPoly) mod 16 < kPoly).
+#ifndef SA_EXP2_POLY_PAIRS
+#define SA_EXP2_POLY_PAIRS 0
+#endif
+
+// P of 32 consecutive scores of a row as 16 words of bf16 pairs, and their
+// sum added to ls (four packed partial sums).
+template <int kPoly>
+__device__ __forceinline__ void p_group(const uint32_t* sv, float2 sl2v, float2 nmv, float2* ls,
+                                        uint32_t* w) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * e]),
+                                            __uint_as_float(sv[2 * e + 1])), sl2v, nmv);
+    float2 pe;
+    if ((e * kPoly) % 16 < kPoly)
+      pe = exp2_poly2(x);
+    else
+      pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+    ls[e & 3] = __fadd2_rn(ls[e & 3], pe);
+    w[e] = ptx::pack_bf16x2(pe.x, pe.y);
+  }
+}
 
 // O row *= alpha in TMEM (rare; out of line so that the softmax keeps its
 // scores in registers without spilling around it)
@@ -330,32 +498,15 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
   float2 ls[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) ls[i] = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int q = 0; q < BN / 32; ++q) {
-    uint32_t w[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[q * 32 + 2 * e]),
-                                              __uint_as_float(sv[q * 32 + 2 * e + 1])),
-                                  sl2v, nmv);
-      const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
-      ls[e & 3] = __fadd2_rn(ls[e & 3], pe);
-      if constexpr (F8) {
-        // four e4m3 per column: pairs e and e+1 share a word
-        const uint32_t pp = ptx::pack_e4m3x2(pe.x, pe.y);
-        if (e & 1)
-          w[e >> 1] |= pp << 16;
-        else
-          w[e >> 1] = pp;
-      } else {
-        w[e] = ptx::pack_bf16x2(pe.x, pe.y);
-      }
-    }
-    if constexpr (F8)
-      ptx::tmem_st8u(sbuf + (uint32_t)(q * 8), w);
-    else
-      ptx::tmem_st16u(sbuf + (uint32_t)(q * 16), w);
-    if (q == 1 && __any_sync(0xffffffffu, alpha < 1.f)) {
+  if constexpr (!F8) {
+    // bf16: groups of 32 keys; the third group is computed before waiting
+    // for the first two groups' TMEM stores, so that wait overlaps work
+    uint32_t wa[16], wb[16];
+    p_group<SA_EXP2_POLY_PAIRS>(sv, sl2v, nmv, ls, wa);
+    ptx::tmem_st16u(sbuf, wa);
+    p_group<SA_EXP2_POLY_PAIRS>(sv + 32, sl2v, nmv, ls, wb);
+    ptx::tmem_st16u(sbuf + 16u, wb);
+    if (__any_sync(0xffffffffu, alpha < 1.f)) {
       // O holds PV of the previous key tile: MMAs complete in issue order and
       // QK of this tile (issued after that PV) has completed
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_od, od_parity, abort_flag, kTimeoutNs)))
@@ -363,15 +514,57 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
       ptx::tc_fence_after();
       rescale_o<HD>(obuf, alpha);
     }
-    if (q == 1 || q == 3) {
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(q == 1 ? bar_pa : bar_pb);
+    p_group<SA_EXP2_POLY_PAIRS>(sv + 64, sl2v, nmv, ls, wa);
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(bar_pa);
+    ptx::tmem_st16u(sbuf + 32u, wa);
+    p_group<SA_EXP2_POLY_PAIRS>(sv + 96, sl2v, nmv, ls, wb);
+    ptx::tmem_st16u(sbuf + 48u, wb);
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(bar_pb);
+    const float2 l2 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+    l = l * alpha + (l2.x + l2.y);
+    return true;
+  } else {
+    // e4m3 exact path (first tile of a unit, or the running max jumped)
+#pragma unroll
+    for (int q = 0; q < BN / 32; ++q) {
+      uint32_t w[8];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[q * 32 + 2 * e]),
+                                                __uint_as_float(sv[q * 32 + 2 * e + 1])),
+                                    sl2v, nmv);
+        const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+        ls[e & 3] = __fadd2_rn(ls[e & 3], pe);
+        // four e4m3 per column: pairs e and e+1 share a word
+        const uint32_t pp = ptx::pack_e4m3x2(pe.x, pe.y);
+        if (e & 1)
+          w[e >> 1] |= pp << 16;
+        else
+          w[e >> 1] = pp;
+      }
+      ptx::tmem_st8u(sbuf + (uint32_t)(q * 8), w);
+      if (q == 1 && __any_sync(0xffffffffu, alpha < 1.f)) {
+        // O holds PV of the previous key tile: MMAs complete in issue order
+        // and QK of this tile (issued after that PV) has completed
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_od, od_parity, abort_flag, kTimeoutNs)))
+          return false;
+        ptx::tc_fence_after();
+        rescale_o<HD>(obuf, alpha);
+      }
+      if (q == 1 || q == 3) {
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(q == 1 ? bar_pa : bar_pb);
+      }
     }
+    const float2 l2 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+    l = l * alpha + (l2.x + l2.y);
+    return true;
   }
-  const float2 l2 = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
-  l = l * alpha + (l2.x + l2.y);
-  return true;
 }
 
 template <int HD, bool F8>
@@ -433,9 +626,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 1;
     atomicOr(p.status, kDeviceErrTimeout);
   };
-  int64_t r0, r1;
-  cta_range(p, blockIdx.x, r0, r1);
-
+  int64_t r0, r1, w0, w1;
+  cta_range(p, blockIdx.x, r0, r1, w0, w1);
+  if (warp < kFirstSoftmaxWarp) {
+  if constexpr (kWarps12) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -444,14 +638,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm_v);
       int n = 0, g = 0;
       bool ok = true;
-      for (int64_t t = r0; ok && t < r1;) {
-        const Seg sg = make_seg(p, t, r1);
-        t = sg.t_end;
+      SegCursor cur;
+      cur.init(p, r0, r1, w0, w1);
+      Seg sg;
+      while (ok && cur.next(p, sg)) {
         if (n > 0 && !ptx::mbar_wait(bar(L::B_QE), (uint32_t)(n - 1) & 1, abort_flag, kTimeoutNs)) {
           ok = false;
           break;
         }
-        const int bh = sg.b * p.H + sg.h;
+        int bh = sg.b * p.H + sg.h;
+        // (a bad coordinate is clamped: the copy still completes the barrier)
+        if (!SA_BOUNDS(bh >= 0 && bh < p.batch * p.H && sg.qp >= 0 &&
+                           (2 * sg.qp + (sg.two ? 1 : 0)) < p.n_q_tiles, 0))
+          bh = 0, sg.qp = 0;
         ptx::mbar_arrive_expect_tx(bar(L::B_QF), (sg.two ? 2u : 1u) * L::kTile);
         for (int i = 0; i < (sg.two ? 2 : 1); ++i)
           for (uint32_t pn = 0; pn < L::kPanels; ++pn)
@@ -465,10 +664,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          const int kr = SA_BOUNDS(kv >= 0 && kv < sg.nkv && (int64_t)kv * BN < p.ntok, 1) ? kv : 0;
           ptx::mbar_arrive_expect_tx(bar(L::B_KF + s), L::kTile);
           for (uint32_t pn = 0; pn < L::kPanels; ++pn)
             ptx::tma_load_3d(base + L::k0 + s * L::kTile + pn * PANEL, &tm_k, bar(L::B_KF + s),
-                             (int)pn * 64, kv * BN, bh);
+                             (int)pn * 64, kr * BN, bh);
           if (u > 0 && !ptx::mbar_wait(bar(L::B_VE + s), (u - 1) & 1, abort_flag, kTimeoutNs)) {
             ok = false;
             ++g;  // K of this tile is in flight: drain it below
@@ -477,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::mbar_arrive_expect_tx(bar(L::B_VF + s), L::kTile);
           for (uint32_t pn = 0; pn < L::kPanels; ++pn)
             ptx::tma_load_3d(base + L::v0 + s * L::kTile + pn * PANEL, &tm_v, bar(L::B_VF + s),
-                             (int)pn * 64, kv * BN, bh);
+                             (int)pn * 64, kr * BN, bh);
         }
       }
       if (!ok) fail();
@@ -535,9 +735,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         pend = false;
         return true;
       };
-      for (int64_t t = r0; ok && t < r1;) {
-        const Seg sg = make_seg(p, t, r1);
-        t = sg.t_end;
+      SegCursor cur;
+      cur.init(p, r0, r1, w0, w1);
+      Seg sg;
+      while (ok && cur.next(p, sg)) {
         if (pend && !issue_pv1()) { ok = false; break; }
         if (!ptx::mbar_wait(bar(L::B_QF), (uint32_t)n & 1, abort_flag, kTimeoutNs)) { ok = false; break; }
         for (int kv = sg.lo; kv < sg.hi; ++kv, ++g) {
@@ -609,21 +810,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::umma_commit(bar(L::B_DR));
       ptx::mbar_wait(bar(L::B_DR), 0, no_abort, kTimeoutNs);
     }
+  }
   } else {
+    if constexpr (kWarps12) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh));
     // ------------------------------------------------------------ softmax + epilogue
-    const int ti = (warp - 2) >> 2;  // query tile: warps 2..5 -> 0, warps 6..9 -> 1
+    const int ti = (warp - kFirstSoftmaxWarp) >> 2;  // query tile of this warp's warpgroup
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t sbuf = t_lane + (uint32_t)ti * 128u;
     const uint32_t obuf = t_lane + 256u + (uint32_t)(ti * HD);
     int gi = 0;
-    bool ok = true, first = true;
-    for (int64_t t = r0; ok && t < r1;) {
-      const Seg sg = make_seg(p, t, r1);
-      t = sg.t_end;
-      const bool seg_first = first;
-      first = false;
+    bool ok = true;
+    SegCursor cur;
+    cur.init(p, r0, r1, w0, w1);
+    Seg sg;
+    while (ok && cur.next(p, sg)) {
       if (ti == 1 && !sg.two) continue;
       // e4m3: scores carry the head's q and k scales, O its v scale
       const float sl2 = F8 ? p.scale_log2 * p.inv_qk[sg.h] : p.scale_log2;
@@ -656,6 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue of this unit piece
       const int tok = (2 * sg.qp + ti) * BM + row;
       if (!sg.partial) {
+        const bool st_ok = SA_BOUNDS(sg.b >= 0 && sg.b < p.batch && sg.h < p.H, 2);
         const float inv = o_scale / l;
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
                              (((int64_t)sg.b * p.Lc + tok) * p.H + sg.h) * HD;
@@ -664,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float ov[32];
           ptx::tmem_ld32(obuf + c * 32, ov);
           ptx::tmem_wait_ld();
-          if (tok < p.Lc) {
+          if (tok < p.Lc && st_ok) {
 #pragma unroll
             for (int g8 = 0; g8 < 4; ++g8) {
               uint4 v;
@@ -677,19 +880,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        const int slot = 2 * (int)blockIdx.x + (seg_first ? 0 : 1);
+        // slot 2c holds the piece that starts the CTA's range, 2c + 1 the
+        // other (a CTA has at most two partial pieces: its first and last)
+        const int slot = 2 * (int)blockIdx.x + (sg.t_end - (sg.hi - sg.lo) == r0 ? 0 : 1);
+        const bool sl_ok = SA_BOUNDS(slot >= 0 && slot < 2 * p.grid, 3);
         float4* po = p.part_o + ((int64_t)slot * 2 + ti) * (HD / 4) * BM + row;
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           float ov[32];
           ptx::tmem_ld32(obuf + c * 32, ov);
           ptx::tmem_wait_ld();
+          if (sl_ok) {
 #pragma unroll
-          for (int g4 = 0; g4 < 8; ++g4)  // partials in output units (v scale removed)
-            po[(c * 8 + g4) * BM] = make_float4(ov[g4 * 4] * o_scale, ov[g4 * 4 + 1] * o_scale,
-                                                ov[g4 * 4 + 2] * o_scale, ov[g4 * 4 + 3] * o_scale);
+            for (int g4 = 0; g4 < 8; ++g4)  // partials in output units (v scale removed)
+              po[(c * 8 + g4) * BM] = make_float4(ov[g4 * 4] * o_scale, ov[g4 * 4 + 1] * o_scale,
+                                                  ov[g4 * 4 + 2] * o_scale, ov[g4 * 4 + 3] * o_scale);
+          }
         }
-        p.part_ml[((int64_t)slot * 2 + ti) * BM + row] = make_float2(m_used, l);
+        if (sl_ok) p.part_ml[((int64_t)slot * 2 + ti) * BM + row] = make_float2(m_used, l);
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar(L::B_OF + ti));  // O_i is free for the next unit
@@ -700,7 +908,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t u = (int64_t)sg.a * p.units_per_stream + (int64_t)sg.h * p.n_pairs + sg.qp;
         int* ctr = p.counters + (u * 2 + ti) * BM + row;
         __threadfence();
-        if (atomicAdd(ctr, 1) == c1 - c0) {
+        if (SA_BOUNDS(u >= 0 && u < (int64_t)p.n_streams * p.units_per_stream && c0 >= 0 &&
+                          c1 < p.grid && c0 <= c1, 4) &&
+            atomicAdd(ctr, 1) == c1 - c0) {
           atomicExch(ctr, 0);
           __threadfence();
           merge_row<HD>(p, ti, row, c0, c1, us,
@@ -742,6 +952,8 @@ cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtenso
   p.n_streams = ap.n_streams;
   p.units_per_stream = p.H * p.n_pairs;
   p.scale_log2 = ap.scale_log2;
+  p.batch = ap.batch;
+  p.ntok = ap.ntok;
   p.out = ap.out;
   p.status = ap.status;
   if (F8)
@@ -765,6 +977,19 @@ cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtenso
   p.split = partials != nullptr && partials_bytes >= need && total >= G;
   if (!p.split) G = (int)std::min<int64_t>(G, units);
   p.grid = G;
+  p.full = 0;
+  p.t1 = 0;
+  if (p.split && kHybrid) {
+    // whole units first when every unit costs the same (equal key counts):
+    // full per CTA, and the rest split; at least G key tiles must remain to
+    // split so that every CTA's share is non-empty
+    bool equal = true;
+    for (int a = 1; a < ap.n_streams; ++a) equal = equal && p.nkv[a] == p.nkv[0];
+    int64_t full = equal ? units / G : 0;
+    while (full > 0 && total - unit_tile_offset(p, full * G) < G) --full;
+    p.full = (int32_t)full;
+    p.t1 = unit_tile_offset(p, full * G);
+  }
   if (p.split) {
     char* w = static_cast<char*>(partials);
     p.part_o = reinterpret_cast<float4*>(w);
@@ -781,7 +1006,18 @@ cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtenso
   return cudaSuccess;
 }
 
+#ifdef SA_DEBUG_BOUNDS
+__global__ void bounds_selftest_kernel() { (void)SA_BOUNDS(threadIdx.x != 0, 31); }
+#endif
+
 }  // namespace
+
+#ifdef SA_DEBUG_BOUNDS
+cudaError_t bounds_selftest(cudaStream_t st) {
+  bounds_selftest_kernel<<<1, 32, 0, st>>>();
+  return cudaGetLastError();
+}
+#endif
 
 size_t attend_partials_bytes(int D, int num_sms, int64_t max_units) {
   const size_t G = (size_t)std::min(num_sms, kMaxCtas);

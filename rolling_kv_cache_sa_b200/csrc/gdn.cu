@@ -41,8 +41,15 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace sa {
+
+// debug build: the bounds word of this file (sites: 0 stream / sub-chunk of a
+// prep block, 1 workspace block written, 2 workspace block read, 3 state
+// slice, 4 sub-chunk token range)
+SA_DEFINE_BOUNDS_WORD(bounds_word_gdn)
+
 namespace {
 
 constexpr int kCt = 64;         // tokens per sub-chunk
@@ -51,6 +58,42 @@ constexpr int kGdnThreads = 256;
 constexpr int kLp = kCt + 4;    // row pitch of the 64 x 64 matrices (16-byte rows)
 constexpr int kVp = kDvs + 4;   // row pitch of the 64 x 32 matrices (16-byte rows)
 constexpr int kTpFloats = 2 * kCt * kCt;   // T and P of one sub-chunk in the workspace
+// The workspace starts with a 1 KiB header holding the device status word of
+// the tensor-core path (bounded waits); the per-sub-chunk blocks follow.
+constexpr size_t kWsHeader = 1024;
+// Tensor-core path (D = 128): per sub-chunk the prep kernel writes the
+// operand images of the sequential kernel's MMAs, bf16, each value x as
+// hi = bf16(x) and lo = bf16(x - hi), in the 128-byte-swizzled layout the
+// tensor core reads (64-column panels; row r at r * 128 bytes of its panel,
+// the 16-byte chunk c of row r stored at chunk c ^ (r mod 8)):
+//   KQ: rows 0..63 the normalised keys, rows 64..127 the normalised queries,
+//       128 columns (2 panels): 32 KiB for hi, 32 KiB for lo;
+//   TM: rows 0..63 T = (I + L)^-1, rows 64..127 M = scale P T, 64 columns:
+//       16 KiB for hi, 16 KiB for lo.
+constexpr uint32_t kImgKQ = 32768, kImgTM = 16384;
+constexpr uint32_t kImgBytes = 2 * kImgKQ + 2 * kImgTM;
+
+// Byte offset of (row, 8-column chunk c) in a 128-byte-swizzled panel.
+__host__ __device__ __forceinline__ uint32_t sw128_off(int row, int c) {
+  return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4));
+}
+
+// Eight floats as bf16 hi = bf16(x) and lo = bf16(x - hi) (round to nearest
+// even), each packed into 16 bytes.
+__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    h[i] = *reinterpret_cast<uint32_t*>(&b);
+    const float r0 = x[2 * i] - __uint_as_float(h[i] << 16);
+    const float r1 = x[2 * i + 1] - __uint_as_float(h[i] & 0xffff0000u);
+    __nv_bfloat162 c = __floats2bfloat162_rn(r0, r1);
+    l[i] = *reinterpret_cast<uint32_t*>(&c);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Rows of K^ and Q^ have pitch D + 4: a multiple of 4 (16-byte aligned rows)
@@ -197,7 +240,7 @@ __device__ __forceinline__ void gate_scan(float g, float beta, float* Gs, float*
 // One CTA per (stream, head, sub-chunk): T = (I + L)^-1 and M = scale P T of
 // the sub-chunk into the workspace, both [64][64] row-major, zero above the
 // diagonal.
-template <int D, typename T>
+template <int D, typename T, bool kImg>
 __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_constant__ GdnParams p) {
   using L = GdnPrepSmem<D>;
   constexpr int KP = L::KP;
@@ -217,6 +260,8 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_c
   const int64_t Tn = p.T;
   const int64_t t0 = (int64_t)j * kCt;
   const int n = (int)(Tn - t0 < kCt ? Tn - t0 : kCt);
+  // (block-uniform: the whole block leaves before any barrier)
+  if (!SA_BOUNDS(b >= 0 && b < p.batch && z < p.n_streams && j < p.n_sub && n > 0, 0)) return;
   const T* q = static_cast<const T*>(p.q);
   const T* k = static_cast<const T*>(p.k);
   const size_t tok_stride = (size_t)H * D;
@@ -231,6 +276,24 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_c
               Gs, Bs, tid, lane);
   }
   __syncthreads();
+  // the call's device status word starts at zero (the prep kernel runs first)
+  if (j == 0 && h == 0 && z == 0 && tid == 0) *reinterpret_cast<int*>(p.workspace) = 0;
+  const size_t blk = ((size_t)z * H + h) * (size_t)p.n_sub + (size_t)j;
+  unsigned char* img = reinterpret_cast<unsigned char*>(p.workspace) + kWsHeader + blk * kImgBytes;
+  if constexpr (kImg) {
+    // the KQ image (before the key and query rows are reused below)
+    if (SA_BOUNDS(blk < (size_t)p.n_streams * H * (size_t)p.n_sub, 1)) {
+      for (int e = tid; e < 2 * kCt * (D / 8); e += kGdnThreads) {
+        const int r = e / (D / 8), cc = e % (D / 8), panel = cc >> 3, c = cc & 7;
+        const float* src = (r < kCt ? Kh + r * KP : Qh + (r - kCt) * KP) + cc * 8;
+        uint4 hi, lo;
+        split8(src, hi, lo);
+        const uint32_t off = (uint32_t)panel * (kImgKQ / 2) + sw128_off(r, c);
+        *reinterpret_cast<uint4*>(img + off) = hi;
+        *reinterpret_cast<uint4*>(img + kImgKQ + off) = lo;
+      }
+    }
+  }
 
     // ---- Gram matrices on the lower triangle -> L and P. Thread (ty, tx)
     // takes rows ty + 16a and columns tx + 16b, b <= a (the pairs a < b lie
@@ -409,16 +472,35 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_c
   }
   __syncthreads();
 
-  // ---- T and M to the workspace, zero above the diagonal
-  float* dst = p.workspace + (((size_t)z * H + h) * (size_t)p.n_sub + (size_t)j) * kTpFloats;
-  for (int e = tid; e < 2 * kCt * (kCt / 4); e += kGdnThreads) {
-    const int mat = e / (kCt * (kCt / 4)), row = (e / (kCt / 4)) % kCt, c4 = (e % (kCt / 4)) * 4;
-    float4 x = ld4((mat ? Lm : Tm) + row * kLp + c4);
-    if (c4 + 0 > row) x.x = 0.f;
-    if (c4 + 1 > row) x.y = 0.f;
-    if (c4 + 2 > row) x.z = 0.f;
-    if (c4 + 3 > row) x.w = 0.f;
-    *reinterpret_cast<float4*>(dst + mat * kCt * kCt + row * kCt + c4) = x;
+  if constexpr (kImg) {
+    // ---- the TM image: T rows then M rows, zero above the diagonal
+    if (!SA_BOUNDS(blk < (size_t)p.n_streams * H * (size_t)p.n_sub, 1)) return;
+    for (int e = tid; e < 2 * kCt * (kCt / 8); e += kGdnThreads) {
+      const int r = e / (kCt / 8), c = e % (kCt / 8), row = r & (kCt - 1);
+      const float* src = (r < kCt ? Tm : Lm) + row * kLp + c * 8;
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = c * 8 + i <= row ? src[i] : 0.f;
+      uint4 hi, lo;
+      split8(x, hi, lo);
+      const uint32_t off = 2 * kImgKQ + sw128_off(r, c);
+      *reinterpret_cast<uint4*>(img + off) = hi;
+      *reinterpret_cast<uint4*>(img + kImgTM + off) = lo;
+    }
+  } else {
+    // ---- T and M to the workspace, zero above the diagonal
+    float* dst = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(p.workspace) + kWsHeader) +
+                 blk * kTpFloats;
+    if (!SA_BOUNDS(blk < (size_t)p.n_streams * H * (size_t)p.n_sub, 1)) return;
+    for (int e = tid; e < 2 * kCt * (kCt / 4); e += kGdnThreads) {
+      const int mat = e / (kCt * (kCt / 4)), row = (e / (kCt / 4)) % kCt, c4 = (e % (kCt / 4)) * 4;
+      float4 x = ld4((mat ? Lm : Tm) + row * kLp + c4);
+      if (c4 + 0 > row) x.x = 0.f;
+      if (c4 + 1 > row) x.y = 0.f;
+      if (c4 + 2 > row) x.z = 0.f;
+      if (c4 + 3 > row) x.w = 0.f;
+      *reinterpret_cast<float4*>(dst + mat * kCt * kCt + row * kCt + c4) = x;
+    }
   }
 }
 
@@ -456,6 +538,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
   const size_t bh0 = (size_t)b * (size_t)Tn * tok_stride + (size_t)h * D;   // (b, t=0, h, d=0)
   const size_t g0 = (size_t)b * (size_t)Tn * H + h;                           // (b, t=0, h)
   const int vcol = slice * kDvs;
+  // (block-uniform: the whole block leaves before any barrier)
+  if (!SA_BOUNDS(b >= 0 && b < p.batch && blockIdx.z < (unsigned)p.n_streams && vcol + kDvs <= D,
+                 3))
+    return;
   float* Sg = p.state + (((size_t)b * H + h) * D + vcol) * D;
 
   // Issues the copies of sub-chunk [t0, t0 + 64) into the staging area (rows
@@ -492,8 +578,12 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
 
   // Issues the copies of T and M = scale P T of sub-chunk j from the
   // workspace (written by gdn_prep_kernel) into Tm and Mm.
-  const float* wsp = p.workspace + ((size_t)blockIdx.z * H + h) * (size_t)p.n_sub * kTpFloats;
+  const float* wsp =
+      reinterpret_cast<const float*>(reinterpret_cast<const unsigned char*>(p.workspace) +
+                                     kWsHeader) +
+      ((size_t)blockIdx.z * H + h) * (size_t)p.n_sub * kTpFloats;
   auto prefetch_tp = [&](int64_t j) {
+    if (!SA_BOUNDS(j >= 0 && j < p.n_sub, 2)) j = 0;
     const float* src = wsp + (size_t)j * kTpFloats;
     for (int c = tid; c < 2 * kCt * (kCt / 4); c += kGdnThreads) {
       const int mat = c / (kCt * (kCt / 4)), row = (c / (kCt / 4)) % kCt, c4 = (c % (kCt / 4)) * 4;
@@ -535,6 +625,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
 
   for (int64_t t0 = 0; t0 < Tn; t0 += kCt) {
     const int n = (int)(Tn - t0 < kCt ? Tn - t0 : kCt);
+    (void)SA_BOUNDS(n > 0 && t0 / kCt < p.n_sub, 4);
     cp_async_wait_all();
     if (tid < kCt) gate_scan(gnext, bnext, Gs, Bs, tid, lane);   // warps 0 and 1
     __syncthreads();
@@ -678,31 +769,457 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
     for (int c = 0; c < NC; ++c) Sg[(size_t)(ur + i) * D + ucol + c] = sreg[i][c];
 }
 
+// ---------------------------------------------------------------- tensor-core sequential pass
+// D = 128. One CTA per (stream, head, 64 value dims of the state): 4 warps
+// for the elementwise work (thread r owns TMEM lane r) and 1 warp that issues
+// the copies and the tcgen05 MMAs. The state slice lives in TMEM, transposed
+// (lane = key dim k, column = value dim v: ST[k][v] = S[v][k]), for the whole
+// call. Per 64-token sub-chunk j, with its operand images from the prep
+// kernel (KQ, TM) arriving by bulk copy one or two sub-chunks ahead:
+//   MMA1  D1[t][v]      = sum_k [K^;Q^][t][k] S[v][k]       (K^ S0^T and Q^ S0^T)
+//   (threads) RHS[t][v] = beta_t (v_t[v] - e^{G_t} D1[t][v]); O_in = scale e^{G_t} D1[64+t][v]
+//   MMA2  D2[t][v]      = sum_s [T;M][t][s] RHS[s][v]      (U = T RHS and the intra-chunk outputs)
+//   (threads) U~[t][v]  = e^{G_last - G_t} D2[t][v]; out = O_in + D2[64+t]
+//   MMA3  ST[k][v]     += sum_t K^[t][k] U~[t][v]            (ST was scaled by e^{G_last})
+//   (threads) the S image of the new state for the next MMA1; ST *= e^{G_last} of j + 1
+// Every product is the three-term split product of bf16 operands:
+// x = hi + lo, a.b ~ a_hi.b_hi + a_hi.b_lo + a_lo.b_hi with fp32 accumulation
+// (about 2^-16 relative per product; a plain bf16 product has 2^-8). Images
+// written by the threads (S, RHS, U~) are 128-byte-swizzled rows of 64
+// values, read as MN-major operands; the K^ rows of KQ serve as the MN-major
+// A operand of MMA3. Every wait is bounded (about 1 s); on expiry the CTA
+// records a device error in the workspace header, drains and returns.
+struct GdnTcSmem {
+  static constexpr uint32_t kq = 0;                         // [2 buffers][hi, lo] KQ images
+  static constexpr uint32_t tm = 4 * kImgKQ;                // [hi, lo] TM image
+  static constexpr uint32_t st = tm + 2 * kImgTM;           // [hi, lo] S image, 128 x 64
+  static constexpr uint32_t rhs = st + 2 * 16384;           // [hi, lo] RHS image, 64 x 64
+  static constexpr uint32_t uu = rhs + 2 * 8192;            // [hi, lo] U~ image, 64 x 64
+  static constexpr uint32_t bars = uu + 2 * 8192;
+  static constexpr int B_KQ = 0, B_TM = 2, B_S = 3, B_D1 = 4, B_RHS = 5, B_D2 = 6, B_U = 7,
+                       B_D3 = 8, B_G = 9, B_DR = 10;
+  static constexpr int kNumBars = 11;
+  static constexpr uint32_t misc = bars + kNumBars * 8;     // TMEM base, abort flags
+  static constexpr uint32_t gs = misc + 16;                 // [2][64] gate prefix sums (log2)
+  static constexpr uint32_t bs = gs + 2 * kCt * 4;          // [2][64] beta
+  static constexpr uint32_t bytes = bs + 2 * kCt * 4;
+  static_assert(bytes <= 232448, "exceeds 227 KB of shared memory per CTA");
+};
+constexpr int kTcThreads = 160;
+constexpr int kTcSlice = 64;
+constexpr uint64_t kTcTimeoutNs = 1000000000ull;
+
+// Row `row` (64 floats) of a single-panel image as bf16 hi and lo.
+__device__ __forceinline__ void put_row64(unsigned char* sm, uint32_t hi_off, uint32_t lo_off,
+                                          int row, const float* x) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 h, l;
+    split8(x + 8 * c, h, l);
+    const uint32_t off = sw128_off(row, c);
+    *reinterpret_cast<uint4*>(sm + hi_off + off) = h;
+    *reinterpret_cast<uint4*>(sm + lo_off + off) = l;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void load64(const T* src, float* x) {
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 u = *reinterpret_cast<const uint4*>(src + 8 * i);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        x[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+        x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float4 u = *reinterpret_cast<const float4*>(src + 4 * i);
+      x[4 * i] = u.x, x[4 * i + 1] = u.y, x[4 * i + 2] = u.z, x[4 * i + 3] = u.w;
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store64(T* dst, const float* x) {
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(x[8 * i + 2 * k], x[8 * i + 2 * k + 1]);
+        w[k] = *reinterpret_cast<uint32_t*>(&b);
+      }
+      *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      *reinterpret_cast<float4*>(dst + 4 * i) =
+          make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_constant__ GdnParams p) {
+  constexpr int D = 128;
+  using L = GdnTcSmem;
+  extern __shared__ __align__(1024) unsigned char smc[];
+  int* status = reinterpret_cast<int*>(p.workspace);
+  const uint32_t base = ptx::smem_u32(smc);
+  if (base & 1023u) {  // 128-byte-swizzled images need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(status, kDeviceErrTimeout);
+    return;
+  }
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int slice = blockIdx.x, h = blockIdx.y, z = blockIdx.z, b = p.stream_of[z];
+  const int H = p.H;
+  const int64_t Tn = p.T;
+  const int nsub = p.n_sub;
+  const int vcol = slice * kTcSlice;
+  const uint32_t bar0 = base + L::bars;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smc + L::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smc + L::misc + 4);
+  volatile int* no_abort = reinterpret_cast<volatile int*>(smc + L::misc + 8);
+  float* Gs = reinterpret_cast<float*>(smc + L::gs);
+  float* Bs = reinterpret_cast<float*>(smc + L::bs);
+  if (!SA_BOUNDS(b >= 0 && b < p.batch && z < p.n_streams && vcol + kTcSlice <= D, 3)) return;
+
+  if (tid == 0) {
+    ptx::mbar_init(bar(L::B_KQ), 1);
+    ptx::mbar_init(bar(L::B_KQ + 1), 1);
+    ptx::mbar_init(bar(L::B_TM), 1);
+    ptx::mbar_init(bar(L::B_S), 128);
+    ptx::mbar_init(bar(L::B_D1), 1);
+    ptx::mbar_init(bar(L::B_RHS), 128);
+    ptx::mbar_init(bar(L::B_D2), 1);
+    ptx::mbar_init(bar(L::B_U), 128);
+    ptx::mbar_init(bar(L::B_D3), 1);
+    ptx::mbar_init(bar(L::B_G), 64);
+    ptx::mbar_init(bar(L::B_DR), 1);
+    *abort_flag = 0;
+    *no_abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 4) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 256);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_st = tmem, t_d1 = tmem + 64, t_d2 = tmem + 128;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicOr(status, kDeviceErrTimeout);
+  };
+  const unsigned char* images = reinterpret_cast<const unsigned char*>(p.workspace) + kWsHeader +
+                                ((size_t)z * H + h) * (size_t)nsub * kImgBytes;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ copies + MMA issue
+    if (lane == 0) {
+      auto load_kq = [&](int j) {
+        const uint32_t dst = base + L::kq + (uint32_t)(j & 1) * 2 * kImgKQ;
+        const unsigned char* src = images + (size_t)j * kImgBytes;
+        ptx::mbar_arrive_expect_tx(bar(L::B_KQ + (j & 1)), 2 * kImgKQ);
+        for (uint32_t o = 0; o < 2 * kImgKQ; o += 16384)
+          ptx::bulk_g2s(dst + o, src + o, 16384, bar(L::B_KQ + (j & 1)));
+      };
+      auto load_tm = [&](int j) {
+        const unsigned char* src = images + (size_t)j * kImgBytes + 2 * kImgKQ;
+        ptx::mbar_arrive_expect_tx(bar(L::B_TM), 2 * kImgTM);
+        for (uint32_t o = 0; o < 2 * kImgTM; o += 16384)
+          ptx::bulk_g2s(base + L::tm + o, src + o, 16384, bar(L::B_TM));
+      };
+      constexpr uint32_t id_kk = ptx::idesc_bf16_f32_ab(128, kTcSlice, false, true);
+      constexpr uint32_t id_mm = ptx::idesc_bf16_f32_ab(128, kTcSlice, true, true);
+      // split-product term i: (A part, B part) = (hi, hi), (hi, lo), (lo, hi)
+      constexpr uint32_t ta[3] = {0, 0, 1}, tb[3] = {0, 1, 0};
+      int kq_issued = 0, kq_done = 0, tm_issued = 0;
+      load_kq(0);
+      ++kq_issued;
+      if (nsub > 1) {
+        load_kq(1);
+        ++kq_issued;
+      }
+      load_tm(0);
+      ++tm_issued;
+      bool ok = true;
+      for (int j = 0; ok && j < nsub; ++j) {
+        const uint32_t par = (uint32_t)j & 1;
+        const uint32_t kqb = base + L::kq + (uint32_t)(j & 1) * 2 * kImgKQ;
+        if (!ptx::mbar_wait(bar(L::B_KQ + (j & 1)), (uint32_t)(j >> 1) & 1, abort_flag, kTcTimeoutNs) ||
+            !ptx::mbar_wait(bar(L::B_S), par, abort_flag, kTcTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        ++kq_done;
+        ptx::tc_fence_after();
+        // MMA1: [K^;Q^] (K-major, 2 panels of 64 key dims) x S image (MN-major)
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = ptx::sdesc_sw128(kqb + ta[i] * kImgKQ + (uint32_t)(kk >> 2) * 16384 +
+                                                    (uint32_t)(kk & 3) * 32, 16, 1024);
+            const uint64_t bd =
+                ptx::sdesc_sw128(base + L::st + tb[i] * 16384 + (uint32_t)kk * 2048, 16384, 1024);
+            ptx::umma_ss(t_d1, a, bd, id_kk, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+        ptx::umma_commit(bar(L::B_D1));
+        if (!ptx::mbar_wait(bar(L::B_TM), par, abort_flag, kTcTimeoutNs) ||
+            !ptx::mbar_wait(bar(L::B_RHS), par, abort_flag, kTcTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        // MMA2: [T;M] (K-major, one panel of 64 tokens) x RHS image (MN-major)
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+#pragma unroll
+          for (int kk = 0; kk < kCt / 16; ++kk) {
+            const uint64_t a =
+                ptx::sdesc_sw128(base + L::tm + ta[i] * kImgTM + (uint32_t)kk * 32, 16, 1024);
+            const uint64_t bd =
+                ptx::sdesc_sw128(base + L::rhs + tb[i] * 8192 + (uint32_t)kk * 2048, 16384, 1024);
+            ptx::umma_ss(t_d2, a, bd, id_kk, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+        ptx::umma_commit(bar(L::B_D2));
+        // the TM buffer is free once MMA2 has read it
+        if (!ptx::mbar_wait(bar(L::B_D2), par, abort_flag, kTcTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        if (j + 1 < nsub) {
+          load_tm(j + 1);
+          ++tm_issued;
+        }
+        if (!ptx::mbar_wait(bar(L::B_U), par, abort_flag, kTcTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        // MMA3: ST += K^ (the key rows of KQ as the MN-major A: 2 panels of 64
+        // key dims LBO apart, 64 token rows) x U~ image (MN-major)
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+#pragma unroll
+          for (int kk = 0; kk < kCt / 16; ++kk) {
+            const uint64_t a =
+                ptx::sdesc_sw128(kqb + ta[i] * kImgKQ + (uint32_t)kk * 2048, 16384, 1024);
+            const uint64_t bd =
+                ptx::sdesc_sw128(base + L::uu + tb[i] * 8192 + (uint32_t)kk * 2048, 16384, 1024);
+            ptx::umma_ss(t_st, a, bd, id_mm, 1u);
+          }
+        ptx::umma_commit(bar(L::B_D3));
+        // the KQ buffer of j is free once MMA3 has read it
+        if (j + 2 < nsub) {
+          if (!ptx::mbar_wait(bar(L::B_D3), par, abort_flag, kTcTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          load_kq(j + 2);
+          ++kq_issued;
+        }
+      }
+      if (!ok) fail();
+      // drain: the copies this thread issued have landed and its MMAs are done
+      for (int jj = kq_done; jj < kq_issued; ++jj)
+        ptx::mbar_wait(bar(L::B_KQ + (jj & 1)), (uint32_t)(jj >> 1) & 1, no_abort, kTcTimeoutNs);
+      if (tm_issued > 0)
+        ptx::mbar_wait(bar(L::B_TM), (uint32_t)(tm_issued - 1) & 1, no_abort, kTcTimeoutNs);
+      ptx::umma_commit(bar(L::B_DR));
+      ptx::mbar_wait(bar(L::B_DR), 0, no_abort, kTcTimeoutNs);
+    }
+  } else {
+    // ------------------------------------------------------------ elementwise (TMEM lane = tid)
+    const int r = tid;  // 0..63: key/U rows, 64..127: query/output rows; also key dim r of ST
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const T* v = static_cast<const T*>(p.v);
+    T* out = static_cast<T*>(p.out);
+    const size_t tok_stride = (size_t)H * D;
+    const size_t bh0 = (size_t)b * (size_t)Tn * tok_stride + (size_t)h * D + vcol;
+    const size_t g0 = (size_t)b * (size_t)Tn * H + h;
+    float* Sg = p.state + ((size_t)b * H + h) * D * D;   // [v][k]
+    auto gates = [&](int j) {
+      // threads 0..63: prefix sums of g log2(e) and beta of sub-chunk j
+      if (r < kCt) {
+        const int64_t t = (int64_t)j * kCt + r;
+        const bool in = t < Tn;
+        gate_scan(in ? p.g[g0 + (size_t)t * H] : 0.f, in ? p.beta[g0 + (size_t)t * H] : 0.f,
+                  Gs + (j & 1) * kCt, Bs + (j & 1) * kCt, r, lane);
+        ptx::mbar_arrive(bar(L::B_G));
+      }
+    };
+    auto gcum = [&](int j, int t) -> float {
+      const float* G = Gs + (j & 1) * kCt;
+      return G[t] + (t >= 32 ? G[31] : 0.f);
+    };
+    bool ok = true;
+    // prologue: the gates of sub-chunk 0, the S image of the initial state and
+    // ST = e^{G_last} S
+    gates(0);
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_G), 0, abort_flag, kTcTimeoutNs))) ok = false;
+    if (ok) {
+      float x[kTcSlice];
+#pragma unroll
+      for (int i = 0; i < kTcSlice; ++i) x[i] = Sg[(size_t)(vcol + i) * D + r];
+      put_row64(smc, L::st, L::st + 16384, r, x);
+      const float dec = ptx::ex2(gcum(0, kCt - 1));
+#pragma unroll
+      for (int i = 0; i < kTcSlice; ++i) x[i] *= dec;
+      ptx::tmem_st32(t_st + lane_off, x);
+      ptx::tmem_st32(t_st + lane_off + 32, x + 32);
+      ptx::tmem_wait_st();
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(L::B_S));
+    }
+    for (int j = 0; ok && j < nsub; ++j) {
+      const uint32_t par = (uint32_t)j & 1;
+      const int64_t t0 = (int64_t)j * kCt;
+      const int tr = r & (kCt - 1);               // token of this row
+      const bool tok_in = t0 + tr < Tn;
+      // values of this sub-chunk's token (key rows), loaded while MMA1 runs
+      float vv[kTcSlice];
+      if (r < kCt) {
+        if (tok_in) {
+          load64(v + bh0 + (size_t)(t0 + tr) * tok_stride, vv);
+        } else {
+#pragma unroll
+          for (int i = 0; i < kTcSlice; ++i) vv[i] = 0.f;
+        }
+      }
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_D1), par, abort_flag, kTcTimeoutNs))) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      float x[kTcSlice];
+      ptx::tmem_ld32(t_d1 + lane_off, x);
+      ptx::tmem_ld32(t_d1 + lane_off + 32, x + 32);
+      ptx::tmem_wait_ld();
+      const float eg = ptx::ex2(gcum(j, tr));
+      if (r < kCt) {
+        const float bt = Bs[(j & 1) * kCt + tr];
+#pragma unroll
+        for (int i = 0; i < kTcSlice; ++i) vv[i] = bt * (vv[i] - eg * x[i]);
+        put_row64(smc, L::rhs, L::rhs + 8192, tr, vv);
+      } else {
+        const float sc = p.scale * eg;
+#pragma unroll
+        for (int i = 0; i < kTcSlice; ++i) vv[i] = sc * x[i];   // (query rows: the inter-chunk output)
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(L::B_RHS));
+      // the gates of the next sub-chunk, while MMA2 runs
+      if (j + 1 < nsub) gates(j + 1);
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_D2), par, abort_flag, kTcTimeoutNs))) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      ptx::tmem_ld32(t_d2 + lane_off, x);
+      ptx::tmem_ld32(t_d2 + lane_off + 32, x + 32);
+      ptx::tmem_wait_ld();
+      if (r < kCt) {
+        const float wt = ptx::ex2(gcum(j, kCt - 1) - gcum(j, tr));
+#pragma unroll
+        for (int i = 0; i < kTcSlice; ++i) x[i] *= wt;
+        put_row64(smc, L::uu, L::uu + 8192, tr, x);
+      } else if (tok_in) {
+#pragma unroll
+        for (int i = 0; i < kTcSlice; ++i) x[i] += vv[i];
+        store64(out + bh0 + (size_t)(t0 + tr) * tok_stride, x);
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(L::B_U));
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_D3), par, abort_flag, kTcTimeoutNs))) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      // the state after sub-chunk j (key dim r, 64 value dims)
+      ptx::tmem_ld32(t_st + lane_off, x);
+      ptx::tmem_ld32(t_st + lane_off + 32, x + 32);
+      ptx::tmem_wait_ld();
+      if (j + 1 < nsub) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_G), (uint32_t)(j + 1) & 1, abort_flag,
+                                                    kTcTimeoutNs))) {
+          ok = false;
+          break;
+        }
+        put_row64(smc, L::st, L::st + 16384, r, x);
+        const float dec = ptx::ex2(gcum(j + 1, kCt - 1));
+#pragma unroll
+        for (int i = 0; i < kTcSlice; ++i) x[i] *= dec;
+        ptx::tmem_st32(t_st + lane_off, x);
+        ptx::tmem_st32(t_st + lane_off + 32, x + 32);
+        ptx::tmem_wait_st();
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(L::B_S));
+      } else {
+#pragma unroll
+        for (int i = 0; i < kTcSlice; ++i) Sg[(size_t)(vcol + i) * D + r] = x[i];
+      }
+    }
+    if (!ok) fail();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 4) ptx::tmem_dealloc(tmem, 256);
+}
+
+// D = 128: the prep kernel writes the operand images and the tensor-core
+// kernel runs the sequential pass; D = 64: fp32 T and M and the CUDA-core
+// sequential kernel.
 template <int D, typename T>
 cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
-  constexpr size_t smem = GdnSmem<D, T>::bytes;
+  constexpr bool kTc = D == 128;
+  constexpr size_t smem = kTc ? GdnTcSmem::bytes : GdnSmem<D, T>::bytes;
   constexpr size_t psmem = GdnPrepSmem<D>::bytes;
   static unsigned configured = 0;   // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 32 || !(configured & (1u << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(gdn_chunk_kernel<D, T>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e;
+    if constexpr (kTc)
+      e = cudaFuncSetAttribute(gdn_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+    else
+      e = cudaFuncSetAttribute(gdn_chunk_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gdn_prep_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)psmem);
+      e = cudaFuncSetAttribute(gdn_prep_kernel<D, T, kTc>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
     if (e != cudaSuccess) return e;
     if (dev < 32) configured |= 1u << dev;
   }
-  gdn_prep_kernel<D, T><<<dim3(p.n_sub, p.H, p.n_streams), kGdnThreads, psmem, st>>>(p);
-  gdn_chunk_kernel<D, T><<<dim3(D / kDvs, p.H, p.n_streams), kGdnThreads, smem, st>>>(p);
+  gdn_prep_kernel<D, T, kTc><<<dim3(p.n_sub, p.H, p.n_streams), kGdnThreads, psmem, st>>>(p);
+  if constexpr (kTc)
+    gdn_tc_kernel<T><<<dim3(D / kTcSlice, p.H, p.n_streams), kTcThreads, smem, st>>>(p);
+  else
+    gdn_chunk_kernel<D, T><<<dim3(D / kDvs, p.H, p.n_streams), kGdnThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t gdn_workspace_bytes(int B, int H, int64_t T) {
-  return (size_t)B * (size_t)H * (size_t)((T + kCt - 1) / kCt) * kTpFloats * sizeof(float);
+size_t gdn_workspace_bytes(int B, int H, int D, int64_t T) {
+  const size_t per = D == 128 ? (size_t)kImgBytes : (size_t)kTpFloats * sizeof(float);
+  return kWsHeader + (size_t)B * (size_t)H * (size_t)((T + kCt - 1) / kCt) * per;
 }
 
 size_t gdn_smem_bytes(int D, int dtype) {

@@ -18,6 +18,49 @@ constexpr int kMaxDt2 = 64;       // d_t / 2 <= 64
 constexpr int kMaxAttnStreams = SA_MAX_STREAMS;
 constexpr int kDeviceErrTimeout = 1;
 
+// Debug build (compiled with -DSA_DEBUG_BOUNDS, libsa_debug.so): every
+// computed index into a buffer (cache rows, partial-result slots, arrival
+// counters, workspace offsets, TMA tile coordinates) is range-checked before
+// the access. A violation sets bit `site` of the source file's bounds word
+// and the access is skipped (a store) or replaced (a load reads zero, a tile
+// coordinate is clamped to 0), so the kernel still ends normally; no trap,
+// no fault. sa_debug_bounds_status reads and clears the words. In the normal
+// build SA_BOUNDS(ok, site) is `true` and costs nothing.
+#ifdef SA_DEBUG_BOUNDS
+#define SA_BOUNDS(ok, site) sa_bounds_ok_((ok), (site))
+// one word per source file (no relocatable device code: each .cu file keeps
+// its own word and host reader, named by the file)
+#define SA_DEFINE_BOUNDS_WORD(reader)                                                 \
+  static __device__ unsigned int g_sa_bounds_word;                                    \
+  static __device__ __forceinline__ bool sa_bounds_ok_(bool ok, int site) {           \
+    if (!ok) atomicOr(&g_sa_bounds_word, 1u << site);                                 \
+    return ok;                                                                        \
+  }                                                                                   \
+  cudaError_t reader(unsigned int* word, cudaStream_t st) {                           \
+    unsigned int w = 0, z = 0;                                                        \
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&w, g_sa_bounds_word, sizeof(w), 0,     \
+                                              cudaMemcpyDeviceToHost, st);            \
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);                              \
+    if (e == cudaSuccess && w)                                                        \
+      e = cudaMemcpyToSymbolAsync(g_sa_bounds_word, &z, sizeof(z), 0,                 \
+                                  cudaMemcpyHostToDevice, st);                        \
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);                              \
+    *word = w;                                                                        \
+    return e;                                                                         \
+  }
+#else
+#define SA_BOUNDS(ok, site) true
+#define SA_DEFINE_BOUNDS_WORD(reader)
+#endif
+// Host readers of the per-file bounds words (debug build only).
+cudaError_t bounds_word_attend_tc(unsigned int* word, cudaStream_t st);
+cudaError_t bounds_word_attend_simt(unsigned int* word, cudaStream_t st);
+cudaError_t bounds_word_rope_append(unsigned int* word, cudaStream_t st);
+cudaError_t bounds_word_gdn(unsigned int* word, cudaStream_t st);
+// Debug build: one thread records a check failure at site 31 of the
+// attention file's word without touching memory (shows the recording path).
+cudaError_t bounds_selftest(cudaStream_t st);
+
 // Fused 3D-RoPE + append (one launch covers up to kMaxEntries (stream, frame)
 // entries; entry e = a*C + i is frame i of the a-th stream of the launch).
 struct AppendParams {
@@ -34,6 +77,7 @@ struct AppendParams {
   int64_t ntok, sf;    // cache rows per (b, h); sink rows per (b, h)
   int32_t dt2, dh2, dw2;
   int32_t n_streams;   // streams in this launch
+  int32_t batch;       // B (the extent of q, k, v and the caches; bounds checks)
   const float* fp8_scale;  // e4m3 cache: [3][H] per-head scales of q, k, v (device)
   int32_t stream_of[kMaxEntries];
   int64_t dest_row[kMaxEntries];   // cache row of the frame's first token
@@ -61,6 +105,7 @@ struct RefreshParams {
   int64_t ntok, sf;
   int32_t dt2, dh2, dw2;
   int32_t n_streams;
+  int32_t batch;       // B (bounds checks)
   int32_t stream_of[kMaxRefresh];
   int64_t ring_rows[kMaxRefresh];    // valid ring rows of the stream
   int64_t sink_rows[kMaxRefresh];    // valid sink rows of the stream
@@ -82,6 +127,7 @@ struct AttnParams {
   const void* v_cache; // (SIMT path)
   int* status;
   int32_t fp8;         // e4m3 operands (SA_BF16_E4M3)
+  int32_t batch;       // B (bounds checks)
   int32_t stream_of[kMaxAttnStreams];
   int32_t n_keys[kMaxAttnStreams];
   float inv_qk[kMaxF8Heads];  // e4m3: 1 / (q_scale * k_scale) per head
@@ -98,8 +144,11 @@ size_t attend_partials_bytes(int D, int num_sms, int64_t max_units);
 
 // Gated DeltaNet block (gdn.cu): T tokens of each listed stream; q, k, v, out
 // [B][T][H][D], g and beta [B][T][H], state [B][H][D][D] fp32 in place.
-// workspace: T and P of every (listed stream, head, 64-token sub-chunk),
-// gdn_workspace_bytes(n_streams, H, T) bytes, 16-byte aligned.
+// workspace: a 1 KiB header (device status word of the tensor-core path),
+// then per (listed stream, head, 64-token sub-chunk) the prep kernel's
+// output (D = 128: the bf16 hi/lo operand images of the sequential
+// tensor-core kernel; D = 64: fp32 T and M); gdn_workspace_bytes(n_streams,
+// H, D, T) bytes, 16-byte aligned.
 struct GdnParams {
   float* state;
   const void* q;
@@ -114,9 +163,10 @@ struct GdnParams {
   float scale;
   int32_t n_streams;
   int32_t n_sub;       // ceil(T / 64)
+  int32_t batch;       // B (bounds checks)
   int32_t stream_of[SA_MAX_STREAMS];
 };
-size_t gdn_workspace_bytes(int B, int H, int64_t T);
+size_t gdn_workspace_bytes(int B, int H, int D, int64_t T);
 size_t gdn_smem_bytes(int D, int dtype);
 cudaError_t launch_gdn(const GdnParams& p, int D, int dtype, cudaStream_t st);
 

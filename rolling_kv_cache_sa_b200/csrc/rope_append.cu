@@ -18,6 +18,12 @@
 #include "ptx.cuh"
 
 namespace sa {
+
+// debug build: the bounds word of this file (sites: 0 input vector, 1 cache
+// row of an appended frame, 2 raw-sink row, 3 rotated-query row, 4 ring row of
+// a refresh, 5 sink row of a refresh or sink update)
+SA_DEFINE_BOUNDS_WORD(bounds_word_rope_append)
+
 namespace {
 
 template <typename T>
@@ -119,11 +125,17 @@ __global__ void __launch_bounds__(256) append_rope_kernel(const __grid_constant_
     const int e = (int)a * p.C + fi;
 
     const int64_t in_off = (((int64_t)b * p.Lc + tok) * p.H + h) * p.D + (int64_t)vc * N;
+    const int64_t bh = (int64_t)b * p.H + h;
+    if (!SA_BOUNDS(b >= 0 && b < p.batch && e < kMaxEntries, 0) ||
+        !SA_BOUNDS(tok < (uint32_t)p.Lc && a < (uint32_t)p.n_streams, 3))
+      continue;
+    const int64_t row = p.dest_row[e] + j;
+    if (!SA_BOUNDS(row >= 0 && row < p.ntok, 1) ||
+        !SA_BOUNDS(p.raw_row[e] < 0 || p.raw_row[e] + j < p.sf, 2))
+      continue;
     float q[N], k[N];
     V::load(static_cast<const char*>(p.q) + in_off * esz, q);
     V::load(static_cast<const char*>(p.k) + in_off * esz, k);
-    const int64_t bh = (int64_t)b * p.H + h;
-    const int64_t row = p.dest_row[e] + j;
     const int64_t cache_off = (bh * p.ntok + row) * p.D + (int64_t)vc * N;
     V::copy(static_cast<char*>(p.v_cache) + cache_off * esz,
             static_cast<const char*>(p.v) + in_off * esz);
@@ -168,6 +180,7 @@ __global__ void __launch_bounds__(256) refresh_kernel(const __grid_constant__ Re
       const int64_t h = i / per_h;
       const int64_t rr = (i - h * per_h) / nvt;
       const int64_t vc = i - h * per_h - rr * nvt;
+      if (!SA_BOUNDS(b >= 0 && b < p.batch && p.sf + rr < p.ntok && vc < nvec, 4)) continue;
       const int64_t off = (((int64_t)b * p.H + h) * p.ntok + p.sf + rr) * p.D + vc * N;
       char* ptr = static_cast<char*>(p.k_cache) + off * esz;
       float k[N];
@@ -188,6 +201,7 @@ __global__ void __launch_bounds__(256) refresh_kernel(const __grid_constant__ Re
       const int s = (int)(rr / p.F);
       const int j = (int)(rr - (int64_t)s * p.F);
       const int y = j / p.fw, x = j - (j / p.fw) * p.fw;
+      if (!SA_BOUNDS(b >= 0 && b < p.batch && rr < p.sf && s < p.S, 5)) continue;
       float k[N];
       char* raw = static_cast<char*>(p.k_raw) + ((bh * p.sf + rr) * p.D + vc * N) * esz;
       V::load_cache(raw, k);
@@ -264,12 +278,18 @@ __global__ void __launch_bounds__(256) append_rope_e4m3_kernel(const __grid_cons
     const int y = j / p.fw, x = j - (j / p.fw) * p.fw;
     const int e = (int)a * p.C + fi;
     const int64_t in_off = (((int64_t)b * p.Lc + tok) * p.H + h) * p.D + (int64_t)vc * N;
+    const int64_t bh = (int64_t)b * p.H + h;
+    if (!SA_BOUNDS(b >= 0 && b < p.batch && e < kMaxEntries, 0) ||
+        !SA_BOUNDS(tok < (uint32_t)p.Lc && a < (uint32_t)p.n_streams, 3))
+      continue;
+    const int64_t row = p.dest_row[e] + j;
+    if (!SA_BOUNDS(row >= 0 && row < p.ntok, 1) ||
+        !SA_BOUNDS(p.raw_row[e] < 0 || p.raw_row[e] + j < p.sf, 2))
+      continue;
     float q[N], k[N], v[N];
     V::load(static_cast<const char*>(p.q) + in_off * 2, q);
     V::load(static_cast<const char*>(p.k) + in_off * 2, k);
     V::load(static_cast<const char*>(p.v) + in_off * 2, v);
-    const int64_t bh = (int64_t)b * p.H + h;
-    const int64_t row = p.dest_row[e] + j;
     const int64_t cache_off = (bh * p.ntok + row) * p.D + (int64_t)vc * N;
     const float sq = __ldg(&p.fp8_scale[h]), sk = __ldg(&p.fp8_scale[p.H + h]),
                 sv = __ldg(&p.fp8_scale[2 * p.H + h]);
@@ -312,6 +332,7 @@ __global__ void __launch_bounds__(256) refresh_e4m3_kernel(const __grid_constant
       const int64_t h = i / per_h;
       const int64_t rr = (i - h * per_h) / nvt;
       const int64_t vc = i - h * per_h - rr * nvt;
+      if (!SA_BOUNDS(b >= 0 && b < p.batch && p.sf + rr < p.ntok && vc < nvec, 4)) continue;
       const int64_t off = (((int64_t)b * p.H + h) * p.ntok + p.sf + rr) * p.D + vc * N;
       uint2* ptr = reinterpret_cast<uint2*>(static_cast<char*>(p.k_cache) + off);
       const float sk = __ldg(&p.fp8_scale[p.H + h]);
@@ -333,6 +354,7 @@ __global__ void __launch_bounds__(256) refresh_e4m3_kernel(const __grid_constant
       const int s = (int)(rr / p.F);
       const int j = (int)(rr - (int64_t)s * p.F);
       const int y = j / p.fw, x = j - (j / p.fw) * p.fw;
+      if (!SA_BOUNDS(b >= 0 && b < p.batch && rr < p.sf && s < p.S, 5)) continue;
       const float sk = __ldg(&p.fp8_scale[p.H + h]);
       float k[N];
       char* raw = static_cast<char*>(p.k_raw) + ((bh * p.sf + rr) * p.D + vc * N) * 2;

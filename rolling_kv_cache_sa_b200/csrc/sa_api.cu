@@ -347,7 +347,7 @@ sa_status sa_gdn_workspace_size(const sa_gdn_config* cfg, size_t* bytes) {
   sa_status st = validate_gdn_config(cfg);
   if (st != SA_OK) return st;
   if (!bytes) return fail(SA_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = sa::gdn_workspace_bytes(cfg->batch, cfg->heads, cfg->tokens);
+  *bytes = sa::gdn_workspace_bytes(cfg->batch, cfg->heads, cfg->head_dim, cfg->tokens);
   return SA_OK;
 }
 
@@ -367,10 +367,10 @@ sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, co
     const uintptr_t ptrs[3] = {(uintptr_t)q, (uintptr_t)k, (uintptr_t)v};
     for (uintptr_t a : ptrs)
       if (a % 16) return fail(SA_ERR_INVALID_ARG, "q, k and v must be 16-byte aligned");
-    if ((uintptr_t)out % esz) return fail(SA_ERR_INVALID_ARG, "out must be aligned to its element");
+    if ((uintptr_t)out % 16) return fail(SA_ERR_INVALID_ARG, "out must be 16-byte aligned");
     if ((uintptr_t)g % 4 || (uintptr_t)beta % 4)
       return fail(SA_ERR_INVALID_ARG, "g and beta must be 4-byte aligned");
-    const size_t need = sa::gdn_workspace_bytes(cfg->batch, cfg->heads, cfg->tokens);
+    const size_t need = sa::gdn_workspace_bytes(cfg->batch, cfg->heads, cfg->head_dim, cfg->tokens);
     if (!workspace || (uintptr_t)workspace % 16)
       return fail(SA_ERR_INVALID_ARG, "workspace must be non-NULL and 16-byte aligned");
     if (workspace_bytes < need)
@@ -401,11 +401,26 @@ sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, co
   p.workspace = static_cast<float*>(workspace);
   p.T = cfg->tokens;
   p.n_sub = (int32_t)((cfg->tokens + 63) / 64);
+  p.batch = cfg->batch;
   p.H = cfg->heads;
   p.scale = cfg->scale > 0.f ? cfg->scale : (float)(1.0 / sqrt((double)cfg->head_dim));
   NvtxRange nv("sa_gdn_chunk");
   e = sa::launch_gdn(p, cfg->head_dim, cfg->dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "gdn launch");
+  return SA_OK;
+}
+
+sa_status sa_gdn_device_status(const void* workspace, sa_stream_t stream) {
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 16)
+    return fail(SA_ERR_INVALID_ARG, "workspace must be non-NULL and 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "gdn status read");
+  if (word & sa::kDeviceErrTimeout)
+    return fail(SA_ERR_DEVICE_TIMEOUT, "a bounded wait of the last sa_gdn_chunk call gave up; its "
+                                       "outputs and state are not valid");
   return SA_OK;
 }
 
@@ -619,6 +634,7 @@ sa_status append_attend(sa_cache* h, const void* q, const void* k, const void* v
     p.dt2 = dt2; p.dh2 = c.rope_dims[1] / 2; p.dw2 = c.rope_dims[2] / 2;
     const size_t n = std::min(act.size() - s0, (size_t)per_launch);
     p.n_streams = (int32_t)n;
+    p.batch = c.batch;
     for (size_t a = 0; a < n; ++a) {
       const sa_chunk_plan& pl = plans[s0 + a];
       p.stream_of[a] = act[s0 + a];
@@ -649,6 +665,7 @@ sa_status append_attend(sa_cache* h, const void* q, const void* k, const void* v
   ap.H = c.heads; ap.Lc = (int32_t)h->Lc; ap.ntok = h->ntok;
   ap.n_q_tiles = (int32_t)((h->Lc + 127) / 128);
   ap.n_streams = (int32_t)act.size();
+  ap.batch = c.batch;
   ap.scale_log2 = (float)((double)h->scale * 1.4426950408889634);
   ap.out = out; ap.q_ws = h->q_ws; ap.k_cache = h->k_cache; ap.v_cache = h->v_cache;
   ap.status = h->d_status;
@@ -716,6 +733,7 @@ sa_status sa_rope_refresh(sa_cache* h, const uint8_t* active, sa_stream_t stream
     p.dt2 = dt2; p.dh2 = c.rope_dims[1] / 2; p.dw2 = c.rope_dims[2] / 2;
     const size_t n = std::min(todo.size() - s0, (size_t)per_launch);
     p.n_streams = (int32_t)n;
+    p.batch = c.batch;
     for (size_t a = 0; a < n; ++a) {
       const int b = todo[s0 + a];
       const int64_t fw_ = h->frames_written[b];
@@ -822,6 +840,7 @@ sa_status sa_sink_update(sa_cache* h, const void* k_new, const void* v_new, floa
     p.dt2 = dt2; p.dh2 = c.rope_dims[1] / 2; p.dw2 = c.rope_dims[2] / 2;
     const size_t n = std::min(act.size() - s0, (size_t)per_launch);
     p.n_streams = (int32_t)n;
+    p.batch = c.batch;
     for (size_t a = 0; a < n; ++a) {
       const int b = act[s0 + a];
       p.stream_of[a] = b;
@@ -1098,6 +1117,47 @@ sa_status sa_get_device_status(sa_cache* h, sa_stream_t stream) {
   return SA_OK;
 }
 
+sa_status sa_debug_bounds_status(sa_stream_t stream) {
+#ifdef SA_DEBUG_BOUNDS
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  struct {
+    const char* file;
+    cudaError_t (*read)(unsigned int*, cudaStream_t);
+  } words[] = {{"attend_tc", sa::bounds_word_attend_tc},
+               {"attend_simt", sa::bounds_word_attend_simt},
+               {"rope_append", sa::bounds_word_rope_append},
+               {"gdn", sa::bounds_word_gdn}};
+  std::string bad;
+  for (const auto& w : words) {
+    unsigned int word = 0;
+    cudaError_t e = w.read(&word, st);
+    if (e != cudaSuccess) return cuda_fail(e, "bounds word read");
+    if (word) {
+      char buf[96];
+      snprintf(buf, sizeof(buf), "%s%s sites 0x%08x", bad.empty() ? "" : ", ", w.file, word);
+      bad += buf;
+    }
+  }
+  if (!bad.empty())
+    return fail(SA_ERR_DEVICE_BOUNDS, "index checks failed in kernels: %s", bad.c_str());
+  return SA_OK;
+#else
+  (void)stream;
+  return fail(SA_ERR_UNSUPPORTED, "not a debug build (libsa_debug.so has the index checks)");
+#endif
+}
+
+sa_status sa_debug_bounds_selftest(sa_stream_t stream) {
+#ifdef SA_DEBUG_BOUNDS
+  cudaError_t e = sa::bounds_selftest(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return SA_OK;
+#else
+  (void)stream;
+  return fail(SA_ERR_UNSUPPORTED, "not a debug build (libsa_debug.so has the index checks)");
+#endif
+}
+
 sa_status sa_profile_begin(sa_cache* h) {
   if (!h) return fail(SA_ERR_INVALID_ARG, "handle is NULL");
   if (h->ev.empty()) {
@@ -1301,6 +1361,7 @@ extern "C" sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cach
     p.dt2 = dt2; p.dh2 = dh2; p.dw2 = dw2;
     const size_t n = std::min(act.size() - s0, (size_t)per_launch);
     p.n_streams = (int32_t)n;
+    p.batch = c.batch;
     for (size_t a = 0; a < n; ++a) {
       const sa_chunk_plan& pl = plans[s0 + a];
       p.stream_of[a] = act[s0 + a];
@@ -1326,6 +1387,7 @@ extern "C" sa_status sa_append_attend_noalloc(const sa_config* cfg, void* k_cach
   ap.H = c.heads; ap.Lc = (int32_t)Lc; ap.ntok = ntok;
   ap.n_q_tiles = (int32_t)((Lc + 127) / 128);
   ap.n_streams = (int32_t)act.size();
+  ap.batch = c.batch;
   const double scale = c.softmax_scale > 0.f ? (double)c.softmax_scale : 1.0 / sqrt((double)D);
   ap.scale_log2 = (float)((double)(float)scale * 1.4426950408889634);
   ap.out = out; ap.q_ws = q_ws; ap.k_cache = k_cache; ap.v_cache = v_cache;

@@ -83,6 +83,13 @@ def sa_gdn_chunk(state: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch
                              mask, ctypes.c_void_p(_stream_ptr(stream))), "sa_gdn_chunk")
 
 
+def sa_gdn_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
+    """Raises SAError(SA_ERR_DEVICE_TIMEOUT) if a bounded wait of the last call
+    that used this workspace gave up (synchronises the stream)."""
+    check(lib().sa_gdn_device_status(workspace.data_ptr(), ctypes.c_void_p(_stream_ptr(stream))),
+          "sa_gdn_device_status")
+
+
 class GDNState:
     """The recurrent state of one GDN block for B streams ([B, H, D, D] fp32,
     zero at the start of each stream) and a workspace for calls of up to

@@ -45,3 +45,18 @@ _ensure_built()
 def has_gpu():
     import torch
     return torch.cuda.is_available()
+
+
+@pytest.fixture(autouse=True)
+def _debug_bounds_words(request):
+    """Under the debug build (SA_LIBRARY_VARIANT=debug), every GPU test ends by
+    reading the kernels' index-check words: a failed check fails the test."""
+    yield
+    if os.environ.get("SA_LIBRARY_VARIANT") != "debug" or request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    from rolling_kv_cache_sa_b200 import _lib
+    st = _lib.lib().sa_debug_bounds_status(None)
+    assert st == _lib.SA_OK, _lib.lib().sa_last_error_string().decode()

@@ -33,6 +33,25 @@ def test_library_exports_every_declared_symbol():
     assert S.sa_abi_version() == 1
 
 
+def test_debug_build_exports_every_declared_symbol():
+    # the debug build (index checks in every kernel) has the same ABI
+    from rolling_kv_cache_sa_b200 import build as B
+    assert os.path.exists(B.DEBUG_LIB)
+    D = ctypes.CDLL(B.DEBUG_LIB)
+    for name in _declared_symbols():
+        assert hasattr(D, name), name
+
+
+def test_debug_entries_refused_by_the_normal_build():
+    # outside the debug build the bounds calls say so, before touching a device
+    L = _lib.lib()
+    if _lib.LIB_PATH.endswith("libsa_debug.so"):
+        pytest.skip("running against the debug build")
+    assert L.sa_debug_bounds_status(None) == _lib.SA_ERR_UNSUPPORTED
+    assert L.sa_debug_bounds_selftest(None) == _lib.SA_ERR_UNSUPPORTED
+    assert b"debug build" in L.sa_last_error_string()
+
+
 def test_invalid_configs_are_rejected():
     base = S.config_for(ALL[1])
     bad = []
@@ -167,10 +186,18 @@ def test_gdn_chunk_validates_pointers():
         _lib.SA_ERR_INVALID_ARG                      # workspace NULL
     n = ctypes.c_size_t()
     assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
-    assert n.value == 2 * 3 * 1 * 32768              # B * H * ceil(64 / 64) * 32 KiB
+    # header + B * H * ceil(T / 64) blocks: 96 KiB of operand images for D = 128
+    # (tensor-core pass), 32 KiB of fp32 T and M for D = 64
+    per = 98304 if c.head_dim == 128 else 32768
+    assert n.value == 1024 + 2 * 3 * 1 * per
     c.tokens = 65
     assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
-    assert n.value == 2 * 3 * 2 * 32768
+    assert n.value == 1024 + 2 * 3 * 2 * per
+    c.head_dim = 64
+    assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
+    assert n.value == 1024 + 2 * 3 * 2 * 32768
+    c.head_dim = 128
+    assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
     assert L.sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, p, n.value - 16, None,
                           None) == _lib.SA_ERR_INVALID_ARG   # workspace too small
     assert b"workspace" in L.sa_last_error_string()

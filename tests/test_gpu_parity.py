@@ -105,6 +105,17 @@ def test_bf16_edge_cases_every_row(name, kw):
     _run(w, steps, rows="all", cache_checks=steps)
 
 
+def test_split_units_every_row():
+    # 2 streams x 8 heads x 2 query-tile pairs = 32 units of up to 14 key tiles
+    # (448 >= the SM count): the persistent attention kernel splits units
+    # between CTAs and merges their partial results; every row is checked,
+    # across ring wrap, refreshes and a ragged start
+    w = Workload("split_units", B=2, H=8, D=128, fh=16, fw=16, C=2, S=1, W=4, n_chunks=5,
+                 dtype="bf16", refresh_period=3, starts=(0, 1))
+    steps = set(range(w.n_steps))
+    _run(w, steps, rows="all", cache_checks={1, 3, 5})
+
+
 def test_fp32_d128():
     w = Workload("fp32_d128", B=2, H=2, D=128, fh=6, fw=10, C=2, S=1, W=4, n_chunks=7,
                  dtype="f32", refresh_period=3, starts=(0, 1), dist=(NORMAL, NORMAL, UNIFORM))
