@@ -52,28 +52,10 @@ constexpr int BM = 128;                  // query rows per tile
 constexpr int BN = 128;                  // keys per tile
 constexpr uint32_t PANEL = 128u * 128u;  // one 128-row x 128-byte swizzled panel
 constexpr uint64_t kTimeoutNs = 1000000000ull;
-// 10 warps (producer, MMA issuer, two softmax warpgroups; 168 registers each
-// thread) or, with SA_ATTN_WARPS12, 12 warps in three warpgroups whose
-// registers are redistributed with setmaxnreg: the producer/MMA warpgroup
-// gives up registers to the two softmax warpgroups (launch 384 x 168 =
-// 128 x kRegLow + 256 x kRegHigh, so the increase always finds its registers).
-#ifndef SA_ATTN_WARPS12
-#define SA_ATTN_WARPS12 0
-#endif
-constexpr bool kWarps12 = SA_ATTN_WARPS12 != 0;
-constexpr int kThreads = kWarps12 ? 384 : 320;
-constexpr int kFirstSoftmaxWarp = kWarps12 ? 4 : 2;
-constexpr int kRegLaunch = 168, kRegLow = 96, kRegHigh = 200;
-static_assert(128 * kRegLow + 256 * kRegHigh <= 384 * kRegLaunch, "register split exceeds the launch");
+constexpr int kThreads = 320;
+constexpr int kFirstSoftmaxWarp = 2;
 constexpr int kMaxCtas = 256;
-#ifndef SA_ATTN_HYBRID
-#define SA_ATTN_HYBRID 1
-#endif
-constexpr bool kHybrid = SA_ATTN_HYBRID != 0;
-#ifndef SA_ATTN_ROTATE
-#define SA_ATTN_ROTATE 1
-#endif
-constexpr bool kRotate = SA_ATTN_ROTATE != 0;
+
 
 struct TcParams {
   int32_t H, Lc, n_q_tiles, n_pairs;
@@ -82,9 +64,6 @@ struct TcParams {
   int32_t batch;      // B (bounds checks)
   int64_t ntok;       // cache rows per (stream, head) (bounds checks)
   int64_t total;      // key tiles over all units
-  int32_t full;       // split mode: whole units per CTA taken first (0: pure stream-K)
-  int32_t pad2_;
-  int64_t t1;         // split mode: first key tile of the units split between CTAs
   void* out;          // [B][Lc][H][D] bf16
   float4* part_o;     // [slots][2][D/4][128] fp32 (row-contiguous per column quad)
   float2* part_ml;    // [slots][2][128] (m in log2 units, l)
@@ -111,24 +90,16 @@ __host__ __device__ inline int64_t unit_tile_offset(const TcParams& p, int64_t u
   return p.prefix[a] + (u - (int64_t)a * p.units_per_stream) * p.nkv[a];
 }
 
-// The key tiles CTA c takes in split mode, [r0, r1): an equal share of the
-// tiles from t1 on (the units split between CTAs). With full > 0 the CTA
-// first takes the whole units [c * full, (c + 1) * full) (tiles [w0, w1)),
-// so only the last units are split and their pieces all run at the end of
-// the launch, close together in time. Without a partials buffer, ranges
-// snap to whole units (w0 = w1).
-__host__ __device__ inline void cta_range(const TcParams& p, int c, int64_t& r0, int64_t& r1,
-                                          int64_t& w0, int64_t& w1) {
+// The key tiles CTA c takes, [r0, r1): an equal share of all units' tiles in
+// split mode (stream-K), else whole units.
+__host__ __device__ inline void cta_range(const TcParams& p, int c, int64_t& r0, int64_t& r1) {
   if (p.split) {
-    w0 = unit_tile_offset(p, (int64_t)c * p.full);
-    w1 = unit_tile_offset(p, (int64_t)(c + 1) * p.full);
-    r0 = p.t1 + (p.total - p.t1) * c / p.grid;
-    r1 = p.t1 + (p.total - p.t1) * (c + 1) / p.grid;
+    r0 = p.total * c / p.grid;
+    r1 = p.total * (c + 1) / p.grid;
   } else {
     const int64_t U = (int64_t)p.n_streams * p.units_per_stream;
     r0 = unit_tile_offset(p, U * c / p.grid);
     r1 = unit_tile_offset(p, U * (c + 1) / p.grid);
-    w0 = w1 = 0;
   }
 }
 
@@ -155,38 +126,32 @@ __host__ __device__ inline Seg make_seg(const TcParams& p, int64_t t, int64_t r1
   return s;
 }
 
-// The order in which a CTA takes its segments: first its whole units [w0, w1)
-// (split mode with full > 0), then its share [r0, r1) of the split units.
-// When r0 falls inside a unit (the head piece of a unit the previous CTA
-// began) and nothing else comes first, that piece goes after the rest of the
-// share, so both pieces of a unit split between CTAs c and c + 1 end near
-// the same time and the last one merges the partials while they are in L2.
-// Every role of the CTA walks the same cursor, so they agree on the order.
+// The order in which a CTA takes the segments of its range [r0, r1): when r0
+// falls inside a unit (its head piece, a unit the previous CTA began), that
+// piece goes last, so both pieces of a unit split between CTAs c and c + 1
+// end in the last part of the launch and the merge reads partials written
+// more recently. Every role of the CTA walks the same cursor, so they agree
+// on the order.
 struct SegCursor {
-  int64_t t, stop;   // current range
-  int64_t nx0, nx1;  // next range
-  int64_t nz0, nz1;  // the one after it
-  __device__ void init(const TcParams& p, int64_t r0, int64_t r1, int64_t w0, int64_t w1) {
-    int64_t h_end = r0;
-    if (kRotate && w0 >= w1 && r0 < r1) {
-      const Seg h = make_seg(p, r0, r1);
+  int64_t t, stop, r0, h_end;
+  bool second;
+  __device__ void init(const TcParams& p, int64_t r0_, int64_t r1) {
+    r0 = r0_;
+    h_end = r0_;
+    if (r0_ < r1) {
+      const Seg h = make_seg(p, r0_, r1);
       if (h.lo > 0 && h.t_end < r1) h_end = h.t_end;
     }
-    t = w0;
-    stop = w1;
-    nx0 = h_end;
-    nx1 = r1;
-    nz0 = r0;
-    nz1 = h_end;
+    t = h_end;
+    stop = r1;
+    second = false;
   }
   __device__ bool next(const TcParams& p, Seg& s) {
-    while (t >= stop) {
-      if (nx0 >= nx1 && nz0 >= nz1) return false;
-      t = nx0;
-      stop = nx1;
-      nx0 = nz0;
-      nx1 = nz1;
-      nz0 = nz1 = 0;
+    if (t >= stop) {
+      if (second || h_end <= r0) return false;
+      t = r0;
+      stop = h_end;
+      second = true;
     }
     s = make_seg(p, t, stop);
     t = s.t_end;
@@ -194,20 +159,18 @@ struct SegCursor {
   }
 };
 
-// CTA whose split share holds key tile t (t >= t1; split mode)
+// CTA whose range holds key tile t (split mode)
 __device__ inline int cta_of(const TcParams& p, int64_t t) {
-  const int64_t n = p.total - p.t1, x = t - p.t1;
-  int c = (int)(x * p.grid / n);
-  while (c + 1 < p.grid && n * (c + 1) / p.grid <= x) ++c;
-  while (c > 0 && n * c / p.grid > x) --c;
+  int c = (int)(t * p.grid / p.total);
+  while (c + 1 < p.grid && p.total * (c + 1) / p.grid <= t) ++c;
+  while (c > 0 && p.total * c / p.grid > t) --c;
   return c;
 }
 
 // Partial slot of the piece that CTA c holds of the unit starting at tile us:
-// slot 2c for the piece that starts c's split share, 2c + 1 for the one that
-// ends it.
+// slot 2c for the piece that starts c's range, 2c + 1 for the one that ends it.
 __device__ inline int piece_slot(const TcParams& p, int c, int c_first, int64_t us) {
-  return 2 * c + ((c == c_first && p.t1 + (p.total - p.t1) * c / p.grid != us) ? 1 : 0);
+  return 2 * c + ((c == c_first && p.total * c / p.grid != us) ? 1 : 0);
 }
 
 // Merge of one query row of a split unit from the partial results of its
@@ -325,51 +288,18 @@ struct Layout {
   static_assert(bytes <= 232448, "exceeds 227 KB of shared memory per CTA");
 };
 
-// 2^x of two floats on the FMA pipe instead of the MUFU unit, by the range
-// reduction of Cody and Waite (1980): x = n + f with n = round(x) and
-// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with constant term 1, fitted
-// here by a minimax linear program on [-1/2, 1/2] (relative error 1.0e-4,
-// below the 2^-9 of the bf16 rounding that P then goes through); 2^n is
-// added to the exponent field. round(x) comes from adding 1.5 * 2^23 (the
-// sum's low mantissa bits hold n), so no conversion instruction is used.
-// x is clamped to -120 first (masked columns are -inf), which keeps the
-// exponent field positive; 2^-120 instead of 0 is negligible against the
-// row's largest term (>= 2^-8).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c1 = 0x1.62f5fap-1f, c2 = 0x1.f00c4cp-3f, c3 = 0x1.c2a21ap-5f;
-  x.x = fmaxf(x.x, -120.f);
-  x.y = fmaxf(x.y, -120.f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));            // kRound + n
-  const float2 r = __ffma2_rn(t, make_float2(-1.f, -1.f), make_float2(kRound, kRound));  // -n
-  const float2 f = __fadd2_rn(x, r);                                      // exact
-  float2 pf = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
-  pf = __ffma2_rn(pf, f, make_float2(c1, c1));
-  pf = __ffma2_rn(pf, f, make_float2(1.f, 1.f));
-  return make_float2(__uint_as_float(__float_as_uint(pf.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(pf.y) + (__float_as_uint(t.y) << 23)));
-}
-
-// Pairs of a 32-score group whose exponentials run on the FMA pipe: kPoly of
-// the 16, spread evenly (pair e when (e * kPoly) mod 16 < kPoly).
-#ifndef SA_EXP2_POLY_PAIRS
-#define SA_EXP2_POLY_PAIRS 0
-#endif
-
 // P of 32 consecutive scores of a row as 16 words of bf16 pairs, and their
-// sum added to ls (four packed partial sums).
-template <int kPoly>
+// sum added to ls (four packed partial sums). The exponentials run on the
+// MUFU unit (4 per clock per SM sub-partition, in f32 or packed bf16x2 form
+// alike); a polynomial on the FMA pipe costs more per element on this chip
+// (FFMA2 issues at half rate), so none is used.
 __device__ __forceinline__ void p_group(const uint32_t* sv, float2 sl2v, float2 nmv, float2* ls,
                                         uint32_t* w) {
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * e]),
                                             __uint_as_float(sv[2 * e + 1])), sl2v, nmv);
-    float2 pe;
-    if ((e * kPoly) % 16 < kPoly)
-      pe = exp2_poly2(x);
-    else
-      pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
+    const float2 pe = make_float2(ptx::ex2(x.x), ptx::ex2(x.y));
     ls[e & 3] = __fadd2_rn(ls[e & 3], pe);
     w[e] = ptx::pack_bf16x2(pe.x, pe.y);
   }
@@ -502,9 +432,9 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
     // bf16: groups of 32 keys; the third group is computed before waiting
     // for the first two groups' TMEM stores, so that wait overlaps work
     uint32_t wa[16], wb[16];
-    p_group<SA_EXP2_POLY_PAIRS>(sv, sl2v, nmv, ls, wa);
+    p_group(sv, sl2v, nmv, ls, wa);
     ptx::tmem_st16u(sbuf, wa);
-    p_group<SA_EXP2_POLY_PAIRS>(sv + 32, sl2v, nmv, ls, wb);
+    p_group(sv + 32, sl2v, nmv, ls, wb);
     ptx::tmem_st16u(sbuf + 16u, wb);
     if (__any_sync(0xffffffffu, alpha < 1.f)) {
       // O holds PV of the previous key tile: MMAs complete in issue order and
@@ -514,12 +444,12 @@ __device__ __forceinline__ bool row_softmax(uint32_t sbuf, uint32_t obuf, int va
       ptx::tc_fence_after();
       rescale_o<HD>(obuf, alpha);
     }
-    p_group<SA_EXP2_POLY_PAIRS>(sv + 64, sl2v, nmv, ls, wa);
+    p_group(sv + 64, sl2v, nmv, ls, wa);
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
     ptx::mbar_arrive(bar_pa);
     ptx::tmem_st16u(sbuf + 32u, wa);
-    p_group<SA_EXP2_POLY_PAIRS>(sv + 96, sl2v, nmv, ls, wb);
+    p_group(sv + 96, sl2v, nmv, ls, wb);
     ptx::tmem_st16u(sbuf + 48u, wb);
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
@@ -626,10 +556,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 1;
     atomicOr(p.status, kDeviceErrTimeout);
   };
-  int64_t r0, r1, w0, w1;
-  cta_range(p, blockIdx.x, r0, r1, w0, w1);
+  int64_t r0, r1;
+  cta_range(p, blockIdx.x, r0, r1);
   if (warp < kFirstSoftmaxWarp) {
-  if constexpr (kWarps12) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -639,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n = 0, g = 0;
       bool ok = true;
       SegCursor cur;
-      cur.init(p, r0, r1, w0, w1);
+      cur.init(p, r0, r1);
       Seg sg;
       while (ok && cur.next(p, sg)) {
         if (n > 0 && !ptx::mbar_wait(bar(L::B_QE), (uint32_t)(n - 1) & 1, abort_flag, kTimeoutNs)) {
@@ -736,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       SegCursor cur;
-      cur.init(p, r0, r1, w0, w1);
+      cur.init(p, r0, r1);
       Seg sg;
       while (ok && cur.next(p, sg)) {
         if (pend && !issue_pv1()) { ok = false; break; }
@@ -812,7 +741,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   } else {
-    if constexpr (kWarps12) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh));
     // ------------------------------------------------------------ softmax + epilogue
     const int ti = (warp - kFirstSoftmaxWarp) >> 2;  // query tile of this warp's warpgroup
     const int quad = warp & 3;       // TMEM lane quadrant this warp may access
@@ -823,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int gi = 0;
     bool ok = true;
     SegCursor cur;
-    cur.init(p, r0, r1, w0, w1);
+    cur.init(p, r0, r1);
     Seg sg;
     while (ok && cur.next(p, sg)) {
       if (ti == 1 && !sg.two) continue;
@@ -977,19 +905,6 @@ cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtenso
   p.split = partials != nullptr && partials_bytes >= need && total >= G;
   if (!p.split) G = (int)std::min<int64_t>(G, units);
   p.grid = G;
-  p.full = 0;
-  p.t1 = 0;
-  if (p.split && kHybrid) {
-    // whole units first when every unit costs the same (equal key counts):
-    // full per CTA, and the rest split; at least G key tiles must remain to
-    // split so that every CTA's share is non-empty
-    bool equal = true;
-    for (int a = 1; a < ap.n_streams; ++a) equal = equal && p.nkv[a] == p.nkv[0];
-    int64_t full = equal ? units / G : 0;
-    while (full > 0 && total - unit_tile_offset(p, full * G) < G) --full;
-    p.full = (int32_t)full;
-    p.t1 = unit_tile_offset(p, full * G);
-  }
   if (p.split) {
     char* w = static_cast<char*>(partials);
     p.part_o = reinterpret_cast<float4*>(w);
