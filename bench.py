@@ -40,7 +40,7 @@ METRIC = "streamed chunks/s and attention TFLOP/s (% of B200 BF16 peak) per conf
 # DRAM bytes (read + write) per launch of the attention kernel, from the ncu
 # capture summarised in profiles/ (512p, steady chunk with 7168 keys), keyed by
 # a hash of the kernel sources it was taken on: a changed kernel reports null.
-PROFILED_TRAFFIC = {"c8df9477bcca4326": 173.17e6, "c8df9477bcca4326/e4m3": 61.97e6}
+PROFILED_TRAFFIC = {"040bfbaec52da310": 154.10e6}
 
 
 def attend_source_hash() -> str:
@@ -868,7 +868,9 @@ def main():
                                       "(7168 keys, cold L2); algorithmic minimum 63 MB (e4m3 "
                                       "Q', K', V in, bf16 O out)") if f8 else
                                      ("ncu dram read+write bytes of one steady-state launch "
-                                      "(7168 keys, cold L2); algorithmic minimum 113 MB")},
+                                      "(7168 keys, cold L2); algorithmic minimum 113.3 MB "
+                                      "(Q' 12.6, K' and V 88.1, O 12.6); the excess is split "
+                                      "units' fp32 partials and K'/V re-reads past L2")},
         "per_config": per_config,
         "cpu_baseline": cpu,
         "e2e": e2e,
