@@ -52,6 +52,15 @@ constexpr int BM = 128;                  // query rows per tile
 constexpr int BN = 128;                  // keys per tile
 constexpr uint32_t PANEL = 128u * 128u;  // one 128-row x 128-byte swizzled panel
 constexpr uint64_t kTimeoutNs = 1000000000ull;
+// A split unit's partial results are dead once merged: their L2 lines are
+// dropped with discard.global.L2 instead of being written back to DRAM
+// (measured on the 512p step: 3.5 MB less DRAM writing per launch, and the
+// append kernel that follows runs 8 % faster with fewer dirty lines to
+// evict; dropping the rotated-query rows as well was measured 1 % slower).
+#ifndef SA_ATTN_DISCARD
+#define SA_ATTN_DISCARD 1
+#endif
+constexpr bool kDiscardPartials = SA_ATTN_DISCARD != 0;
 constexpr int kThreads = 320;
 constexpr int kFirstSoftmaxWarp = 2;
 constexpr int kMaxCtas = 256;
@@ -829,6 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar(L::B_OF + ti));  // O_i is free for the next unit
+
       if (sg.partial) {
         // count this piece in for the row; the last one merges all pieces
         const int64_t us = sg.t_end - (sg.hi - sg.lo) - sg.lo;
@@ -836,6 +846,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t u = (int64_t)sg.a * p.units_per_stream + (int64_t)sg.h * p.n_pairs + sg.qp;
         int* ctr = p.counters + (u * 2 + ti) * BM + row;
         __threadfence();
+        bool merged = false;
         if (SA_BOUNDS(u >= 0 && u < (int64_t)p.n_streams * p.units_per_stream && c0 >= 0 &&
                           c1 < p.grid && c0 <= c1, 4) &&
             atomicAdd(ctr, 1) == c1 - c0) {
@@ -845,6 +856,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tok < p.Lc ? static_cast<__nv_bfloat16*>(p.out) +
                                          (((int64_t)sg.b * p.Lc + tok) * p.H + sg.h) * HD
                                    : nullptr);
+          merged = true;
+        }
+        if (kDiscardPartials && __all_sync(0xffffffffu, merged)) {
+          // every row of this warp is merged: the pieces' partial results of
+          // these 32 rows are dead; drop their L2 lines without a write-back
+          // (a 128-byte line holds 8 rows of one column quad)
+          for (int c = c0; c <= c1; ++c) {
+            const int sl = piece_slot(p, c, c0, us);
+            const char* pb = reinterpret_cast<const char*>(
+                p.part_o + ((int64_t)sl * 2 + ti) * (HD / 4) * BM + quad * 32);
+#pragma unroll 1
+            for (int i = lane; i < (HD / 4) * 4; i += 32)
+              asm volatile("discard.global.L2 [%0], 128;" ::"l"(pb + (i >> 2) * (BM * 16) +
+                                                                 (i & 3) * 128)
+                           : "memory");
+            if (lane < 2)
+              asm volatile("discard.global.L2 [%0], 128;" ::"l"(
+                               reinterpret_cast<const char*>(p.part_ml + ((int64_t)sl * 2 + ti) * BM +
+                                                             quad * 32) + lane * 128)
+                           : "memory");
+          }
         }
       }
     }
