@@ -5,8 +5,9 @@
 // tiles of all units are laid end to end; a persistent grid of one CTA per SM
 // takes equal contiguous ranges of that sequence (stream-K), so no SM idles
 // in a last partial wave. A unit cut by range boundaries is finished inside
-// the same launch: every piece stores its fp32 partial result (unnormalised
-// O, running max, row sum) and counts itself in on a per-row counter; the
+// the same launch: every piece stores its partial result (its output
+// normalised by its own row sum, in fp16, and the running max and row sum in
+// fp32) and counts itself in on a per-row counter; the
 // thread that arrives last for a row merges all pieces of that row and
 // writes it (no waiting on other CTAs). Without a partials buffer, ranges
 // snap to whole units instead.
@@ -31,6 +32,7 @@
 // Every wait is bounded (about 1 s); on expiry the CTA records a device error,
 // drains its outstanding copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <string.h>
 
 #include <algorithm>
@@ -74,7 +76,8 @@ struct TcParams {
   int64_t ntok;       // cache rows per (stream, head) (bounds checks)
   int64_t total;      // key tiles over all units
   void* out;          // [B][Lc][H][D] bf16
-  float4* part_o;     // [slots][2][D/4][128] fp32 (row-contiguous per column quad)
+  uint4* part_o;      // [slots][2][D/8][128] the piece's O / l as fp16, 8 columns per
+                      // 16 bytes, row-contiguous per group of 8 columns
   float2* part_ml;    // [slots][2][128] (m in log2 units, l)
   int* counters;      // [units][2][128] pieces counted in; back to 0 after the merge
   int* status;
@@ -182,26 +185,86 @@ __device__ inline int piece_slot(const TcParams& p, int c, int c_first, int64_t 
   return 2 * c + ((c == c_first && p.total * c / p.grid != us) ? 1 : 0);
 }
 
+// Eight fp16 of a 16-byte word as floats.
+__device__ __forceinline__ void unpack_h8(uint4 u, float* x) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+
+// Eight floats as fp16 (round to nearest) in a 16-byte word.
+__device__ __forceinline__ uint4 pack_h8(const float* x) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Merge of one query row of a split unit from the partial results of its
-// pieces (CTAs c0..c1): O = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,
+// pieces (CTAs c0..c1). Piece k stored its normalised output P_k = O_k / l_k
+// in fp16 (|P_k| <= max |v|; relative step 2^-11, a quarter of the final bf16
+// rounding) and (m_k, l_k) in fp32:
+//   O = sum_k w_k P_k,  w_k = 2^(m_k - M) l_k / sum_j 2^(m_j - M) l_j,
 // stored as bf16 to dst (nullptr: a padding row past Lc, nothing stored).
-// The other pieces' partials were written long before and are usually out of
-// L2, so every line of this row is first prefetched into L2 (one memory
-// latency for all of them instead of one per piece and column chunk); two
-// pieces -- the only case at the workload sizes, where a CTA's range is longer
-// than a unit -- are then read together. Kept out of line so the softmax
-// loop's register allocation does not see it.
+// All CTAs merge at about the same time, at the end of the launch, so the
+// bytes read here bound the merge: fp16 halves them. The other piece's
+// partials were written long before and are usually out of L2: the row's
+// lines are prefetched into L2 first. Two pieces (the only case at the
+// workload sizes, where a CTA's range is longer than a unit) are read
+// together. Kept out of line so the softmax loop's register allocation does
+// not see it.
 template <int HD>
 __device__ __noinline__ void merge_row(const TcParams& p, int ti, int row, int c0, int c1,
                                        int64_t us, __nv_bfloat16* dst) {
+  constexpr int kG = HD / 8;  // 16-byte groups of a row
+  if (c1 == c0 + 1) {
+    const int s0 = piece_slot(p, c0, c0, us), s1 = piece_slot(p, c1, c0, us);
+    if (!SA_BOUNDS(s0 >= 0 && s0 < 2 * p.grid && s1 >= 0 && s1 < 2 * p.grid, 5)) return;
+    const uint4* a0 = p.part_o + ((int64_t)s0 * 2 + ti) * kG * BM + row;
+    const uint4* a1 = p.part_o + ((int64_t)s1 * 2 + ti) * kG * BM + row;
+    if (!dst) return;
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a0 + g * BM));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a1 + g * BM));
+    }
+    const float2 ml0 = __ldcg(p.part_ml + ((int64_t)s0 * 2 + ti) * BM + row);
+    const float2 ml1 = __ldcg(p.part_ml + ((int64_t)s1 * 2 + ti) * BM + row);
+    const float M = fmaxf(ml0.x, ml1.x);
+    const float e0 = ptx::ex2(ml0.x - M) * ml0.y, e1 = ptx::ex2(ml1.x - M) * ml1.y;
+    const float inv = 1.f / (e0 + e1);
+    const float w0 = e0 * inv, w1 = e1 * inv;
+    uint4 x0[kG], x1[kG];
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      x0[g] = __ldcg(a0 + g * BM);
+      x1[g] = __ldcg(a1 + g * BM);
+    }
+#pragma unroll
+    for (int g = 0; g < kG; ++g) {
+      float u[8], v[8];
+      unpack_h8(x0[g], u);
+      unpack_h8(x1[g], v);
+      uint4 o;
+      o.x = ptx::pack_bf16x2(fmaf(w0, u[0], w1 * v[0]), fmaf(w0, u[1], w1 * v[1]));
+      o.y = ptx::pack_bf16x2(fmaf(w0, u[2], w1 * v[2]), fmaf(w0, u[3], w1 * v[3]));
+      o.z = ptx::pack_bf16x2(fmaf(w0, u[4], w1 * v[4]), fmaf(w0, u[5], w1 * v[5]));
+      o.w = ptx::pack_bf16x2(fmaf(w0, u[6], w1 * v[6]), fmaf(w0, u[7], w1 * v[7]));
+      *reinterpret_cast<uint4*>(dst + g * 8) = o;
+    }
+    return;
+  }
   float M = -INFINITY;
   for (int c = c0; c <= c1; ++c) {
     const int sl = piece_slot(p, c, c0, us);
     if (!SA_BOUNDS(sl >= 0 && sl < 2 * p.grid, 5)) return;
-    const float4* src = p.part_o + ((int64_t)sl * 2 + ti) * (HD / 4) * BM + row;
-#pragma unroll
-    for (int g4 = 0; g4 < HD / 4; ++g4)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(src + g4 * BM));
     M = fmaxf(M, __ldcg(p.part_ml + ((int64_t)sl * 2 + ti) * BM + row).x);
   }
   float Ls = 0.f;
@@ -210,62 +273,34 @@ __device__ __noinline__ void merge_row(const TcParams& p, int ti, int row, int c
     const float2 ml = __ldcg(p.part_ml + ((int64_t)sl * 2 + ti) * BM + row);
     Ls += ptx::ex2(ml.x - M) * ml.y;
   }
-  const float inv = 1.f / Ls;
   if (!dst) return;
-  if (c1 == c0 + 1) {
-    const int s0 = piece_slot(p, c0, c0, us), s1 = piece_slot(p, c1, c0, us);
-    const float w0 = ptx::ex2(__ldcg(p.part_ml + ((int64_t)s0 * 2 + ti) * BM + row).x - M) * inv;
-    const float w1 = ptx::ex2(__ldcg(p.part_ml + ((int64_t)s1 * 2 + ti) * BM + row).x - M) * inv;
-    const float4* a0 = p.part_o + ((int64_t)s0 * 2 + ti) * (HD / 4) * BM + row;
-    const float4* a1 = p.part_o + ((int64_t)s1 * 2 + ti) * (HD / 4) * BM + row;
+  const float inv = 1.f / Ls;
 #pragma unroll 1
-    for (int cc = 0; cc < HD / 32; ++cc) {
-      float4 x0[8], x1[8];
-#pragma unroll
-      for (int g4 = 0; g4 < 8; ++g4) {
-        x0[g4] = __ldcg(a0 + (cc * 8 + g4) * BM);
-        x1[g4] = __ldcg(a1 + (cc * 8 + g4) * BM);
-      }
-#pragma unroll
-      for (int g8 = 0; g8 < 4; ++g8) {
-        const float4 u0 = x0[2 * g8], u1 = x0[2 * g8 + 1], v0 = x1[2 * g8], v1 = x1[2 * g8 + 1];
-        uint4 o;
-        o.x = ptx::pack_bf16x2(fmaf(w0, u0.x, w1 * v0.x), fmaf(w0, u0.y, w1 * v0.y));
-        o.y = ptx::pack_bf16x2(fmaf(w0, u0.z, w1 * v0.z), fmaf(w0, u0.w, w1 * v0.w));
-        o.z = ptx::pack_bf16x2(fmaf(w0, u1.x, w1 * v1.x), fmaf(w0, u1.y, w1 * v1.y));
-        o.w = ptx::pack_bf16x2(fmaf(w0, u1.z, w1 * v1.z), fmaf(w0, u1.w, w1 * v1.w));
-        *reinterpret_cast<uint4*>(dst + cc * 32 + g8 * 8) = o;
-      }
-    }
-    return;
-  }
-#pragma unroll 1
-  for (int cc = 0; cc < HD / 32; ++cc) {
+  for (int g0 = 0; g0 < kG; g0 += 4) {  // 32 columns at a time
     float acc[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] = 0.f;
     for (int c = c0; c <= c1; ++c) {
       const int sl = piece_slot(p, c, c0, us);
       const float2 ml = __ldcg(p.part_ml + ((int64_t)sl * 2 + ti) * BM + row);
-      const float w = ptx::ex2(ml.x - M);
-      const float4* src = p.part_o + (((int64_t)sl * 2 + ti) * (HD / 4) + cc * 8) * BM + row;
+      const float w = ptx::ex2(ml.x - M) * ml.y * inv;
+      const uint4* src = p.part_o + ((int64_t)sl * 2 + ti) * kG * BM + row;
 #pragma unroll
-      for (int g4 = 0; g4 < 8; ++g4) {
-        const float4 v = __ldcg(src + g4 * BM);
-        acc[g4 * 4 + 0] = fmaf(w, v.x, acc[g4 * 4 + 0]);
-        acc[g4 * 4 + 1] = fmaf(w, v.y, acc[g4 * 4 + 1]);
-        acc[g4 * 4 + 2] = fmaf(w, v.z, acc[g4 * 4 + 2]);
-        acc[g4 * 4 + 3] = fmaf(w, v.w, acc[g4 * 4 + 3]);
+      for (int g = 0; g < 4; ++g) {
+        float u[8];
+        unpack_h8(__ldcg(src + (g0 + g) * BM), u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[g * 8 + i] = fmaf(w, u[i], acc[g * 8 + i]);
       }
     }
 #pragma unroll
-    for (int g8 = 0; g8 < 4; ++g8) {
+    for (int g = 0; g < 4; ++g) {
       uint4 v;
-      v.x = ptx::pack_bf16x2(acc[g8 * 8 + 0] * inv, acc[g8 * 8 + 1] * inv);
-      v.y = ptx::pack_bf16x2(acc[g8 * 8 + 2] * inv, acc[g8 * 8 + 3] * inv);
-      v.z = ptx::pack_bf16x2(acc[g8 * 8 + 4] * inv, acc[g8 * 8 + 5] * inv);
-      v.w = ptx::pack_bf16x2(acc[g8 * 8 + 6] * inv, acc[g8 * 8 + 7] * inv);
-      *reinterpret_cast<uint4*>(dst + cc * 32 + g8 * 8) = v;
+      v.x = ptx::pack_bf16x2(acc[g * 8 + 0], acc[g * 8 + 1]);
+      v.y = ptx::pack_bf16x2(acc[g * 8 + 2], acc[g * 8 + 3]);
+      v.z = ptx::pack_bf16x2(acc[g * 8 + 4], acc[g * 8 + 5]);
+      v.w = ptx::pack_bf16x2(acc[g * 8 + 6], acc[g * 8 + 7]);
+      *reinterpret_cast<uint4*>(dst + (g0 + g) * 8) = v;
     }
   }
 }
@@ -799,21 +834,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv = o_scale / l;
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
                              (((int64_t)sg.b * p.Lc + tok) * p.H + sg.h) * HD;
+        // the whole O row in one TMEM round trip
+        float ov[HD];
 #pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          float ov[32];
-          ptx::tmem_ld32(obuf + c * 32, ov);
-          ptx::tmem_wait_ld();
-          if (tok < p.Lc && st_ok) {
+        for (int c = 0; c < HD / 32; ++c) ptx::tmem_ld32(obuf + c * 32, ov + c * 32);
+        ptx::tmem_wait_ld();
+        if (tok < p.Lc && st_ok) {
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-              uint4 v;
-              v.x = ptx::pack_bf16x2(ov[g8 * 8 + 0] * inv, ov[g8 * 8 + 1] * inv);
-              v.y = ptx::pack_bf16x2(ov[g8 * 8 + 2] * inv, ov[g8 * 8 + 3] * inv);
-              v.z = ptx::pack_bf16x2(ov[g8 * 8 + 4] * inv, ov[g8 * 8 + 5] * inv);
-              v.w = ptx::pack_bf16x2(ov[g8 * 8 + 6] * inv, ov[g8 * 8 + 7] * inv);
-              *reinterpret_cast<uint4*>(dst + c * 32 + g8 * 8) = v;
-            }
+          for (int g8 = 0; g8 < HD / 8; ++g8) {
+            uint4 v;
+            v.x = ptx::pack_bf16x2(ov[g8 * 8 + 0] * inv, ov[g8 * 8 + 1] * inv);
+            v.y = ptx::pack_bf16x2(ov[g8 * 8 + 2] * inv, ov[g8 * 8 + 3] * inv);
+            v.z = ptx::pack_bf16x2(ov[g8 * 8 + 4] * inv, ov[g8 * 8 + 5] * inv);
+            v.w = ptx::pack_bf16x2(ov[g8 * 8 + 6] * inv, ov[g8 * 8 + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + g8 * 8) = v;
           }
         }
       } else {
@@ -821,18 +855,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // other (a CTA has at most two partial pieces: its first and last)
         const int slot = 2 * (int)blockIdx.x + (sg.t_end - (sg.hi - sg.lo) == r0 ? 0 : 1);
         const bool sl_ok = SA_BOUNDS(slot >= 0 && slot < 2 * p.grid, 3);
-        float4* po = p.part_o + ((int64_t)slot * 2 + ti) * (HD / 4) * BM + row;
+        uint4* po = p.part_o + ((int64_t)slot * 2 + ti) * (HD / 8) * BM + row;
+        float ov[HD];
 #pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          float ov[32];
-          ptx::tmem_ld32(obuf + c * 32, ov);
-          ptx::tmem_wait_ld();
-          if (sl_ok) {
+        for (int c = 0; c < HD / 32; ++c) ptx::tmem_ld32(obuf + c * 32, ov + c * 32);
+        ptx::tmem_wait_ld();
+        if (sl_ok) {
+          // normalised, in output units (v scale removed), fp16
+          const float nrm = o_scale / l;
 #pragma unroll
-            for (int g4 = 0; g4 < 8; ++g4)  // partials in output units (v scale removed)
-              po[(c * 8 + g4) * BM] = make_float4(ov[g4 * 4] * o_scale, ov[g4 * 4 + 1] * o_scale,
-                                                  ov[g4 * 4 + 2] * o_scale, ov[g4 * 4 + 3] * o_scale);
-          }
+          for (int i = 0; i < HD; ++i) ov[i] *= nrm;
+#pragma unroll
+          for (int g = 0; g < HD / 8; ++g) po[g * BM] = pack_h8(ov + g * 8);
         }
         if (sl_ok) p.part_ml[((int64_t)slot * 2 + ti) * BM + row] = make_float2(m_used, l);
       }
@@ -861,13 +895,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kDiscardPartials && __all_sync(0xffffffffu, merged)) {
           // every row of this warp is merged: the pieces' partial results of
           // these 32 rows are dead; drop their L2 lines without a write-back
-          // (a 128-byte line holds 8 rows of one column quad)
+          // (a 128-byte line holds 8 rows of one 8-column group)
           for (int c = c0; c <= c1; ++c) {
             const int sl = piece_slot(p, c, c0, us);
             const char* pb = reinterpret_cast<const char*>(
-                p.part_o + ((int64_t)sl * 2 + ti) * (HD / 4) * BM + quad * 32);
+                p.part_o + ((int64_t)sl * 2 + ti) * (HD / 8) * BM + quad * 32);
 #pragma unroll 1
-            for (int i = lane; i < (HD / 4) * 4; i += 32)
+            for (int i = lane; i < (HD / 8) * 4; i += 32)
               asm volatile("discard.global.L2 [%0], 128;" ::"l"(pb + (i >> 2) * (BM * 16) +
                                                                  (i & 3) * 128)
                            : "memory");
@@ -939,7 +973,7 @@ cudaError_t launch_tc(const AttnParams& ap, const CUtensorMap* tq, const CUtenso
   p.grid = G;
   if (p.split) {
     char* w = static_cast<char*>(partials);
-    p.part_o = reinterpret_cast<float4*>(w);
+    p.part_o = reinterpret_cast<uint4*>(w);
     w += (size_t)2 * G * 2 * BM * HD * sizeof(float);
     p.part_ml = reinterpret_cast<float2*>(w);
     w += (size_t)2 * G * 2 * BM * sizeof(float2);
