@@ -357,7 +357,6 @@ sa_status sa_gdn_chunk(const sa_gdn_config* cfg, float* state, const void* q, co
                        sa_stream_t stream) {
   sa_status vst = validate_gdn_config(cfg);
   if (vst != SA_OK) return vst;
-  const size_t esz = cfg->dtype == SA_F32 ? 4 : 2;
   if (!state) return fail(SA_ERR_INVALID_ARG, "state is NULL");
   if (reinterpret_cast<uintptr_t>(state) % 16)
     return fail(SA_ERR_INVALID_ARG, "state must be 16-byte aligned");
