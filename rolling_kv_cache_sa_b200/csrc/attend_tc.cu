@@ -679,6 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (F8) ptx::umma_ts_f8(d, a, b, id, acc); else ptx::umma_ts(d, a, b, id, acc);
       };
       const uint32_t o0 = tmem + 256u, o1 = tmem + 256u + HD;
+      const uint64_t dq = ptx::sdesc_sw128(base + L::q0, 16, 1024);
       int n = 0, g = 0, g1 = 0, nseg1 = 0;
       bool ok = true;
       // PV1 of the previous key tile, issued after the next QK0
@@ -689,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             !ptx::mbar_wait(bar(L::B_OF + 1), (uint32_t)(pend_nseg1 - 1) & 1, abort_flag, kTimeoutNs))
           return false;
         const int s = pend_g % ST;
-        const uint32_t vb = base + L::v0 + s * L::kTile;
+        const uint64_t dv = ptx::sdesc_sw128(base + L::v0 + s * L::kTile, PANEL, 1024);
         for (int h2 = 0; h2 < 2; ++h2) {
           if (!ptx::mbar_wait(bar((h2 == 0 ? L::B_PF : L::B_PB) + 1), (uint32_t)pend_g1 & 1,
                               abort_flag, kTimeoutNs))
@@ -698,9 +699,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k2 = 0; k2 < kPvHalf; ++k2) {
             const int kk = h2 * kPvHalf + k2;
-            mma_ts(o1, tmem + 128u + (uint32_t)kk * 8u,
-                   ptx::sdesc_sw128(vb + (uint32_t)kk * kVStep, PANEL, 1024), idesc_pv,
-                   (!pend_first || kk > 0) ? 1u : 0u);
+            mma_ts(o1, tmem + 128u + (uint32_t)kk * 8u, ptx::sdesc_add(dv, (uint32_t)kk * kVStep),
+                   idesc_pv, (!pend_first || kk > 0) ? 1u : 0u);
           }
         }
         ptx::umma_commit(bar(L::B_OD + 1));
@@ -719,12 +719,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t u = (uint32_t)(g / ST);
           if (!ptx::mbar_wait(bar(L::B_KF + s), u & 1, abort_flag, kTimeoutNs)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t kb = base + L::k0 + s * L::kTile;
+          const uint64_t dk = ptx::sdesc_sw128(base + L::k0 + s * L::kTile, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kQkSteps; ++kk) {
             const uint32_t off = qk_off(kk);
-            mma_ss(tmem, ptx::sdesc_sw128(base + L::q0 + off, 16, 1024),
-                   ptx::sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            mma_ss(tmem, ptx::sdesc_add(dq, off), ptx::sdesc_add(dk, off), idesc_qk,
+                   kk > 0 ? 1u : 0u);
           }
           ptx::umma_commit(bar(L::B_SF + 0));
           if (pend && !issue_pv1()) { ok = false; break; }
@@ -732,8 +732,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kQkSteps; ++kk) {
               const uint32_t off = qk_off(kk);
-              mma_ss(tmem + 128u, ptx::sdesc_sw128(base + L::q0 + L::kTile + off, 16, 1024),
-                     ptx::sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + 128u, ptx::sdesc_add(dq, L::kTile + off), ptx::sdesc_add(dk, off),
+                     idesc_qk, kk > 0 ? 1u : 0u);
             }
             ptx::umma_commit(bar(L::B_SF + 1));
           }
@@ -745,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const uint32_t vb = base + L::v0 + s * L::kTile;
+          const uint64_t dv = ptx::sdesc_sw128(base + L::v0 + s * L::kTile, PANEL, 1024);
           for (int h2 = 0; h2 < 2 && ok; ++h2) {
             if (!ptx::mbar_wait(bar((h2 == 0 ? L::B_PF : L::B_PB) + 0), (uint32_t)g & 1, abort_flag,
                                 kTimeoutNs)) {
@@ -756,9 +756,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k2 = 0; k2 < kPvHalf; ++k2) {
               const int kk = h2 * kPvHalf + k2;
-              mma_ts(o0, tmem + (uint32_t)kk * 8u,
-                     ptx::sdesc_sw128(vb + (uint32_t)kk * kVStep, PANEL, 1024), idesc_pv,
-                     (kv > sg.lo || kk > 0) ? 1u : 0u);
+              mma_ts(o0, tmem + (uint32_t)kk * 8u, ptx::sdesc_add(dv, (uint32_t)kk * kVStep),
+                     idesc_pv, (kv > sg.lo || kk > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;

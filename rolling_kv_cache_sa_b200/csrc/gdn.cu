@@ -27,17 +27,22 @@
 //     [A 0; C B]^-1 = [A^-1 0; -B^-1 C A^-1  B^-1].
 //
 // Two kernels per call:
-//  * gdn_prep_kernel: one CTA per (stream, head, sub-chunk), all independent.
+//  * the prep kernel: one CTA per (stream, head, sub-chunk), all independent.
 //    It computes what depends only on K, Q, g and beta -- T = (I + L)^-1 and
-//    M = scale P T -- and writes both (64 x 64 fp32 each) to the workspace.
-//    With U = T RHS, the intra-chunk part of the outputs is P U = M RHS, so the
-//    sequential pass gets U and the outputs from one sweep over RHS.
-//  * gdn_chunk_kernel: one CTA per (stream, head, 32 value rows of the state).
-//    Rows of S evolve independently, so a CTA owns its 32 x D slice of the
-//    state for the whole call (in registers, with a copy in shared memory for
-//    the products that read it by rows) and walks the sub-chunks in order,
-//    loading each one's T and P from the workspace one sub-chunk ahead.
-// All arithmetic is fp32 on the CUDA cores.
+//    M = scale P T. With U = T RHS, the intra-chunk part of the outputs is
+//    P U = M RHS, so the sequential pass gets U and the outputs from one
+//    sweep over RHS.
+//  * the sequential pass: one CTA per (stream, head, slice of value rows of
+//    the state). Rows of S evolve independently, so a CTA owns its slice of
+//    the state for the whole call and walks the sub-chunks in order.
+// D = 128 runs on the tensor core: gdn_prep_tc_kernel forms the Gram
+// matrices with tcgen05 MMAs and writes bf16 hi/lo operand images of K^, Q^,
+// T and M; gdn_tc_kernel keeps a 64-column state slice in TMEM (both
+// described where they are defined). D = 64 runs in fp32 on the CUDA cores:
+// gdn_prep_kernel writes T and M (64 x 64 fp32 each) and gdn_chunk_kernel
+// keeps a 32-row state slice in registers, with a copy in shared memory for
+// the products that read it by rows, loading each sub-chunk's T and M one
+// sub-chunk ahead.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -237,10 +242,194 @@ __device__ __forceinline__ void gate_scan(float g, float beta, float* Gs, float*
   Gs[tid] = gl;
 }
 
-// One CTA per (stream, head, sub-chunk): T = (I + L)^-1 and M = scale P T of
-// the sub-chunk into the workspace, both [64][64] row-major, zero above the
-// diagonal.
-template <int D, typename T, bool kImg>
+// T = (I + L)^-1 of one sub-chunk: L strictly lower in Lm (pitch kLp), T
+// into Tm, Xm merge scratch (32 x 33 floats); all kGdnThreads threads take
+// part and the last step ends with a barrier.
+__device__ __forceinline__ void unit_lower_inverse(const float* Lm, float* Tm, float* Xm, int tid,
+                                                   int warp, int lane) {
+  // ---- diagonal 16 x 16 blocks of (I + L)^-1: thread (blk, j) solves for
+  // column j of its block
+  if (tid < 64) {
+    const int r0 = (tid >> 4) * 16, j = tid & 15;
+    float x[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      float acc = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < t; ++s2) acc = fmaf(Lm[(r0 + t) * kLp + r0 + s2], x[s2], acc);
+      x[t] = t < j ? 0.f : (t == j ? 1.f : -acc);
+    }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) Tm[(r0 + t) * kLp + r0 + j] = x[t];
+  }
+  __syncthreads();
+
+  // ---- merge to 32 x 32 blocks (rows r0+16.., columns r0.., r0 = 0, 32):
+  // X = L21 T11, then T21 = -T22 X
+#pragma unroll
+  for (int e0 = 0; e0 < 512; e0 += kGdnThreads) {
+    const int e = e0 + tid;
+    const int pp = e >> 8, i = (e >> 4) & 15, j = e & 15, r0 = pp * 32;
+    float acc = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2)
+      if (s2 >= j)
+        acc = fmaf(Lm[(r0 + 16 + i) * kLp + r0 + s2], Tm[(r0 + s2) * kLp + r0 + j], acc);
+    Xm[pp * 272 + i * 17 + j] = acc;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int e0 = 0; e0 < 512; e0 += kGdnThreads) {
+    const int e = e0 + tid;
+    const int pp = e >> 8, i = (e >> 4) & 15, j = e & 15, r0 = pp * 32;
+    float acc = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2)
+      if (s2 <= i)
+        acc = fmaf(Tm[(r0 + 16 + i) * kLp + r0 + 16 + s2], Xm[pp * 272 + s2 * 17 + j], acc);
+    Tm[(r0 + 16 + i) * kLp + r0 + j] = -acc;
+  }
+  __syncthreads();
+  // ---- merge to the full 64 x 64 inverse (rows 32.., columns 0..31): warp
+  // w takes rows 4w .. 4w+3 of the 32 x 32 block, lane j its column j
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int j = lane;
+#pragma unroll
+    for (int s4 = 0; s4 < 32; s4 += 4) {
+      float4 l4[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) l4[r] = ld4(Lm + (32 + warp * 4 + r) * kLp + s4);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float tv = s4 + u >= j ? Tm[(s4 + u) * kLp + j] : 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float lv = u == 0 ? l4[r].x : u == 1 ? l4[r].y : u == 2 ? l4[r].z : l4[r].w;
+          acc[r] = fmaf(lv, tv, acc[r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) Xm[(warp * 4 + r) * 33 + j] = acc[r];
+  }
+  __syncthreads();
+  {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int j = lane;
+#pragma unroll
+    for (int s4 = 0; s4 < 32; s4 += 4) {
+      float4 t4[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) t4[r] = ld4(Tm + (32 + warp * 4 + r) * kLp + 32 + s4);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float xv = Xm[(s4 + u) * 33 + j];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float tv = u == 0 ? t4[r].x : u == 1 ? t4[r].y : u == 2 ? t4[r].z : t4[r].w;
+          if (s4 + u <= warp * 4 + r) acc[r] = fmaf(tv, xv, acc[r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) Tm[(32 + warp * 4 + r) * kLp + j] = -acc[r];
+  }
+  __syncthreads();
+}
+
+// M = P T of one sub-chunk (both lower triangular, pitch kLp) into Mm, which
+// may alias the L of unit_lower_inverse (dead by then). The outputs'
+// intra-chunk part is P U = P T RHS = M RHS. Ends with a barrier.
+__device__ __forceinline__ void p_times_t(const float* Pm, const float* Tm, float* Mm, int tid) {
+  // thread (ty, tx) takes rows ty + 16a and columns tx + 16b, b <= a
+  {
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[10];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int r = 0; r < kCt; ++r) {
+      float pv[4], tv[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const int t = ty + 16 * a, s2 = tx + 16 * a;
+        pv[a] = r <= t ? Pm[t * kLp + r] : 0.f;
+        tv[a] = r >= s2 ? Tm[r * kLp + s2] : 0.f;
+      }
+      int i = 0;
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb <= a; ++bb, ++i) acc[i] = fmaf(pv[a], tv[bb], acc[i]);
+    }
+    int i = 0;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const int t = ty + 16 * a, s2 = tx + 16 * bb;
+        float mv = 0.f;
+        if (bb <= a) {
+          if (s2 <= t) mv = acc[i];
+          ++i;
+        }
+        Mm[t * kLp + s2] = mv;
+      }
+  }
+  __syncthreads();
+}
+
+// M = P T of one sub-chunk in 4 x 4 register blocks: Pt holds P transposed
+// (Pt[s][t] = P[t][s], zero for s > t) and Tm is T with zeros above the
+// diagonal; Mm (pitch kLp, may alias the dead L) gets the 136 lower blocks
+// (thread i < 136 takes block i in row-major order of (bt, bs), bs <= bt).
+// Block (bt, bs) needs r in [4 bs, 4 bt + 4); each warp loops over the union
+// of its threads' ranges, the zeros making the extra terms vanish. Ends with
+// a barrier.
+__device__ __forceinline__ void p_times_t_blocked(const float* Pt, const float* Tm, float* Mm,
+                                                  int tid, int warp) {
+  constexpr int kBlocks = (kCt / 4) * (kCt / 4 + 1) / 2;   // 136
+  if (warp * 32 < kBlocks) {
+    int bt = 0, rem = tid < kBlocks ? tid : kBlocks - 1;
+    while (rem > bt) rem -= ++bt;
+    const int bs = rem;
+    // the warp's range: its first block has the smallest bs (0 unless the
+    // warp starts inside row bt), its last the largest bt
+    const int first = warp * 32, last = min(first + 31, kBlocks - 1);
+    int bt_f = 0, rem_f = first;
+    while (rem_f > bt_f) rem_f -= ++bt_f;
+    int bt_l = 0, rem_l = last;
+    while (rem_l > bt_l) rem_l -= ++bt_l;
+    const int r_lo = bt_f == bt_l ? 4 * rem_f : 0, r_hi = 4 * bt_l + 4;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+#pragma unroll 4
+    for (int r = r_lo; r < r_hi; ++r) {
+      const float4 pv = ld4(Pt + r * kLp + 4 * bt);
+      const float4 tv = ld4(Tm + r * kLp + 4 * bs);
+      const float pa[4] = {pv.x, pv.y, pv.z, pv.w}, tb[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(pa[a], tb[c], acc[a][c]);
+    }
+    if (tid < kBlocks) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+        st4(Mm + (4 * bt + a) * kLp + 4 * bs, make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]));
+    }
+  }
+  __syncthreads();
+}
+
+// Prep of the CUDA-core path (D = 64): one CTA per (stream, head,
+// sub-chunk), T = (I + L)^-1 and M = scale P T of the sub-chunk into the
+// workspace, both [64][64] row-major, zero above the diagonal.
+template <int D, typename T>
 __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_constant__ GdnParams p) {
   using L = GdnPrepSmem<D>;
   constexpr int KP = L::KP;
@@ -279,215 +468,57 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_c
   // the call's device status word starts at zero (the prep kernel runs first)
   if (j == 0 && h == 0 && z == 0 && tid == 0) *reinterpret_cast<int*>(p.workspace) = 0;
   const size_t blk = ((size_t)z * H + h) * (size_t)p.n_sub + (size_t)j;
-  unsigned char* img = reinterpret_cast<unsigned char*>(p.workspace) + kWsHeader + blk * kImgBytes;
-  if constexpr (kImg) {
-    // the KQ image (before the key and query rows are reused below)
-    if (SA_BOUNDS(blk < (size_t)p.n_streams * H * (size_t)p.n_sub, 1)) {
-      for (int e = tid; e < 2 * kCt * (D / 8); e += kGdnThreads) {
-        const int r = e / (D / 8), cc = e % (D / 8), panel = cc >> 3, c = cc & 7;
-        const float* src = (r < kCt ? Kh + r * KP : Qh + (r - kCt) * KP) + cc * 8;
-        uint4 hi, lo;
-        split8(src, hi, lo);
-        const uint32_t off = (uint32_t)panel * (kImgKQ / 2) + sw128_off(r, c);
-        *reinterpret_cast<uint4*>(img + off) = hi;
-        *reinterpret_cast<uint4*>(img + kImgKQ + off) = lo;
-      }
-    }
-  }
 
-    // ---- Gram matrices on the lower triangle -> L and P. Thread (ty, tx)
-    // takes rows ty + 16a and columns tx + 16b, b <= a (the pairs a < b lie
-    // above the diagonal).
-    {
-      const int ty = tid >> 4, tx = tid & 15;
-      float akk[10], aqk[10];
-#pragma unroll
-      for (int i = 0; i < 10; ++i) akk[i] = aqk[i] = 0.f;
-#pragma unroll 2
-      for (int d = 0; d < D; d += 4) {
-        float4 kr[4], qr[4], kc[4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          kr[a] = ld4(Kh + (ty + 16 * a) * KP + d);
-          qr[a] = ld4(Qh + (ty + 16 * a) * KP + d);
-          kc[a] = ld4(Kh + (tx + 16 * a) * KP + d);
-        }
-        int i = 0;
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int bb = 0; bb <= a; ++bb, ++i) {
-            akk[i] = dot4(kr[a], kc[bb], akk[i]);
-            aqk[i] = dot4(qr[a], kc[bb], aqk[i]);
-          }
-      }
-      int i = 0;
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          const int t = ty + 16 * a, s = tx + 16 * bb;
-          float lv = 0.f, pv = 0.f;
-          if (bb <= a) {
-            if (s <= t) {
-              const float e = ex2f(gcum(t) - gcum(s));
-              if (s < t) lv = Bs[t] * e * akk[i];
-              pv = p.scale * e * aqk[i];
-            }
-            ++i;
-          }
-          Lm[t * kLp + s] = lv;
-          Pm[t * kLp + s] = pv;
-        }
-    }
-    __syncthreads();
-
-    // ---- diagonal 16 x 16 blocks of (I + L)^-1: thread (blk, j) solves for
-    // column j of its block
-    if (tid < 64) {
-      const int r0 = (tid >> 4) * 16, j = tid & 15;
-      float x[16];
-#pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        float acc = 0.f;
-#pragma unroll
-        for (int s2 = 0; s2 < t; ++s2) acc = fmaf(Lm[(r0 + t) * kLp + r0 + s2], x[s2], acc);
-        x[t] = t < j ? 0.f : (t == j ? 1.f : -acc);
-      }
-#pragma unroll
-      for (int t = 0; t < 16; ++t) Tm[(r0 + t) * kLp + r0 + j] = x[t];
-    }
-    __syncthreads();
-
-    // ---- merge to 32 x 32 blocks (rows r0+16.., columns r0.., r0 = 0, 32):
-    // X = L21 T11, then T21 = -T22 X
-#pragma unroll
-    for (int e0 = 0; e0 < 512; e0 += kGdnThreads) {
-      const int e = e0 + tid;
-      const int pp = e >> 8, i = (e >> 4) & 15, j = e & 15, r0 = pp * 32;
-      float acc = 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2)
-        if (s2 >= j)
-          acc = fmaf(Lm[(r0 + 16 + i) * kLp + r0 + s2], Tm[(r0 + s2) * kLp + r0 + j], acc);
-      Xm[pp * 272 + i * 17 + j] = acc;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int e0 = 0; e0 < 512; e0 += kGdnThreads) {
-      const int e = e0 + tid;
-      const int pp = e >> 8, i = (e >> 4) & 15, j = e & 15, r0 = pp * 32;
-      float acc = 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2)
-        if (s2 <= i)
-          acc = fmaf(Tm[(r0 + 16 + i) * kLp + r0 + 16 + s2], Xm[pp * 272 + s2 * 17 + j], acc);
-      Tm[(r0 + 16 + i) * kLp + r0 + j] = -acc;
-    }
-    __syncthreads();
-    // ---- merge to the full 64 x 64 inverse (rows 32.., columns 0..31): warp
-    // w takes rows 4w .. 4w+3 of the 32 x 32 block, lane j its column j
-    {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int j = lane;
-#pragma unroll
-      for (int s4 = 0; s4 < 32; s4 += 4) {
-        float4 l4[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) l4[r] = ld4(Lm + (32 + warp * 4 + r) * kLp + s4);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float tv = s4 + u >= j ? Tm[(s4 + u) * kLp + j] : 0.f;
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const float lv = u == 0 ? l4[r].x : u == 1 ? l4[r].y : u == 2 ? l4[r].z : l4[r].w;
-            acc[r] = fmaf(lv, tv, acc[r]);
-          }
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) Xm[(warp * 4 + r) * 33 + j] = acc[r];
-    }
-    __syncthreads();
-    {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int j = lane;
-#pragma unroll
-      for (int s4 = 0; s4 < 32; s4 += 4) {
-        float4 t4[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) t4[r] = ld4(Tm + (32 + warp * 4 + r) * kLp + 32 + s4);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float xv = Xm[(s4 + u) * 33 + j];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const float tv = u == 0 ? t4[r].x : u == 1 ? t4[r].y : u == 2 ? t4[r].z : t4[r].w;
-            if (s4 + u <= warp * 4 + r) acc[r] = fmaf(tv, xv, acc[r]);
-          }
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) Tm[(32 + warp * 4 + r) * kLp + j] = -acc[r];
-    }
-    __syncthreads();
-
-  // ---- M = P T (lower triangular; L is no longer needed, M takes its place).
-  // The outputs' intra-chunk part is P U = P T RHS = M RHS. Thread (ty, tx)
-  // takes rows ty + 16a and columns tx + 16b, b <= a.
+  // ---- Gram matrices on the lower triangle -> L and P. Thread (ty, tx)
+  // takes rows ty + 16a and columns tx + 16b, b <= a (the pairs a < b lie
+  // above the diagonal).
   {
-    float* Mm = Lm;
     const int ty = tid >> 4, tx = tid & 15;
-    float acc[10];
+    float akk[10], aqk[10];
 #pragma unroll
-    for (int i = 0; i < 10; ++i) acc[i] = 0.f;
-#pragma unroll 4
-    for (int r = 0; r < kCt; ++r) {
-      float pv[4], tv[4];
+    for (int i = 0; i < 10; ++i) akk[i] = aqk[i] = 0.f;
+#pragma unroll 2
+    for (int d = 0; d < D; d += 4) {
+      float4 kr[4], qr[4], kc[4];
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
-        const int t = ty + 16 * a, s2 = tx + 16 * a;
-        pv[a] = r <= t ? Pm[t * kLp + r] : 0.f;
-        tv[a] = r >= s2 ? Tm[r * kLp + s2] : 0.f;
+        kr[a] = ld4(Kh + (ty + 16 * a) * KP + d);
+        qr[a] = ld4(Qh + (ty + 16 * a) * KP + d);
+        kc[a] = ld4(Kh + (tx + 16 * a) * KP + d);
       }
       int i = 0;
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int bb = 0; bb <= a; ++bb, ++i) acc[i] = fmaf(pv[a], tv[bb], acc[i]);
+        for (int bb = 0; bb <= a; ++bb, ++i) {
+          akk[i] = dot4(kr[a], kc[bb], akk[i]);
+          aqk[i] = dot4(qr[a], kc[bb], aqk[i]);
+        }
     }
-    int i = 0;   // (the last reads of L were in the merges, before the barrier above)
+    int i = 0;
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int bb = 0; bb < 4; ++bb) {
-        const int t = ty + 16 * a, s2 = tx + 16 * bb;
-        float mv = 0.f;
+        const int t = ty + 16 * a, s = tx + 16 * bb;
+        float lv = 0.f, pv = 0.f;
         if (bb <= a) {
-          if (s2 <= t) mv = acc[i];
+          if (s <= t) {
+            const float e = ex2f(gcum(t) - gcum(s));
+            if (s < t) lv = Bs[t] * e * akk[i];
+            pv = p.scale * e * aqk[i];
+          }
           ++i;
         }
-        Mm[t * kLp + s2] = mv;
+        Lm[t * kLp + s] = lv;
+        Pm[t * kLp + s] = pv;
       }
   }
   __syncthreads();
+  unit_lower_inverse(Lm, Tm, Xm, tid, warp, lane);
+  p_times_t(Pm, Tm, Lm, tid);
 
-  if constexpr (kImg) {
-    // ---- the TM image: T rows then M rows, zero above the diagonal
-    if (!SA_BOUNDS(blk < (size_t)p.n_streams * H * (size_t)p.n_sub, 1)) return;
-    for (int e = tid; e < 2 * kCt * (kCt / 8); e += kGdnThreads) {
-      const int r = e / (kCt / 8), c = e % (kCt / 8), row = r & (kCt - 1);
-      const float* src = (r < kCt ? Tm : Lm) + row * kLp + c * 8;
-      float x[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = c * 8 + i <= row ? src[i] : 0.f;
-      uint4 hi, lo;
-      split8(x, hi, lo);
-      const uint32_t off = 2 * kImgKQ + sw128_off(r, c);
-      *reinterpret_cast<uint4*>(img + off) = hi;
-      *reinterpret_cast<uint4*>(img + kImgTM + off) = lo;
-    }
-  } else {
+  {
     // ---- T and M to the workspace, zero above the diagonal
     float* dst = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(p.workspace) + kWsHeader) +
                  blk * kTpFloats;
@@ -501,6 +532,230 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_c
       if (c4 + 3 > row) x.w = 0.f;
       *reinterpret_cast<float4*>(dst + mat * kCt * kCt + row * kCt + c4) = x;
     }
+  }
+}
+
+// Shared memory of gdn_prep_tc_kernel (bytes from a 1024-byte-aligned base:
+// the 128-byte-swizzled image needs it).
+struct GdnPrepTcSmem {
+  static constexpr uint32_t img = 0;                   // [hi, lo] KQ image; later T and merge scratch
+  static constexpr uint32_t lm = 2 * kImgKQ;           // [64][68] f32 L, later M
+  static constexpr uint32_t pm = lm + kCt * kLp * 4;   // [64][68] f32 P
+  static constexpr uint32_t gs = pm + kCt * kLp * 4;   // [64] in-warp prefix sums of g log2(e)
+  static constexpr uint32_t bs = gs + kCt * 4;         // [64] beta
+  static constexpr uint32_t bar = bs + kCt * 4;        // mbarrier of the Gram MMA
+  static constexpr uint32_t misc = bar + 8;            // TMEM base address; a word never set
+  static constexpr uint32_t bytes = misc + 8;
+  static_assert(kCt * kLp * 4 + 32 * 33 * 4 <= 2 * kImgKQ, "T and the merge scratch fit in the image");
+};
+constexpr uint64_t kPrepTimeoutNs = 1000000000ull;
+
+// Four floats as bf16 hi = bf16(x) and lo = bf16(x - hi), each packed into 8 bytes.
+__device__ __forceinline__ void split4(float4 x, uint2& hi, uint2& lo) {
+  const float v[4] = {x.x, x.y, x.z, x.w};
+  uint32_t h[2], l[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    h[i] = *reinterpret_cast<uint32_t*>(&b);
+    __nv_bfloat162 c = __floats2bfloat162_rn(v[2 * i] - __uint_as_float(h[i] << 16),
+                                             v[2 * i + 1] - __uint_as_float(h[i] & 0xffff0000u));
+    l[i] = *reinterpret_cast<uint32_t*>(&c);
+  }
+  hi = make_uint2(h[0], h[1]);
+  lo = make_uint2(l[0], l[1]);
+}
+
+// Prep of the tensor-core path (D = 128): one CTA per (stream, head,
+// sub-chunk), computing the same T = (I + L)^-1 and M = scale P T as
+// gdn_prep_kernel, with the Gram matrices on the tensor core. The normalised
+// key and query rows are split into bf16 hi and lo and written once, as the
+// KQ operand image, to shared memory and to the workspace; one thread issues
+// [K^;Q^] K^T (128 x 64, fp32 in TMEM) as the three-term split product over
+// that image (the product the sequential pass uses for its own contractions,
+// about 2^-16 relative per term); the threads read it back and form L and P
+// (key rows and query rows of the product). Then T, M and the TM image.
+template <typename T>
+__global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_tc_kernel(const __grid_constant__ GdnParams p) {
+  constexpr int D = 128;
+  using L = GdnPrepTcSmem;
+  extern __shared__ __align__(1024) unsigned char smp[];
+  int* status = reinterpret_cast<int*>(p.workspace);
+  const uint32_t base = ptx::smem_u32(smp);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j = blockIdx.x, h = blockIdx.y, z = blockIdx.z, b = p.stream_of[z];
+  const int H = p.H;
+  const int64_t Tn = p.T;
+  const int64_t t0 = (int64_t)j * kCt;
+  const int n = (int)(Tn - t0 < kCt ? Tn - t0 : kCt);
+  // (block-uniform: the whole block leaves before any barrier)
+  if (!SA_BOUNDS(b >= 0 && b < p.batch && z < p.n_streams && j < p.n_sub && n > 0, 0)) return;
+  // the call's device status word starts at zero (the prep kernel runs first)
+  if (j == 0 && h == 0 && z == 0 && tid == 0) *status = 0;
+  if (base & 1023u) {
+    if (tid == 0) atomicOr(status, kDeviceErrTimeout);
+    return;
+  }
+  float* Lm = reinterpret_cast<float*>(smp + L::lm);
+  float* Pm = reinterpret_cast<float*>(smp + L::pm);
+  float* Gs = reinterpret_cast<float*>(smp + L::gs);
+  float* Bs = reinterpret_cast<float*>(smp + L::bs);
+  float* Tm = reinterpret_cast<float*>(smp + L::img);   // after the Gram MMA has read the image
+  float* Xm = Tm + kCt * kLp;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smp + L::misc);
+  volatile int* no_abort = reinterpret_cast<volatile int*>(smp + L::misc + 4);
+  const uint32_t bar = base + L::bar;
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 64);
+    ptx::tmem_relinquish();
+  }
+  if (tid == 0) {
+    ptx::mbar_init(bar, 1);
+    *no_abort = 0;
+    ptx::fence_mbar_init();
+  }
+  const T* q = static_cast<const T*>(p.q);
+  const T* k = static_cast<const T*>(p.k);
+  const size_t tok_stride = (size_t)H * D;
+  const size_t row0 = ((size_t)b * (size_t)Tn + (size_t)t0) * tok_stride + (size_t)h * D;
+  const size_t g0 = ((size_t)b * (size_t)Tn + (size_t)t0) * H + h;
+  const size_t blk = ((size_t)z * H + h) * (size_t)p.n_sub + (size_t)j;
+  const bool blk_ok = SA_BOUNDS(blk < (size_t)p.n_streams * H * (size_t)p.n_sub, 1);
+  unsigned char* img_g = reinterpret_cast<unsigned char*>(p.workspace) + kWsHeader + blk * kImgBytes;
+  auto gcum = [&](int t) -> float { return Gs[t] + (t >= 32 ? Gs[31] : 0.f); };
+
+  // ---- rows: warp w normalises key and query rows w + 8i (i < 8); lane l
+  // holds columns 4l .. 4l + 3, one half of the image's 16-byte chunk l / 2
+  // (chunks 0..7 in panel 0, 8..15 in panel 1); rows past n are zero. All
+  // loads (and the gates') are issued before any is used.
+  float gv = 0.f, bv = 0.f;
+  if (tid < n) {
+    gv = p.g[g0 + (size_t)tid * H];
+    bv = p.beta[g0 + (size_t)tid * H];
+  }
+  float4 kr[8], qr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = warp + 8 * i;
+    kr[i] = qr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < n) {
+      kr[i] = ld_raw4(k + row0 + (size_t)r * tok_stride + 4 * lane);
+      qr[i] = ld_raw4(q + row0 + (size_t)r * tok_stride + 4 * lane);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = warp + 8 * i;
+    const float4 kx = kr[i], qx = qr[i];
+    float sk = dot4(kx, kx, 0.f), sq = dot4(qx, qx, 0.f);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sk += __shfl_xor_sync(0xffffffffu, sk, o);
+      sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    }
+    const float ik = sk > 0.f ? rsqrtf(sk) : 0.f;
+    const float iq = sq > 0.f ? rsqrtf(sq) : 0.f;
+    uint2 kh, kl, qh, ql;
+    split4(make_float4(kx.x * ik, kx.y * ik, kx.z * ik, kx.w * ik), kh, kl);
+    split4(make_float4(qx.x * iq, qx.y * iq, qx.z * iq, qx.w * iq), qh, ql);
+    const int cc = lane >> 1;
+    const uint32_t in = (uint32_t)(cc >> 3) * (kImgKQ / 2) + (uint32_t)(lane & 1) * 8;
+    const uint32_t ok_ = in + sw128_off(r, cc & 7), oq = in + sw128_off(kCt + r, cc & 7);
+    *reinterpret_cast<uint2*>(smp + L::img + ok_) = kh;
+    *reinterpret_cast<uint2*>(smp + L::img + kImgKQ + ok_) = kl;
+    *reinterpret_cast<uint2*>(smp + L::img + oq) = qh;
+    *reinterpret_cast<uint2*>(smp + L::img + kImgKQ + oq) = ql;
+    if (blk_ok) {
+      *reinterpret_cast<uint2*>(img_g + ok_) = kh;
+      *reinterpret_cast<uint2*>(img_g + kImgKQ + ok_) = kl;
+      *reinterpret_cast<uint2*>(img_g + oq) = qh;
+      *reinterpret_cast<uint2*>(img_g + kImgKQ + oq) = ql;
+    }
+  }
+  if (tid < kCt) gate_scan(gv, bv, Gs, Bs, tid, lane);
+  ptx::fence_proxy_async_smem();   // the image, written by the threads, is read by the MMA
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- [K^;Q^] K^T: A = all 128 image rows, B = the 64 key rows, both
+  // K-major (two panels of 64 key dims); terms (hi, hi), (hi, lo), (lo, hi)
+  if (tid == 0) {
+    constexpr uint32_t id = ptx::idesc_bf16_f32_ab(128, kCt, false, false);
+    constexpr uint32_t ta[3] = {0, 0, 1}, tb[3] = {0, 1, 0};
+    const uint64_t d0 = ptx::sdesc_sw128(base + L::img, 16, 1024);
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (uint32_t)(kk >> 2) * (kImgKQ / 2) + (uint32_t)(kk & 3) * 32;
+        ptx::umma_ss(tmem, ptx::sdesc_add(d0, ta[i] * kImgKQ + koff),
+                     ptx::sdesc_add(d0, tb[i] * kImgKQ + koff), id, (i > 0 || kk > 0) ? 1u : 0u);
+      }
+    ptx::umma_commit(bar);
+  }
+  const bool done = __syncthreads_and(ptx::mbar_wait(bar, 0, no_abort, kPrepTimeoutNs));
+  ptx::tc_fence_after();
+  if (done) {
+    // TMEM lane 32 (w mod 4) + l is product row `row` (key rows 0..63 give
+    // L, query rows 64..127 give P); warps 0-3 read columns 0..31, 4-7 32..63
+    float x[32];
+    ptx::tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(32 * (warp >> 2)), x);
+    ptx::tmem_wait_ld();
+    const int row = 32 * (warp & 3) + lane, t = row & (kCt - 1), s0 = 32 * (warp >> 2);
+    const bool isq = row >= kCt;
+    const float gt = gcum(t), mul = isq ? p.scale : Bs[t];
+    if (!isq) {
+      // L row-major
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int s = s0 + 4 * c4 + e;
+          o[e] = s < t ? mul * ex2f(gt - gcum(s)) * x[4 * c4 + e] : 0.f;
+        }
+        st4(Lm + t * kLp + s0 + 4 * c4, make_float4(o[0], o[1], o[2], o[3]));
+      }
+    } else {
+      // P transposed (Pm[s][t]): the lanes of a warp hold consecutive t
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int s = s0 + e;
+        Pm[s * kLp + t] = s <= t ? mul * ex2f(gt - gcum(s)) * x[e] : 0.f;
+      }
+    }
+    // T's 16 x 16 blocks above the diagonal, which the inverse leaves
+    // untouched, are zero (the blocked M = P T reads whole 4 x 4 blocks)
+    for (int e = tid; e < kCt * kCt; e += kGdnThreads) {
+      const int r = e >> 6, c = e & (kCt - 1);
+      if ((c >> 4) > (r >> 4)) Tm[r * kLp + c] = 0.f;
+    }
+  } else if (tid == 0) {
+    atomicOr(status, kDeviceErrTimeout);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 64);
+  if (!done) return;
+
+  unit_lower_inverse(Lm, Tm, Xm, tid, warp, lane);
+  p_times_t_blocked(Pm, Tm, Lm, tid, warp);
+
+  // ---- the TM image: T rows then M rows, zero above the diagonal
+  if (!blk_ok) return;
+  for (int e = tid; e < 2 * kCt * (kCt / 8); e += kGdnThreads) {
+    const int r = e / (kCt / 8), c = e % (kCt / 8), row = r & (kCt - 1);
+    const float* src = (r < kCt ? Tm : Lm) + row * kLp + c * 8;
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = c * 8 + i <= row ? src[i] : 0.f;
+    uint4 hi, lo;
+    split8(x, hi, lo);
+    const uint32_t off = 2 * kImgKQ + sw128_off(r, c);
+    *reinterpret_cast<uint4*>(img_g + off) = hi;
+    *reinterpret_cast<uint4*>(img_g + kImgTM + off) = lo;
   }
 }
 
@@ -943,6 +1198,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
       constexpr uint32_t id_mm = ptx::idesc_bf16_f32_ab(128, kTcSlice, true, true);
       // split-product term i: (A part, B part) = (hi, hi), (hi, lo), (lo, hi)
       constexpr uint32_t ta[3] = {0, 0, 1}, tb[3] = {0, 1, 0};
+      // base descriptors of the fixed operand buffers (MN-major images have
+      // their 64-column panels 16 KiB apart, rows 8 x 128 bytes per core group)
+      const uint64_t d_st = ptx::sdesc_sw128(base + L::st, 16384, 1024);
+      const uint64_t d_tm = ptx::sdesc_sw128(base + L::tm, 16, 1024);
+      const uint64_t d_rhs = ptx::sdesc_sw128(base + L::rhs, 16384, 1024);
+      const uint64_t d_uu = ptx::sdesc_sw128(base + L::uu, 16384, 1024);
       int kq_issued = 0, kq_done = 0, tm_issued = 0;
       load_kq(0);
       ++kq_issued;
@@ -964,16 +1225,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
         ++kq_done;
         ptx::tc_fence_after();
         // MMA1: [K^;Q^] (K-major, 2 panels of 64 key dims) x S image (MN-major)
+        const uint64_t a1 = ptx::sdesc_sw128(kqb, 16, 1024);
 #pragma unroll
         for (int i = 0; i < 3; ++i)
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a = ptx::sdesc_sw128(kqb + ta[i] * kImgKQ + (uint32_t)(kk >> 2) * 16384 +
-                                                    (uint32_t)(kk & 3) * 32, 16, 1024);
-            const uint64_t bd =
-                ptx::sdesc_sw128(base + L::st + tb[i] * 16384 + (uint32_t)kk * 2048, 16384, 1024);
-            ptx::umma_ss(t_d1, a, bd, id_kk, (i > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            ptx::umma_ss(t_d1,
+                         ptx::sdesc_add(a1, ta[i] * kImgKQ + (uint32_t)(kk >> 2) * 16384 +
+                                                (uint32_t)(kk & 3) * 32),
+                         ptx::sdesc_add(d_st, tb[i] * 16384 + (uint32_t)kk * 2048), id_kk,
+                         (i > 0 || kk > 0) ? 1u : 0u);
         ptx::umma_commit(bar(L::B_D1));
         if (!ptx::mbar_wait(bar(L::B_TM), par, abort_flag, kTcTimeoutNs) ||
             !ptx::mbar_wait(bar(L::B_RHS), par, abort_flag, kTcTimeoutNs)) {
@@ -985,13 +1246,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
 #pragma unroll
         for (int i = 0; i < 3; ++i)
 #pragma unroll
-          for (int kk = 0; kk < kCt / 16; ++kk) {
-            const uint64_t a =
-                ptx::sdesc_sw128(base + L::tm + ta[i] * kImgTM + (uint32_t)kk * 32, 16, 1024);
-            const uint64_t bd =
-                ptx::sdesc_sw128(base + L::rhs + tb[i] * 8192 + (uint32_t)kk * 2048, 16384, 1024);
-            ptx::umma_ss(t_d2, a, bd, id_kk, (i > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kCt / 16; ++kk)
+            ptx::umma_ss(t_d2, ptx::sdesc_add(d_tm, ta[i] * kImgTM + (uint32_t)kk * 32),
+                         ptx::sdesc_add(d_rhs, tb[i] * 8192 + (uint32_t)kk * 2048), id_kk,
+                         (i > 0 || kk > 0) ? 1u : 0u);
         ptx::umma_commit(bar(L::B_D2));
         // the TM buffer is free once MMA2 has read it
         if (!ptx::mbar_wait(bar(L::B_D2), par, abort_flag, kTcTimeoutNs)) {
@@ -1009,16 +1267,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
         ptx::tc_fence_after();
         // MMA3: ST += K^ (the key rows of KQ as the MN-major A: 2 panels of 64
         // key dims LBO apart, 64 token rows) x U~ image (MN-major)
+        const uint64_t a3 = ptx::sdesc_sw128(kqb, 16384, 1024);
 #pragma unroll
         for (int i = 0; i < 3; ++i)
 #pragma unroll
-          for (int kk = 0; kk < kCt / 16; ++kk) {
-            const uint64_t a =
-                ptx::sdesc_sw128(kqb + ta[i] * kImgKQ + (uint32_t)kk * 2048, 16384, 1024);
-            const uint64_t bd =
-                ptx::sdesc_sw128(base + L::uu + tb[i] * 8192 + (uint32_t)kk * 2048, 16384, 1024);
-            ptx::umma_ss(t_st, a, bd, id_mm, 1u);
-          }
+          for (int kk = 0; kk < kCt / 16; ++kk)
+            ptx::umma_ss(t_st, ptx::sdesc_add(a3, ta[i] * kImgKQ + (uint32_t)kk * 2048),
+                         ptx::sdesc_add(d_uu, tb[i] * 8192 + (uint32_t)kk * 2048), id_mm, 1u);
         ptx::umma_commit(bar(L::B_D3));
         // the KQ buffer of j is free once MMA3 has read it
         if (j + 2 < nsub) {
@@ -1189,7 +1444,7 @@ template <int D, typename T>
 cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
   constexpr bool kTc = D == 128;
   constexpr size_t smem = kTc ? GdnTcSmem::bytes : GdnSmem<D, T>::bytes;
-  constexpr size_t psmem = GdnPrepSmem<D>::bytes;
+  constexpr size_t psmem = kTc ? (size_t)GdnPrepTcSmem::bytes : GdnPrepSmem<D>::bytes;
   static unsigned configured = 0;   // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1201,13 +1456,21 @@ cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
     else
       e = cudaFuncSetAttribute(gdn_chunk_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gdn_prep_kernel<D, T, kTc>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    if (e == cudaSuccess) {
+      if constexpr (kTc)
+        e = cudaFuncSetAttribute(gdn_prep_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)psmem);
+      else
+        e = cudaFuncSetAttribute(gdn_prep_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)psmem);
+    }
     if (e != cudaSuccess) return e;
     if (dev < 32) configured |= 1u << dev;
   }
-  gdn_prep_kernel<D, T, kTc><<<dim3(p.n_sub, p.H, p.n_streams), kGdnThreads, psmem, st>>>(p);
+  if constexpr (kTc)
+    gdn_prep_tc_kernel<T><<<dim3(p.n_sub, p.H, p.n_streams), kGdnThreads, psmem, st>>>(p);
+  else
+    gdn_prep_kernel<D, T><<<dim3(p.n_sub, p.H, p.n_streams), kGdnThreads, psmem, st>>>(p);
   if constexpr (kTc)
     gdn_tc_kernel<T><<<dim3(D / kTcSlice, p.H, p.n_streams), kTcThreads, smem, st>>>(p);
   else

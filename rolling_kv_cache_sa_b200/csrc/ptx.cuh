@@ -271,6 +271,16 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// The descriptor d moved by `bytes` (a multiple of 16) in shared memory. The
+// start address is the low 14-bit field (address >> 4); shared-memory
+// addresses stay below 2^18, so the sum never carries out of that field.
+// Stepping one base descriptor this way keeps the per-MMA work to one add,
+// where building each descriptor from its address costs a dependent chain
+// in front of every MMA issue.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) {
+  return d + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, dense.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
 //   15 A major (0 = K), 16 B major (1 = MN), 17-22 N >> 3, 24-28 M >> 4.
