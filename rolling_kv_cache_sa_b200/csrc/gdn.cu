@@ -538,16 +538,21 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_kernel(const __grid_c
 // Shared memory of gdn_prep_tc_kernel (bytes from a 1024-byte-aligned base:
 // the 128-byte-swizzled image needs it).
 struct GdnPrepTcSmem {
-  static constexpr uint32_t img = 0;                   // [hi, lo] KQ image; later T and merge scratch
-  static constexpr uint32_t lm = 2 * kImgKQ;           // [64][68] f32 L, later M
-  static constexpr uint32_t pm = lm + kCt * kLp * 4;   // [64][68] f32 P
-  static constexpr uint32_t gs = pm + kCt * kLp * 4;   // [64] in-warp prefix sums of g log2(e)
+  static constexpr uint32_t img = 0;                   // [hi, lo] KQ image, read by the Gram MMA
+  // once the MMA has completed, the image region holds:
+  static constexpr uint32_t lm = 0;                    // [64][68] f32 L, later M
+  static constexpr uint32_t pm = lm + kCt * kLp * 4;   // [64][68] f32 P, transposed
+  static constexpr uint32_t tm = pm + kCt * kLp * 4;   // [64][68] f32 T
+  static constexpr uint32_t xm = tm + kCt * kLp * 4;   // [32][33] f32 merge scratch
+  static constexpr uint32_t gs = 2 * kImgKQ;           // [64] in-warp prefix sums of g log2(e)
   static constexpr uint32_t bs = gs + kCt * 4;         // [64] beta
   static constexpr uint32_t bar = bs + kCt * 4;        // mbarrier of the Gram MMA
   static constexpr uint32_t misc = bar + 8;            // TMEM base address; a word never set
   static constexpr uint32_t bytes = misc + 8;
-  static_assert(kCt * kLp * 4 + 32 * 33 * 4 <= 2 * kImgKQ, "T and the merge scratch fit in the image");
+  static_assert(xm + 32 * 33 * 4 <= 2 * kImgKQ, "L, P, T and the merge scratch fit in the image");
 };
+// three CTAs per SM: 3 x 66 KB of shared memory, 3 x 64 TMEM columns
+constexpr int kPrepTcCtasPerSm = 3;
 constexpr uint64_t kPrepTimeoutNs = 1000000000ull;
 
 // Four floats as bf16 hi = bf16(x) and lo = bf16(x - hi), each packed into 8 bytes.
@@ -576,7 +581,8 @@ __device__ __forceinline__ void split4(float4 x, uint2& hi, uint2& lo) {
 // about 2^-16 relative per term); the threads read it back and form L and P
 // (key rows and query rows of the product). Then T, M and the TM image.
 template <typename T>
-__global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_tc_kernel(const __grid_constant__ GdnParams p) {
+__global__ void __launch_bounds__(kGdnThreads, kPrepTcCtasPerSm)
+    gdn_prep_tc_kernel(const __grid_constant__ GdnParams p) {
   constexpr int D = 128;
   using L = GdnPrepTcSmem;
   extern __shared__ __align__(1024) unsigned char smp[];
@@ -600,8 +606,8 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_tc_kernel(const __gri
   float* Pm = reinterpret_cast<float*>(smp + L::pm);
   float* Gs = reinterpret_cast<float*>(smp + L::gs);
   float* Bs = reinterpret_cast<float*>(smp + L::bs);
-  float* Tm = reinterpret_cast<float*>(smp + L::img);   // after the Gram MMA has read the image
-  float* Xm = Tm + kCt * kLp;
+  float* Tm = reinterpret_cast<float*>(smp + L::tm);
+  float* Xm = reinterpret_cast<float*>(smp + L::xm);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smp + L::misc);
   volatile int* no_abort = reinterpret_cast<volatile int*>(smp + L::misc + 4);
   const uint32_t bar = base + L::bar;
@@ -633,43 +639,49 @@ __global__ void __launch_bounds__(kGdnThreads, 2) gdn_prep_tc_kernel(const __gri
     gv = p.g[g0 + (size_t)tid * H];
     bv = p.beta[g0 + (size_t)tid * H];
   }
-  float4 kr[8], qr[8];
+  // rows in two batches of four (within the register budget of three CTAs
+  // per SM)
+  constexpr int kB = 4;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = warp + 8 * i;
-    kr[i] = qr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < n) {
-      kr[i] = ld_raw4(k + row0 + (size_t)r * tok_stride + 4 * lane);
-      qr[i] = ld_raw4(q + row0 + (size_t)r * tok_stride + 4 * lane);
+  for (int i0 = 0; i0 < 8; i0 += kB) {
+    float4 kr[kB], qr[kB];
+#pragma unroll
+    for (int i = 0; i < kB; ++i) {
+      const int r = warp + 8 * (i0 + i);
+      kr[i] = qr[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < n) {
+        kr[i] = ld_raw4(k + row0 + (size_t)r * tok_stride + 4 * lane);
+        qr[i] = ld_raw4(q + row0 + (size_t)r * tok_stride + 4 * lane);
+      }
     }
-  }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = warp + 8 * i;
-    const float4 kx = kr[i], qx = qr[i];
-    float sk = dot4(kx, kx, 0.f), sq = dot4(qx, qx, 0.f);
+    for (int i = 0; i < kB; ++i) {
+      const int r = warp + 8 * (i0 + i);
+      const float4 kx = kr[i], qx = qr[i];
+      float sk = dot4(kx, kx, 0.f), sq = dot4(qx, qx, 0.f);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sk += __shfl_xor_sync(0xffffffffu, sk, o);
-      sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    }
-    const float ik = sk > 0.f ? rsqrtf(sk) : 0.f;
-    const float iq = sq > 0.f ? rsqrtf(sq) : 0.f;
-    uint2 kh, kl, qh, ql;
-    split4(make_float4(kx.x * ik, kx.y * ik, kx.z * ik, kx.w * ik), kh, kl);
-    split4(make_float4(qx.x * iq, qx.y * iq, qx.z * iq, qx.w * iq), qh, ql);
-    const int cc = lane >> 1;
-    const uint32_t in = (uint32_t)(cc >> 3) * (kImgKQ / 2) + (uint32_t)(lane & 1) * 8;
-    const uint32_t ok_ = in + sw128_off(r, cc & 7), oq = in + sw128_off(kCt + r, cc & 7);
-    *reinterpret_cast<uint2*>(smp + L::img + ok_) = kh;
-    *reinterpret_cast<uint2*>(smp + L::img + kImgKQ + ok_) = kl;
-    *reinterpret_cast<uint2*>(smp + L::img + oq) = qh;
-    *reinterpret_cast<uint2*>(smp + L::img + kImgKQ + oq) = ql;
-    if (blk_ok) {
-      *reinterpret_cast<uint2*>(img_g + ok_) = kh;
-      *reinterpret_cast<uint2*>(img_g + kImgKQ + ok_) = kl;
-      *reinterpret_cast<uint2*>(img_g + oq) = qh;
-      *reinterpret_cast<uint2*>(img_g + kImgKQ + oq) = ql;
+      for (int o = 16; o > 0; o >>= 1) {
+        sk += __shfl_xor_sync(0xffffffffu, sk, o);
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      }
+      const float ik = sk > 0.f ? rsqrtf(sk) : 0.f;
+      const float iq = sq > 0.f ? rsqrtf(sq) : 0.f;
+      uint2 kh, kl, qh, ql;
+      split4(make_float4(kx.x * ik, kx.y * ik, kx.z * ik, kx.w * ik), kh, kl);
+      split4(make_float4(qx.x * iq, qx.y * iq, qx.z * iq, qx.w * iq), qh, ql);
+      const int cc = lane >> 1;
+      const uint32_t in = (uint32_t)(cc >> 3) * (kImgKQ / 2) + (uint32_t)(lane & 1) * 8;
+      const uint32_t ok_ = in + sw128_off(r, cc & 7), oq = in + sw128_off(kCt + r, cc & 7);
+      *reinterpret_cast<uint2*>(smp + L::img + ok_) = kh;
+      *reinterpret_cast<uint2*>(smp + L::img + kImgKQ + ok_) = kl;
+      *reinterpret_cast<uint2*>(smp + L::img + oq) = qh;
+      *reinterpret_cast<uint2*>(smp + L::img + kImgKQ + oq) = ql;
+      if (blk_ok) {
+        *reinterpret_cast<uint2*>(img_g + ok_) = kh;
+        *reinterpret_cast<uint2*>(img_g + kImgKQ + ok_) = kl;
+        *reinterpret_cast<uint2*>(img_g + oq) = qh;
+        *reinterpret_cast<uint2*>(img_g + kImgKQ + oq) = ql;
+      }
     }
   }
   if (tid < kCt) gate_scan(gv, bv, Gs, Bs, tid, lane);
