@@ -40,7 +40,7 @@ METRIC = "streamed chunks/s and attention TFLOP/s (% of B200 BF16 peak) per conf
 # DRAM bytes (read + write) per launch of the attention kernel, from the ncu
 # capture summarised in profiles/ (512p, steady chunk with 7168 keys), keyed by
 # a hash of the kernel sources it was taken on: a changed kernel reports null.
-PROFILED_TRAFFIC = {"37ffe72da4da716a": 137.36e6}
+PROFILED_TRAFFIC = {"031578c3b0278178": 137.59e6, "031578c3b0278178/e4m3": 54.17e6}
 
 
 def attend_source_hash() -> str:
@@ -150,9 +150,10 @@ def gpu_id_for(dev: int) -> str:
 
 
 # ------------------------------------------------------------------ oracle timing
-def oracle_sample(w, rank_stream: int = 0, budget_rows: int = 40960):
+def oracle_sample(w, rank_stream: int = 0, budget_rows: int = 1 << 30):
     """Times the fp64 oracle on one steady-state chunk: key build plus
-    `budget_rows` output rows, extrapolated linearly to a whole chunk."""
+    `budget_rows` output rows (by default every row of the chunk),
+    extrapolated linearly to a whole chunk when fewer."""
     import numpy as np
 
     import oracle as O
@@ -174,9 +175,11 @@ def oracle_sample(w, rank_stream: int = 0, budget_rows: int = 40960):
     per_chunk = t_fixed + per_row * w.Lc * w.H
     return {"value": 1.0 / per_chunk, "unit": "chunks/s", "cores": O.num_threads(),
             "kind": "oracle",
-            "sample": f"{w.name} chunk {c}: visible-key build + {n} of {w.Lc * w.H} (token, head) "
-                      f"output rows in fp64, extrapolated linearly to the whole chunk "
-                      f"({t_fixed + t_rows:.1f} s of CPU time)"}
+            "sample": (f"{w.name} chunk {c}: visible-key build + " +
+                       (f"all {n} (token, head) output rows in fp64" if n == w.Lc * w.H else
+                        f"{n} of {w.Lc * w.H} (token, head) output rows in fp64, extrapolated "
+                        f"linearly to the whole chunk") +
+                       f" ({t_fixed + t_rows:.1f} s of CPU time)")}
 
 
 def run_reference(args, w, rank, world):
@@ -230,21 +233,29 @@ def gdn_flops_per_token(D: int, ct: int = 64) -> float:
     return 6.0 * D * D + 4.0 * (ct + 1) * D + ct * ct / 3.0
 
 
-def gdn_oracle_sample(w, g_scale: float, n_tok: int = 256):
+def gdn_oracle_sample(w, g_scale: float, n_chunks: int = 0, n_tok: int = 0):
+    """Times the fp64 oracle on consecutive chunks of stream 0 (the state
+    carried between them): n_chunks whole chunks (0: every chunk of a step),
+    or only the first n_tok tokens of chunk 0 when n_tok > 0 (short samples)."""
     import numpy as np
 
     import oracle as O
-    q, k, v, g, beta = O.gdn_inputs(w, 0, 0, g_scale)
     st = np.zeros((w.H, w.D, w.D))
-    t0 = time.perf_counter()
-    O.gdn_chunk(1.0 / np.sqrt(w.D), st, q[:n_tok], k[:n_tok], v[:n_tok], g[:n_tok], beta[:n_tok])
-    dt = time.perf_counter() - t0
-    per_chunk = dt * w.Lc / n_tok
+    chunks = 1 if n_tok else (n_chunks or w.n_chunks)
+    toks = n_tok if n_tok else w.Lc
+    dt = 0.0
+    for c in range(chunks):
+        q, k, v, g, beta = O.gdn_inputs(w, 0, c, g_scale)
+        t0 = time.perf_counter()
+        O.gdn_chunk(1.0 / np.sqrt(w.D), st, q[:toks], k[:toks], v[:toks], g[:toks], beta[:toks])
+        dt += time.perf_counter() - t0
+    per_chunk = dt * w.Lc / (toks * chunks)
+    what = (f"the first {toks} of {w.Lc} tokens of one chunk, extrapolated linearly to the chunk"
+            if n_tok else f"{chunks} consecutive chunks of one stream ({w.Lc} tokens each)")
     return {"value": 1.0 / per_chunk, "unit": "chunks/s", "cores": O.num_threads(),
             "kind": "oracle",
-            "sample": f"{w.name}: the first {n_tok} of {w.Lc} tokens of one chunk, all {w.H} heads "
-                      f"(fp64 token-by-token recurrence, heads across threads), extrapolated "
-                      f"linearly to the chunk ({dt:.2f} s of CPU time)"}
+            "sample": f"{w.name}: {what}, all {w.H} heads (fp64 token-by-token recurrence, heads "
+                      f"across threads; {dt:.2f} s of CPU time, input generation not timed)"}
 
 
 def gdn_config_json(w, world, g_scale):
@@ -264,7 +275,7 @@ def run_gdn(args, w, rank, world):
             return
         per = []
         for i in range(args.warmup + args.steps):
-            r = gdn_oracle_sample(w, g_scale, n_tok=64)
+            r = gdn_oracle_sample(w, g_scale, n_tok=256)
             if i >= args.warmup:
                 per.append(1.0 / r["value"])
         ms_step = 1000.0 * w.n_chunks * w.B * statistics.mean(per)
@@ -379,10 +390,14 @@ def run_gdn(args, w, rank, world):
     hbm_pk, bf16_burst, _, pk_src = peaks()
     peak = bf16_burst if tc else alu_peak
     n_sub = (w.Lc + 63) // 64
-    # tensor-core FLOPs the sequential pass issues per call: per (head, 64-token
-    # block) K^S^T and Q^S^T (2 x 128 x D x D), T and M times the right-hand side
-    # (2 x 128 x 64 x D) and the state update (2 x D x 64 x D), three split terms each
-    issued = 3.0 * (2 * 128 * w.D * w.D + 2 * 128 * 64 * w.D + 2 * w.D * 64 * w.D) * n_sub * w.H * B
+    # tensor-core FLOPs issued per call, per (head, 64-token block), three split
+    # terms each: in the prep kernel the Gram matrices [K^;Q^] K^T (2 x 128 x 64 x D,
+    # once per head); in the sequential pass (once per 64-column value slice, two
+    # slices per head) K^S^T and Q^S^T (2 x 128 x D x 64), T and M times the
+    # right-hand side (2 x 128 x 64 x 64) and the state update (2 x D x 64 x 64)
+    slices = w.D // 64
+    issued = 3.0 * (2 * 128 * 64 * w.D + slices * (2 * 128 * w.D * 64 + 2 * 128 * 64 * 64 +
+                                                    2 * w.D * 64 * 64)) * n_sub * w.H * B
     bytes_per_launch = B * (w.Lc * w.H * w.D * esz * 4 + w.Lc * w.H * 8 + 2 * w.H * w.D * w.D * 4)
     # (the workspace of the prep kernel's per-block output is written and read
     # back, mostly through L2, and is not algorithmic traffic)
@@ -434,7 +449,7 @@ def run_gdn(args, w, rank, world):
         "ms_per_chunk": ms_step / chunks_per_step,
         "launch_mode": "cuda graph of one step, replayed",
         "roofline": {"bound": "tensor" if tc else "alu",
-                     "kernel": (f"gdn_prep_kernel<{w.D}> + gdn_tc_kernel (one call)" if tc else
+                     "kernel": ("gdn_prep_tc_kernel + gdn_tc_kernel (one call)" if tc else
                                 f"gdn_prep_kernel<{w.D}> + gdn_chunk_kernel<{w.D}> (one call)"),
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
