@@ -754,11 +754,23 @@ def per_config_entry(res, note):
             "step": note, "config": config_json(w, 1),
             "attention_tflops": fr["attention_tflops"],
             "attention_frac_of_burst": fr["attention_frac_of_burst"],
+            "attention_frac_of_burst_per_clock": clock_normalised(fr["attention_frac_of_burst"],
+                                                                  res["clocks"]),
             "attention_frac_of_nominal": fr["attention_frac_of_nominal"],
             "append_gbs": fr["append_gbs"], "append_frac_of_hbm": fr["append_frac_of_hbm"],
             "kernel_ms_per_step": res["kernel_ms_per_step"],
             "attention_launches_per_step": res["att_launches_per_step"],
             "gpu_launches": res["launches"], "clocks": res["clocks"]}
+
+
+def clock_normalised(frac, clocks):
+    """The fraction scaled by max / median SM clock of the timed region: what
+    the same kernel reaches per clock cycle, for comparing configurations whose
+    power draw puts them at different clocks (the tensor pipe's rate is
+    proportional to the SM clock). None without a clock record."""
+    if frac is None or not clocks or not clocks.get("sm_mhz") or not clocks.get("sm_max_mhz"):
+        return None
+    return frac * clocks["sm_max_mhz"] / clocks["sm_mhz"]
 
 
 def main():
@@ -873,6 +885,8 @@ def main():
                      "peak_source": (f"{pk_src} bf16 burst x 2 (fp8 nominal ratio)" if f8 else
                                      f"{pk_src} bf16 burst (kernel timed per launch)"),
                      "frac_of_sustained": res["achieved"] / (mul * pk_sust),
+                     "frac_per_clock": clock_normalised(res["achieved"] / (mul * pk_burst),
+                                                        res.get("clocks")),
                      "frac_of_nominal": res["achieved"] / (mul * NOMINAL_BF16_TFLOPS),
                      "nominal_peak": mul * NOMINAL_BF16_TFLOPS,
                      "algorithmic_flops_per_launch": res["att_flops_per_launch"],
