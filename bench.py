@@ -275,7 +275,7 @@ def run_gdn(args, w, rank, world):
             return
         per = []
         for i in range(args.warmup + args.steps):
-            r = gdn_oracle_sample(w, g_scale, n_tok=256)
+            r = gdn_oracle_sample(w, g_scale, n_chunks=1)
             if i >= args.warmup:
                 per.append(1.0 / r["value"])
         ms_step = 1000.0 * w.n_chunks * w.B * statistics.mean(per)
