@@ -1037,9 +1037,9 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_chunk_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------- tensor-core sequential pass
-// D = 128. One CTA per (stream, head, 64 value dims of the state): 4 warps
-// for the elementwise work (thread r owns TMEM lane r) and 1 warp that issues
-// the copies and the tcgen05 MMAs. The state slice lives in TMEM, transposed
+// D = 128. One CTA per (stream, head, 64 value dims of the state): 16 warps
+// for the elementwise work (four threads per TMEM lane r, 16 value columns
+// each) and 1 warp that issues the copies and the tcgen05 MMAs. The state slice lives in TMEM, transposed
 // (lane = key dim k, column = value dim v: ST[k][v] = S[v][k]), for the whole
 // call. Per 64-token sub-chunk j, with its operand images from the prep
 // kernel (KQ, TM) arriving by bulk copy one or two sub-chunks ahead:
@@ -1072,28 +1072,52 @@ struct GdnTcSmem {
   static constexpr uint32_t bytes = bs + 2 * kCt * 4;
   static_assert(bytes <= 232448, "exceeds 227 KB of shared memory per CTA");
 };
-constexpr int kTcThreads = 160;
 constexpr int kTcSlice = 64;
+// elementwise warps: warps w, w + 4, w + 8 and w + 12 share TMEM lanes
+// 32 (w % 4) .. + 31 and take 16 value columns each of those rows (the
+// elementwise phases are on the sequential chain: 16 warps shorten them
+// against 4 or 8)
+constexpr int kTcElemWarps = 16;
+constexpr int kTcCols = kTcSlice / (kTcElemWarps / 4);   // values per thread
+constexpr int kTcThreads = 32 * kTcElemWarps + 32;
+static_assert(kTcCols == 32 || kTcCols == 16, "two or four threads per TMEM lane");
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* x) {
+  if constexpr (N == 32)
+    ptx::tmem_ld32(taddr, x);
+  else
+    ptx::tmem_ld16(taddr, x);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* x) {
+  if constexpr (N == 32)
+    ptx::tmem_st32(taddr, x);
+  else
+    ptx::tmem_st16u(taddr, reinterpret_cast<const uint32_t*>(x));
+}
 constexpr uint64_t kTcTimeoutNs = 1000000000ull;
 
-// Row `row` (64 floats) of a single-panel image as bf16 hi and lo.
-__device__ __forceinline__ void put_row64(unsigned char* sm, uint32_t hi_off, uint32_t lo_off,
-                                          int row, const float* x) {
+// NV floats of row `row` of a single-panel image, from 16-byte column group
+// c0 on, as bf16 hi and lo.
+template <int NV>
+__device__ __forceinline__ void put_row(unsigned char* sm, uint32_t hi_off, uint32_t lo_off,
+                                        int row, int c0, const float* x) {
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < NV / 8; ++c) {
     uint4 h, l;
     split8(x + 8 * c, h, l);
-    const uint32_t off = sw128_off(row, c);
+    const uint32_t off = sw128_off(row, c0 + c);
     *reinterpret_cast<uint4*>(sm + hi_off + off) = h;
     *reinterpret_cast<uint4*>(sm + lo_off + off) = l;
   }
 }
 
-template <typename T>
-__device__ __forceinline__ void load64(const T* src, float* x) {
+template <int NV, typename T>
+__device__ __forceinline__ void load_row(const T* src, float* x) {
   if constexpr (sizeof(T) == 2) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < NV / 8; ++i) {
       const uint4 u = *reinterpret_cast<const uint4*>(src + 8 * i);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -1104,18 +1128,18 @@ __device__ __forceinline__ void load64(const T* src, float* x) {
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < NV / 4; ++i) {
       const float4 u = *reinterpret_cast<const float4*>(src + 4 * i);
       x[4 * i] = u.x, x[4 * i + 1] = u.y, x[4 * i + 2] = u.z, x[4 * i + 3] = u.w;
     }
   }
 }
 
-template <typename T>
-__device__ __forceinline__ void store64(T* dst, const float* x) {
+template <int NV, typename T>
+__device__ __forceinline__ void store_row(T* dst, const float* x) {
   if constexpr (sizeof(T) == 2) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < NV / 8; ++i) {
       uint32_t w[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -1126,7 +1150,7 @@ __device__ __forceinline__ void store64(T* dst, const float* x) {
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < NV / 4; ++i)
       *reinterpret_cast<float4*>(dst + 4 * i) =
           make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
   }
@@ -1162,11 +1186,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
     ptx::mbar_init(bar(L::B_KQ), 1);
     ptx::mbar_init(bar(L::B_KQ + 1), 1);
     ptx::mbar_init(bar(L::B_TM), 1);
-    ptx::mbar_init(bar(L::B_S), 128);
+    ptx::mbar_init(bar(L::B_S), 32 * kTcElemWarps);
     ptx::mbar_init(bar(L::B_D1), 1);
-    ptx::mbar_init(bar(L::B_RHS), 128);
+    ptx::mbar_init(bar(L::B_RHS), 32 * kTcElemWarps);
     ptx::mbar_init(bar(L::B_D2), 1);
-    ptx::mbar_init(bar(L::B_U), 128);
+    ptx::mbar_init(bar(L::B_U), 32 * kTcElemWarps);
     ptx::mbar_init(bar(L::B_D3), 1);
     ptx::mbar_init(bar(L::B_G), 64);
     ptx::mbar_init(bar(L::B_DR), 1);
@@ -1174,7 +1198,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
     *no_abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kTcElemWarps) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), 256);
     ptx::tmem_relinquish();
   }
@@ -1190,7 +1214,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
   const unsigned char* images = reinterpret_cast<const unsigned char*>(p.workspace) + kWsHeader +
                                 ((size_t)z * H + h) * (size_t)nsub * kImgBytes;
 
-  if (warp == 4) {
+  if (warp == kTcElemWarps) {
     // ------------------------------------------------------------ copies + MMA issue
     if (lane == 0) {
       auto load_kq = [&](int j) {
@@ -1307,18 +1331,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
       ptx::mbar_wait(bar(L::B_DR), 0, no_abort, kTcTimeoutNs);
     }
   } else {
-    // ------------------------------------------------------------ elementwise (TMEM lane = tid)
-    const int r = tid;  // 0..63: key/U rows, 64..127: query/output rows; also key dim r of ST
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------------------ elementwise
+    // TMEM lane r: 0..63 key/U rows, 64..127 query/output rows; also key dim r
+    // of ST. Columns [cb, cb + 32) of the slice.
+    const int r = (warp & 3) * 32 + lane;
+    const int grp = warp >> 2;   // column group
+    const int cb = grp * kTcCols;
+    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
     const T* v = static_cast<const T*>(p.v);
     T* out = static_cast<T*>(p.out);
     const size_t tok_stride = (size_t)H * D;
-    const size_t bh0 = (size_t)b * (size_t)Tn * tok_stride + (size_t)h * D + vcol;
+    const size_t bh0 = (size_t)b * (size_t)Tn * tok_stride + (size_t)h * D + vcol + cb;
     const size_t g0 = (size_t)b * (size_t)Tn * H + h;
     float* Sg = p.state + ((size_t)b * H + h) * D * D;   // [v][k]
     auto gates = [&](int j) {
       // threads 0..63: prefix sums of g log2(e) and beta of sub-chunk j
-      if (r < kCt) {
+      if (grp == 0 && r < kCt) {
         const int64_t t = (int64_t)j * kCt + r;
         const bool in = t < Tn;
         gate_scan(in ? p.g[g0 + (size_t)t * H] : 0.f, in ? p.beta[g0 + (size_t)t * H] : 0.f,
@@ -1336,15 +1364,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
     gates(0);
     if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_G), 0, abort_flag, kTcTimeoutNs))) ok = false;
     if (ok) {
-      float x[kTcSlice];
+      float x[kTcCols];
 #pragma unroll
-      for (int i = 0; i < kTcSlice; ++i) x[i] = Sg[(size_t)(vcol + i) * D + r];
-      put_row64(smc, L::st, L::st + 16384, r, x);
+      for (int i = 0; i < kTcCols; ++i) x[i] = Sg[(size_t)(vcol + cb + i) * D + r];
+      put_row<kTcCols>(smc, L::st, L::st + 16384, r, cb / 8, x);
       const float dec = ptx::ex2(gcum(0, kCt - 1));
 #pragma unroll
-      for (int i = 0; i < kTcSlice; ++i) x[i] *= dec;
-      ptx::tmem_st32(t_st + lane_off, x);
-      ptx::tmem_st32(t_st + lane_off + 32, x + 32);
+      for (int i = 0; i < kTcCols; ++i) x[i] *= dec;
+      tmem_st_cols<kTcCols>(t_st + lane_off + cb, x);
       ptx::tmem_wait_st();
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
@@ -1356,13 +1383,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
       const int tr = r & (kCt - 1);               // token of this row
       const bool tok_in = t0 + tr < Tn;
       // values of this sub-chunk's token (key rows), loaded while MMA1 runs
-      float vv[kTcSlice];
+      float vv[kTcCols];
       if (r < kCt) {
         if (tok_in) {
-          load64(v + bh0 + (size_t)(t0 + tr) * tok_stride, vv);
+          load_row<kTcCols>(v + bh0 + (size_t)(t0 + tr) * tok_stride, vv);
         } else {
 #pragma unroll
-          for (int i = 0; i < kTcSlice; ++i) vv[i] = 0.f;
+          for (int i = 0; i < kTcCols; ++i) vv[i] = 0.f;
         }
       }
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_D1), par, abort_flag, kTcTimeoutNs))) {
@@ -1370,20 +1397,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
         break;
       }
       ptx::tc_fence_after();
-      float x[kTcSlice];
-      ptx::tmem_ld32(t_d1 + lane_off, x);
-      ptx::tmem_ld32(t_d1 + lane_off + 32, x + 32);
+      float x[kTcCols];
+      tmem_ld_cols<kTcCols>(t_d1 + lane_off + cb, x);
       ptx::tmem_wait_ld();
       const float eg = ptx::ex2(gcum(j, tr));
       if (r < kCt) {
         const float bt = Bs[(j & 1) * kCt + tr];
 #pragma unroll
-        for (int i = 0; i < kTcSlice; ++i) vv[i] = bt * (vv[i] - eg * x[i]);
-        put_row64(smc, L::rhs, L::rhs + 8192, tr, vv);
+        for (int i = 0; i < kTcCols; ++i) vv[i] = bt * (vv[i] - eg * x[i]);
+        put_row<kTcCols>(smc, L::rhs, L::rhs + 8192, tr, cb / 8, vv);
       } else {
         const float sc = p.scale * eg;
 #pragma unroll
-        for (int i = 0; i < kTcSlice; ++i) vv[i] = sc * x[i];   // (query rows: the inter-chunk output)
+        for (int i = 0; i < kTcCols; ++i) vv[i] = sc * x[i];   // (query rows: the inter-chunk output)
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
@@ -1395,18 +1421,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
         break;
       }
       ptx::tc_fence_after();
-      ptx::tmem_ld32(t_d2 + lane_off, x);
-      ptx::tmem_ld32(t_d2 + lane_off + 32, x + 32);
+      tmem_ld_cols<kTcCols>(t_d2 + lane_off + cb, x);
       ptx::tmem_wait_ld();
       if (r < kCt) {
         const float wt = ptx::ex2(gcum(j, kCt - 1) - gcum(j, tr));
 #pragma unroll
-        for (int i = 0; i < kTcSlice; ++i) x[i] *= wt;
-        put_row64(smc, L::uu, L::uu + 8192, tr, x);
+        for (int i = 0; i < kTcCols; ++i) x[i] *= wt;
+        put_row<kTcCols>(smc, L::uu, L::uu + 8192, tr, cb / 8, x);
       } else if (tok_in) {
 #pragma unroll
-        for (int i = 0; i < kTcSlice; ++i) x[i] += vv[i];
-        store64(out + bh0 + (size_t)(t0 + tr) * tok_stride, x);
+        for (int i = 0; i < kTcCols; ++i) x[i] += vv[i];
+        store_row<kTcCols>(out + bh0 + (size_t)(t0 + tr) * tok_stride, x);
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
@@ -1416,9 +1441,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
         break;
       }
       ptx::tc_fence_after();
-      // the state after sub-chunk j (key dim r, 64 value dims)
-      ptx::tmem_ld32(t_st + lane_off, x);
-      ptx::tmem_ld32(t_st + lane_off + 32, x + 32);
+      // the state after sub-chunk j (key dim r, 32 value dims)
+      tmem_ld_cols<kTcCols>(t_st + lane_off + cb, x);
       ptx::tmem_wait_ld();
       if (j + 1 < nsub) {
         if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_G), (uint32_t)(j + 1) & 1, abort_flag,
@@ -1426,19 +1450,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
           ok = false;
           break;
         }
-        put_row64(smc, L::st, L::st + 16384, r, x);
+        put_row<kTcCols>(smc, L::st, L::st + 16384, r, cb / 8, x);
         const float dec = ptx::ex2(gcum(j + 1, kCt - 1));
 #pragma unroll
-        for (int i = 0; i < kTcSlice; ++i) x[i] *= dec;
-        ptx::tmem_st32(t_st + lane_off, x);
-        ptx::tmem_st32(t_st + lane_off + 32, x + 32);
+        for (int i = 0; i < kTcCols; ++i) x[i] *= dec;
+        tmem_st_cols<kTcCols>(t_st + lane_off + cb, x);
         ptx::tmem_wait_st();
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar(L::B_S));
       } else {
 #pragma unroll
-        for (int i = 0; i < kTcSlice; ++i) Sg[(size_t)(vcol + i) * D + r] = x[i];
+        for (int i = 0; i < kTcCols; ++i) Sg[(size_t)(vcol + cb + i) * D + r] = x[i];
       }
     }
     if (!ok) fail();
@@ -1446,7 +1469,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == 4) ptx::tmem_dealloc(tmem, 256);
+  if (warp == kTcElemWarps) ptx::tmem_dealloc(tmem, 256);
 }
 
 // D = 128: the prep kernel writes the operand images and the tensor-core
