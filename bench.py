@@ -233,6 +233,17 @@ def gdn_flops_per_token(D: int, ct: int = 64) -> float:
     return 6.0 * D * D + 4.0 * (ct + 1) * D + ct * ct / 3.0
 
 
+def gdn_launches_per_call(w, n_active: int) -> int:
+    """Kernels one sa_gdn_chunk call launches: the prep and the sequential
+    pass, or both twice when the library splits a D = 128 call of at least 8
+    sub-chunks into halves (the pass then leaves at least half the SMs to the
+    prep of the second half)."""
+    n_sub = (w.Lc + 63) // 64
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    split = w.D == 128 and n_sub >= 8 and 2 * (w.D // 64) * w.H * n_active <= sms
+    return 4 if split else 2
+
+
 def gdn_oracle_sample(w, g_scale: float, n_chunks: int = 0, n_tok: int = 0):
     """Times the fp64 oracle on consecutive chunks of stream 0 (the state
     carried between them): n_chunks whole chunks (0: every chunk of a step),
@@ -462,9 +473,9 @@ def run_gdn(args, w, rank, world):
                      "algorithmic_flops_per_launch": flops_per_launch,
                      "hbm_bytes_per_launch": bytes_per_launch,
                      "hbm_frac": bytes_per_launch / avg_launch_s / 1e9 / hbm,
-                     "duration": "mean of CUDA events around each call (its two launches) on "
+                     "duration": "mean of CUDA events around each call (all its launches) on "
                                  "the launch stream, eager pass", "traffic": None},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * nC * args.steps, "clocks": clocks,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gdn_launches_per_call(w, B) * nC * args.steps, "clocks": clocks,
         "call_ms": {"mean": statistics.mean(launch_ms),
                       "p50": float(np.percentile(launch_ms, 50)),
                       "p99": float(np.percentile(launch_ms, 99))},

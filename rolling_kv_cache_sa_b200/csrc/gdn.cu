@@ -581,21 +581,22 @@ __device__ __forceinline__ void split4(float4 x, uint2& hi, uint2& lo) {
 // about 2^-16 relative per term); the threads read it back and form L and P
 // (key rows and query rows of the product). Then T, M and the TM image.
 template <typename T>
-__global__ void __launch_bounds__(kGdnThreads, kPrepTcCtasPerSm)
-    gdn_prep_tc_kernel(const __grid_constant__ GdnParams p) {
+__device__ __forceinline__ void prep_tc_body(const GdnParams& p) {
   constexpr int D = 128;
   using L = GdnPrepTcSmem;
   extern __shared__ __align__(1024) unsigned char smp[];
   int* status = reinterpret_cast<int*>(p.workspace);
   const uint32_t base = ptx::smem_u32(smp);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int j = blockIdx.x, h = blockIdx.y, z = blockIdx.z, b = p.stream_of[z];
+  const int j = p.j_begin + (int)blockIdx.x, h = blockIdx.y, z = blockIdx.z, b = p.stream_of[z];
   const int H = p.H;
   const int64_t Tn = p.T;
   const int64_t t0 = (int64_t)j * kCt;
   const int n = (int)(Tn - t0 < kCt ? Tn - t0 : kCt);
   // (block-uniform: the whole block leaves before any barrier)
-  if (!SA_BOUNDS(b >= 0 && b < p.batch && z < p.n_streams && j < p.n_sub && n > 0, 0)) return;
+  if (!SA_BOUNDS(b >= 0 && b < p.batch && z < p.n_streams && j < p.j_end && j < p.n_sub && n > 0,
+                 0))
+    return;
   // the call's device status word starts at zero (the prep kernel runs first)
   if (j == 0 && h == 0 && z == 0 && tid == 0) *status = 0;
   if (base & 1023u) {
@@ -769,6 +770,20 @@ __global__ void __launch_bounds__(kGdnThreads, kPrepTcCtasPerSm)
     *reinterpret_cast<uint4*>(img_g + off) = hi;
     *reinterpret_cast<uint4*>(img_g + kImgTM + off) = lo;
   }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kGdnThreads, kPrepTcCtasPerSm)
+    gdn_prep_tc_kernel(const __grid_constant__ GdnParams p) {
+  prep_tc_body<T>(p);
+  // A prep piece launched while the previous pass piece still runs
+  // (programmatic dependent launch) must not complete before that pass: the
+  // next pass piece, which starts when this grid completes, continues from
+  // its state. One thread of the last CTA waits for the previous grid, after
+  // its own work, so the other CTAs leave their slots free.
+  if (p.pdl_wait && threadIdx.x == 0 && blockIdx.x == gridDim.x - 1 &&
+      blockIdx.y == gridDim.y - 1 && blockIdx.z == gridDim.z - 1)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 template <int D, typename T>
@@ -1097,6 +1112,8 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* x) {
     ptx::tmem_st16u(taddr, reinterpret_cast<const uint32_t*>(x));
 }
 constexpr uint64_t kTcTimeoutNs = 1000000000ull;
+// a call of at least this many sub-chunks runs in two pieces (launch_gdn_t)
+constexpr int kGdnSplitMin = 8;
 
 // NV floats of row `row` of a single-panel image, from 16-byte column group
 // c0 on, as bf16 hi and lo.
@@ -1172,7 +1189,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
   const int H = p.H;
   const int64_t Tn = p.T;
   const int nsub = p.n_sub;
+  // sub-chunks [j0, j0 + nl) of the call; barrier parities and buffers follow
+  // the local index jl = j - j0 (every barrier starts at phase 0 in a launch)
+  const int j0 = p.j_begin, nl = p.j_end - p.j_begin;
   const int vcol = slice * kTcSlice;
+  // the next prep piece (if any) may start on the SMs this grid leaves free
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t bar0 = base + L::bars;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smc + L::misc);
@@ -1180,7 +1202,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
   volatile int* no_abort = reinterpret_cast<volatile int*>(smc + L::misc + 8);
   float* Gs = reinterpret_cast<float*>(smc + L::gs);
   float* Bs = reinterpret_cast<float*>(smc + L::bs);
-  if (!SA_BOUNDS(b >= 0 && b < p.batch && z < p.n_streams && vcol + kTcSlice <= D, 3)) return;
+  if (!SA_BOUNDS(b >= 0 && b < p.batch && z < p.n_streams && vcol + kTcSlice <= D && j0 >= 0 &&
+                     nl > 0 && p.j_end <= nsub,
+                 3))
+    return;
 
   if (tid == 0) {
     ptx::mbar_init(bar(L::B_KQ), 1);
@@ -1217,15 +1242,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
   if (warp == kTcElemWarps) {
     // ------------------------------------------------------------ copies + MMA issue
     if (lane == 0) {
-      auto load_kq = [&](int j) {
-        const uint32_t dst = base + L::kq + (uint32_t)(j & 1) * 2 * kImgKQ;
-        const unsigned char* src = images + (size_t)j * kImgBytes;
-        ptx::mbar_arrive_expect_tx(bar(L::B_KQ + (j & 1)), 2 * kImgKQ);
+      auto load_kq = [&](int jl) {
+        const uint32_t dst = base + L::kq + (uint32_t)(jl & 1) * 2 * kImgKQ;
+        const unsigned char* src = images + (size_t)(j0 + jl) * kImgBytes;
+        ptx::mbar_arrive_expect_tx(bar(L::B_KQ + (jl & 1)), 2 * kImgKQ);
         for (uint32_t o = 0; o < 2 * kImgKQ; o += 16384)
-          ptx::bulk_g2s(dst + o, src + o, 16384, bar(L::B_KQ + (j & 1)));
+          ptx::bulk_g2s(dst + o, src + o, 16384, bar(L::B_KQ + (jl & 1)));
       };
-      auto load_tm = [&](int j) {
-        const unsigned char* src = images + (size_t)j * kImgBytes + 2 * kImgKQ;
+      auto load_tm = [&](int jl) {
+        const unsigned char* src = images + (size_t)(j0 + jl) * kImgBytes + 2 * kImgKQ;
         ptx::mbar_arrive_expect_tx(bar(L::B_TM), 2 * kImgTM);
         for (uint32_t o = 0; o < 2 * kImgTM; o += 16384)
           ptx::bulk_g2s(base + L::tm + o, src + o, 16384, bar(L::B_TM));
@@ -1243,17 +1268,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
       int kq_issued = 0, kq_done = 0, tm_issued = 0;
       load_kq(0);
       ++kq_issued;
-      if (nsub > 1) {
+      if (nl > 1) {
         load_kq(1);
         ++kq_issued;
       }
       load_tm(0);
       ++tm_issued;
       bool ok = true;
-      for (int j = 0; ok && j < nsub; ++j) {
-        const uint32_t par = (uint32_t)j & 1;
-        const uint32_t kqb = base + L::kq + (uint32_t)(j & 1) * 2 * kImgKQ;
-        if (!ptx::mbar_wait(bar(L::B_KQ + (j & 1)), (uint32_t)(j >> 1) & 1, abort_flag, kTcTimeoutNs) ||
+      for (int jl = 0; ok && jl < nl; ++jl) {
+        const uint32_t par = (uint32_t)jl & 1;
+        const uint32_t kqb = base + L::kq + (uint32_t)(jl & 1) * 2 * kImgKQ;
+        if (!ptx::mbar_wait(bar(L::B_KQ + (jl & 1)), (uint32_t)(jl >> 1) & 1, abort_flag, kTcTimeoutNs) ||
             !ptx::mbar_wait(bar(L::B_S), par, abort_flag, kTcTimeoutNs)) {
           ok = false;
           break;
@@ -1292,8 +1317,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
           ok = false;
           break;
         }
-        if (j + 1 < nsub) {
-          load_tm(j + 1);
+        if (jl + 1 < nl) {
+          load_tm(jl + 1);
           ++tm_issued;
         }
         if (!ptx::mbar_wait(bar(L::B_U), par, abort_flag, kTcTimeoutNs)) {
@@ -1311,13 +1336,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
             ptx::umma_ss(t_st, ptx::sdesc_add(a3, ta[i] * kImgKQ + (uint32_t)kk * 2048),
                          ptx::sdesc_add(d_uu, tb[i] * 8192 + (uint32_t)kk * 2048), id_mm, 1u);
         ptx::umma_commit(bar(L::B_D3));
-        // the KQ buffer of j is free once MMA3 has read it
-        if (j + 2 < nsub) {
+        // the KQ buffer of jl is free once MMA3 has read it
+        if (jl + 2 < nl) {
           if (!ptx::mbar_wait(bar(L::B_D3), par, abort_flag, kTcTimeoutNs)) {
             ok = false;
             break;
           }
-          load_kq(j + 2);
+          load_kq(jl + 2);
           ++kq_issued;
         }
       }
@@ -1344,22 +1369,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
     const size_t bh0 = (size_t)b * (size_t)Tn * tok_stride + (size_t)h * D + vcol + cb;
     const size_t g0 = (size_t)b * (size_t)Tn * H + h;
     float* Sg = p.state + ((size_t)b * H + h) * D * D;   // [v][k]
-    auto gates = [&](int j) {
-      // threads 0..63: prefix sums of g log2(e) and beta of sub-chunk j
+    auto gates = [&](int jl) {
+      // threads 0..63: prefix sums of g log2(e) and beta of sub-chunk j0 + jl
       if (grp == 0 && r < kCt) {
-        const int64_t t = (int64_t)j * kCt + r;
+        const int64_t t = (int64_t)(j0 + jl) * kCt + r;
         const bool in = t < Tn;
         gate_scan(in ? p.g[g0 + (size_t)t * H] : 0.f, in ? p.beta[g0 + (size_t)t * H] : 0.f,
-                  Gs + (j & 1) * kCt, Bs + (j & 1) * kCt, r, lane);
+                  Gs + (jl & 1) * kCt, Bs + (jl & 1) * kCt, r, lane);
         ptx::mbar_arrive(bar(L::B_G));
       }
     };
-    auto gcum = [&](int j, int t) -> float {
-      const float* G = Gs + (j & 1) * kCt;
+    auto gcum = [&](int jl, int t) -> float {
+      const float* G = Gs + (jl & 1) * kCt;
       return G[t] + (t >= 32 ? G[31] : 0.f);
     };
     bool ok = true;
-    // prologue: the gates of sub-chunk 0, the S image of the initial state and
+    // prologue: the gates of sub-chunk j0, the S image of the initial state and
     // ST = e^{G_last} S
     gates(0);
     if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_G), 0, abort_flag, kTcTimeoutNs))) ok = false;
@@ -1377,9 +1402,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar(L::B_S));
     }
-    for (int j = 0; ok && j < nsub; ++j) {
-      const uint32_t par = (uint32_t)j & 1;
-      const int64_t t0 = (int64_t)j * kCt;
+    for (int jl = 0; ok && jl < nl; ++jl) {
+      const uint32_t par = (uint32_t)jl & 1;
+      const int64_t t0 = (int64_t)(j0 + jl) * kCt;
       const int tr = r & (kCt - 1);               // token of this row
       const bool tok_in = t0 + tr < Tn;
       // values of this sub-chunk's token (key rows), loaded while MMA1 runs
@@ -1400,9 +1425,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
       float x[kTcCols];
       tmem_ld_cols<kTcCols>(t_d1 + lane_off + cb, x);
       ptx::tmem_wait_ld();
-      const float eg = ptx::ex2(gcum(j, tr));
+      const float eg = ptx::ex2(gcum(jl, tr));
       if (r < kCt) {
-        const float bt = Bs[(j & 1) * kCt + tr];
+        const float bt = Bs[(jl & 1) * kCt + tr];
 #pragma unroll
         for (int i = 0; i < kTcCols; ++i) vv[i] = bt * (vv[i] - eg * x[i]);
         put_row<kTcCols>(smc, L::rhs, L::rhs + 8192, tr, cb / 8, vv);
@@ -1415,7 +1440,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar(L::B_RHS));
       // the gates of the next sub-chunk, while MMA2 runs
-      if (j + 1 < nsub) gates(j + 1);
+      if (jl + 1 < nl) gates(jl + 1);
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_D2), par, abort_flag, kTcTimeoutNs))) {
         ok = false;
         break;
@@ -1424,7 +1449,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
       tmem_ld_cols<kTcCols>(t_d2 + lane_off + cb, x);
       ptx::tmem_wait_ld();
       if (r < kCt) {
-        const float wt = ptx::ex2(gcum(j, kCt - 1) - gcum(j, tr));
+        const float wt = ptx::ex2(gcum(jl, kCt - 1) - gcum(jl, tr));
 #pragma unroll
         for (int i = 0; i < kTcCols; ++i) x[i] *= wt;
         put_row<kTcCols>(smc, L::uu, L::uu + 8192, tr, cb / 8, x);
@@ -1441,17 +1466,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
         break;
       }
       ptx::tc_fence_after();
-      // the state after sub-chunk j (key dim r, 32 value dims)
+      // the state after sub-chunk j0 + jl (key dim r, this thread's value dims)
       tmem_ld_cols<kTcCols>(t_st + lane_off + cb, x);
       ptx::tmem_wait_ld();
-      if (j + 1 < nsub) {
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_G), (uint32_t)(j + 1) & 1, abort_flag,
+      if (jl + 1 < nl) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_G), (uint32_t)(jl + 1) & 1, abort_flag,
                                                     kTcTimeoutNs))) {
           ok = false;
           break;
         }
         put_row<kTcCols>(smc, L::st, L::st + 16384, r, cb / 8, x);
-        const float dec = ptx::ex2(gcum(j + 1, kCt - 1));
+        const float dec = ptx::ex2(gcum(jl + 1, kCt - 1));
 #pragma unroll
         for (int i = 0; i < kTcCols; ++i) x[i] *= dec;
         tmem_st_cols<kTcCols>(t_st + lane_off + cb, x);
@@ -1502,15 +1527,61 @@ cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (dev < 32) configured |= 1u << dev;
   }
-  if constexpr (kTc)
-    gdn_prep_tc_kernel<T><<<dim3(p.n_sub, p.H, p.n_streams), kGdnThreads, psmem, st>>>(p);
-  else
-    gdn_prep_kernel<D, T><<<dim3(p.n_sub, p.H, p.n_streams), kGdnThreads, psmem, st>>>(p);
-  if constexpr (kTc)
-    gdn_tc_kernel<T><<<dim3(D / kTcSlice, p.H, p.n_streams), kTcThreads, smem, st>>>(p);
-  else
-    gdn_chunk_kernel<D, T><<<dim3(D / kDvs, p.H, p.n_streams), kGdnThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  if constexpr (!kTc) {
+    GdnParams q = p;
+    q.j_begin = 0;
+    q.j_end = p.n_sub;
+    q.pdl_wait = 0;
+    gdn_prep_kernel<D, T><<<dim3(p.n_sub, p.H, p.n_streams), kGdnThreads, psmem, st>>>(q);
+    gdn_chunk_kernel<D, T><<<dim3(D / kDvs, p.H, p.n_streams), kGdnThreads, smem, st>>>(q);
+    return cudaGetLastError();
+  } else {
+    // The sequential pass occupies one SM per (stream, head, value slice) and
+    // leaves the others idle, while the prep of every sub-chunk must precede
+    // the pass that reads it. So the call runs in pieces of sub-chunks: prep
+    // piece k + 1 is launched as a programmatic dependent of pass piece k and
+    // runs on the idle SMs while that pass runs (it reads only the inputs and
+    // writes only its own sub-chunks' images); pass piece k + 1 starts when
+    // prep piece k + 1 has completed, which is after pass piece k (see
+    // gdn_prep_tc_kernel), and continues from the state that pass stored.
+    int sms = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // Two halves: each further piece adds a launch hand-off of 5-7 us
+    // (measured on the 512p call, 32 sub-chunks: 0.161 ms in two pieces,
+    // 0.169 in four, 0.186 in eight, 0.177 unsplit). Split only when the pass
+    // leaves at least half of the SMs to the prep.
+    const int pass_ctas = (D / kTcSlice) * p.H * p.n_streams;
+    const int piece = (p.n_sub >= kGdnSplitMin && 2 * pass_ctas <= sms) ? (p.n_sub + 1) / 2
+                                                                        : p.n_sub;
+    for (int jb = 0; jb < p.n_sub; jb += piece) {
+      GdnParams q = p;
+      q.j_begin = jb;
+      q.j_end = jb + piece < p.n_sub ? jb + piece : p.n_sub;
+      q.pdl_wait = jb > 0;
+      const dim3 pg((unsigned)(q.j_end - q.j_begin), (unsigned)p.H, (unsigned)p.n_streams);
+      if (jb == 0) {
+        gdn_prep_tc_kernel<T><<<pg, kGdnThreads, psmem, st>>>(q);
+      } else {
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = pg;
+        lc.blockDim = dim3(kGdnThreads);
+        lc.dynamicSmemBytes = psmem;
+        lc.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = at;
+        lc.numAttrs = 1;
+        e = cudaLaunchKernelEx(&lc, gdn_prep_tc_kernel<T>, q);
+        if (e != cudaSuccess) return e;
+      }
+      gdn_tc_kernel<T><<<dim3(D / kTcSlice, p.H, p.n_streams), kTcThreads, smem, st>>>(q);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
 }
 
 }  // namespace

@@ -164,6 +164,9 @@ struct GdnParams {
   int32_t n_streams;
   int32_t n_sub;       // ceil(T / 64)
   int32_t batch;       // B (bounds checks)
+  int32_t j_begin;     // sub-chunks [j_begin, j_end) of this launch (tensor-core path)
+  int32_t j_end;
+  int32_t pdl_wait;    // prep launched ahead of the previous pass piece: see launch_gdn_t
   int32_t stream_of[SA_MAX_STREAMS];
 };
 size_t gdn_workspace_bytes(int B, int H, int D, int64_t T);

@@ -136,6 +136,16 @@ def test_gdn_token_counts(fh, fw):
     _run_streams(w, [(1,), (1,)], 0.05, 1.0)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gdn_pieces_with_ragged_tail(dtype):
+    # 2,107 tokens per call: 33 sub-chunks, the last of 59 tokens. With D = 128
+    # and few heads a call runs in pieces of sub-chunks (the prep of one piece
+    # overlapping the sequential pass of the previous, which hands its state
+    # on through global memory); an inactive stream in one call.
+    w = _w(128, dtype, 43, 49, B=2, H=3, seed=5)
+    _run_streams(w, [(1, 1), (1, 0), (1, 1)], 0.02, 0.0)
+
+
 def test_gdn_zero_tokens_and_no_active_stream_are_no_ops():
     gdn = _gdn()
     st0 = torch.randn(2, 2, 64, 64, device="cuda")
