@@ -236,8 +236,9 @@ def gdn_flops_per_token(D: int, ct: int = 64) -> float:
 def gdn_launches_per_call(w, n_active: int) -> int:
     """Kernels one sa_gdn_chunk call launches: the prep and the sequential
     pass, or both twice when the library splits a D = 128 call of at least 8
-    sub-chunks into halves (the pass then leaves at least half the SMs to the
-    prep of the second half)."""
+    sub-chunks into two pieces (the pass then leaves at least half the SMs to
+    the prep of the second piece)."""
+    import torch
     n_sub = (w.Lc + 63) // 64
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     split = w.D == 128 and n_sub >= 8 and 2 * (w.D // 64) * w.H * n_active <= sms

@@ -453,10 +453,11 @@ typedef struct {
  *          and M = scale P T (P the decay-masked q.k matrix) into the
  *          workspace; the other walks the blocks in order and updates the
  *          state. With D = 128, at least 8 blocks and a pass that leaves half
- *          of the SMs idle, the call runs as two halves of its blocks: the
- *          first kernel's second half is a programmatic dependent launch that
- *          runs beside the first half's pass (four launches in stream order;
- *          a later kernel on `stream` still starts after all of them).
+ *          of the SMs idle, the call runs in two pieces of its blocks (3/8
+ *          and 5/8): the first kernel's second piece is a programmatic
+ *          dependent launch that runs beside the first piece's pass (four
+ *          launches in stream order; a later kernel on `stream` still starts
+ *          after all of them).
  * Precision. D = 64: fp32 arithmetic on the CUDA cores. D = 128: the
  * sequential pass runs its contractions (K S^T, Q S^T, T and M times the
  * right-hand side, the state update) on the tensor cores as three-term split

@@ -1538,29 +1538,34 @@ cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
   } else {
     // The sequential pass occupies one SM per (stream, head, value slice) and
     // leaves the others idle, while the prep of every sub-chunk must precede
-    // the pass that reads it. So the call runs in pieces of sub-chunks: prep
-    // piece k + 1 is launched as a programmatic dependent of pass piece k and
-    // runs on the idle SMs while that pass runs (it reads only the inputs and
-    // writes only its own sub-chunks' images); pass piece k + 1 starts when
-    // prep piece k + 1 has completed, which is after pass piece k (see
-    // gdn_prep_tc_kernel), and continues from the state that pass stored.
+    // the pass that reads it. So the call runs in two pieces of sub-chunks:
+    // the second prep is launched as a programmatic dependent of the first
+    // pass and runs on the idle SMs while that pass runs (it reads only the
+    // inputs and writes only its own sub-chunks' images); the second pass
+    // starts when the second prep has completed, which is after the first
+    // pass (see gdn_prep_tc_kernel), and continues from the state that pass
+    // stored.
     int sms = 0;
     cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    // Two halves: each further piece adds a launch hand-off of 5-7 us
-    // (measured on the 512p call, 32 sub-chunks: 0.161 ms in two pieces,
-    // 0.169 in four, 0.186 in eight, 0.177 unsplit). Split only when the pass
-    // leaves at least half of the SMs to the prep.
+    // Two pieces: each further piece adds a launch hand-off of 5-7 us
+    // (measured on the 512p call, 32 sub-chunks: 0.161 ms in two halves,
+    // 0.169 in four pieces, 0.186 in eight, 0.177 unsplit). The first piece
+    // takes 3/8 of the sub-chunks: its prep is exposed, while the larger
+    // second prep still fits beside the first pass (first pieces of 10, 12,
+    // 14 and 16 of 32: 0.166, 0.158, 0.162 and 0.162 ms). Split only when the
+    // pass leaves at least half of the SMs to the prep.
     const int pass_ctas = (D / kTcSlice) * p.H * p.n_streams;
-    const int piece = (p.n_sub >= kGdnSplitMin && 2 * pass_ctas <= sms) ? (p.n_sub + 1) / 2
+    const int first = (p.n_sub >= kGdnSplitMin && 2 * pass_ctas <= sms) ? (3 * p.n_sub + 7) / 8
                                                                         : p.n_sub;
-    for (int jb = 0; jb < p.n_sub; jb += piece) {
+    for (int jb = 0; jb < p.n_sub;) {
       GdnParams q = p;
       q.j_begin = jb;
-      q.j_end = jb + piece < p.n_sub ? jb + piece : p.n_sub;
-      q.pdl_wait = jb > 0;
+      q.j_end = jb == 0 ? first : p.n_sub;
+      jb = q.j_end;
+      q.pdl_wait = q.j_begin > 0;
       const dim3 pg((unsigned)(q.j_end - q.j_begin), (unsigned)p.H, (unsigned)p.n_streams);
-      if (jb == 0) {
+      if (q.j_begin == 0) {
         gdn_prep_tc_kernel<T><<<pg, kGdnThreads, psmem, st>>>(q);
       } else {
         cudaLaunchConfig_t lc = {};

@@ -146,6 +146,14 @@ def test_gdn_pieces_with_ragged_tail(dtype):
     _run_streams(w, [(1, 1), (1, 0), (1, 1)], 0.02, 0.0)
 
 
+def test_gdn_many_heads_one_piece():
+    # 2,048 tokens per call (32 sub-chunks) over 4 streams x 12 heads: the
+    # pass needs 96 CTAs, more than half of the SMs, so a call runs as one
+    # piece; then a call with one active stream (24 CTAs), which is split.
+    w = _w(128, "bf16", 32, 64, B=4, H=12, seed=7)
+    _run_streams(w, [(1, 1, 1, 1), (0, 0, 1, 0)], 0.002, 0.0)
+
+
 def test_gdn_zero_tokens_and_no_active_stream_are_no_ops():
     gdn = _gdn()
     st0 = torch.randn(2, 2, 64, 64, device="cuda")
