@@ -452,12 +452,14 @@ typedef struct {
  *          keys and queries, the triangular inverse T of the chunkwise form
  *          and M = scale P T (P the decay-masked q.k matrix) into the
  *          workspace; the other walks the blocks in order and updates the
- *          state. With D = 128, at least 8 blocks and a pass that leaves half
- *          of the SMs idle, the call runs in two pieces of its blocks (3/8
- *          and 5/8): the first kernel's second piece is a programmatic
- *          dependent launch that runs beside the first piece's pass (four
- *          launches in stream order; a later kernel on `stream` still starts
- *          after all of them).
+ *          state. With D = 128 the kernels are chained by programmatic
+ *          dependent launches (the pass sets up while its prep finishes), and
+ *          a call of at least 8 blocks whose pass leaves half of the SMs idle
+ *          runs in two pieces of its blocks (3/8 and 5/8), the second piece's
+ *          prep beside the first piece's pass. A later kernel on `stream`
+ *          starts after all of them (one that the caller launches as a
+ *          programmatic dependent must execute griddepcontrol.wait before it
+ *          reads the outputs or the state).
  * Precision. D = 64: fp32 arithmetic on the CUDA cores. D = 128: the
  * sequential pass runs its contractions (K S^T, Q S^T, T and M times the
  * right-hand side, the state update) on the tensor cores as three-term split

@@ -776,9 +776,14 @@ template <typename T>
 __global__ void __launch_bounds__(kGdnThreads, kPrepTcCtasPerSm)
     gdn_prep_tc_kernel(const __grid_constant__ GdnParams p) {
   prep_tc_body<T>(p);
+  // The pass that reads these images is a programmatic dependent of this
+  // grid: it may be scheduled once every CTA has done its work (signalling
+  // earlier would let its CTAs take whole SMs from this grid's later CTAs);
+  // it runs its set-up and then waits for this grid to complete.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // A prep piece launched while the previous pass piece still runs
   // (programmatic dependent launch) must not complete before that pass: the
-  // next pass piece, which starts when this grid completes, continues from
+  // next pass piece, which waits for this grid to complete, continues from
   // its state. One thread of the last CTA waits for the previous grid, after
   // its own work, so the other CTAs leave their slots free.
   if (p.pdl_wait && threadIdx.x == 0 && blockIdx.x == gridDim.x - 1 &&
@@ -1232,6 +1237,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_st = tmem, t_d1 = tmem + 64, t_d2 = tmem + 128;
+  // launched as a programmatic dependent of the prep: nothing the prep (or,
+  // through it, the previous pass piece) writes is read before this point
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   auto fail = [&]() {
     *abort_flag = 1;
     atomicOr(status, kDeviceErrTimeout);
@@ -1541,10 +1549,12 @@ cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
     // the pass that reads it. So the call runs in two pieces of sub-chunks:
     // the second prep is launched as a programmatic dependent of the first
     // pass and runs on the idle SMs while that pass runs (it reads only the
-    // inputs and writes only its own sub-chunks' images); the second pass
-    // starts when the second prep has completed, which is after the first
-    // pass (see gdn_prep_tc_kernel), and continues from the state that pass
-    // stored.
+    // inputs and writes only its own sub-chunks' images). Every pass is a
+    // programmatic dependent of its prep: it runs its set-up once the prep's
+    // CTAs have done their work and reads nothing before the prep grid has
+    // completed, which for the second prep is after the first pass (see
+    // gdn_prep_tc_kernel); so the second pass continues from the state the
+    // first one stored.
     int sms = 0;
     cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
@@ -1581,8 +1591,22 @@ cudaError_t launch_gdn_t(const GdnParams& p, cudaStream_t st) {
         e = cudaLaunchKernelEx(&lc, gdn_prep_tc_kernel<T>, q);
         if (e != cudaSuccess) return e;
       }
-      gdn_tc_kernel<T><<<dim3(D / kTcSlice, p.H, p.n_streams), kTcThreads, smem, st>>>(q);
-      e = cudaGetLastError();
+      {
+        // the pass as a programmatic dependent of its prep: its set-up and
+        // launch overlap the end of the prep (measured 0.150 against 0.157
+        // ms per 512p call)
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(D / kTcSlice, p.H, p.n_streams);
+        lc.blockDim = dim3(kTcThreads);
+        lc.dynamicSmemBytes = smem;
+        lc.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = at;
+        lc.numAttrs = 1;
+        e = cudaLaunchKernelEx(&lc, gdn_tc_kernel<T>, q);
+      }
       if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
