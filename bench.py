@@ -235,13 +235,13 @@ def gdn_flops_per_token(D: int, ct: int = 64) -> float:
 
 def gdn_launches_per_call(w, n_active: int) -> int:
     """Kernels one sa_gdn_chunk call launches: the prep and the sequential
-    pass, or both twice when the library splits a D = 128 call of at least 8
+    pass, or both twice when the library splits a call of at least 8
     sub-chunks into two pieces (the pass then leaves at least half the SMs to
     the prep of the second piece)."""
     import torch
     n_sub = (w.Lc + 63) // 64
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    split = w.D == 128 and n_sub >= 8 and 2 * (w.D // 64) * w.H * n_active <= sms
+    split = n_sub >= 8 and 2 * (w.D // 64) * w.H * n_active <= sms
     return 4 if split else 2
 
 
@@ -398,18 +398,19 @@ def run_gdn(args, w, rank, world):
     avg_launch_s = statistics.mean(launch_ms) / 1000.0
     achieved = flops_per_launch / avg_launch_s / 1e12
     alu_peak = FP32_LANES_PER_SM * SM_COUNT * 2 * SM_MAX_GHZ / 1e3
-    tc = w.D == 128  # the sequential pass runs on the tensor cores (bf16 split products)
     hbm_pk, bf16_burst, _, pk_src = peaks()
-    peak = bf16_burst if tc else alu_peak
+    peak = bf16_burst   # both kernels issue bf16 tensor-core MMAs (split products)
     n_sub = (w.Lc + 63) // 64
     # tensor-core FLOPs issued per call, per (head, 64-token block), three split
-    # terms each: in the prep kernel the Gram matrices [K^;Q^] K^T (2 x 128 x 64 x D,
-    # once per head); in the sequential pass (once per 64-column value slice, two
-    # slices per head) K^S^T and Q^S^T (2 x 128 x D x 64), T and M times the
-    # right-hand side (2 x 128 x 64 x 64) and the state update (2 x D x 64 x 64)
+    # terms each, with the key dims Dk = 128 (D = 64 is padded): in the prep
+    # kernel the Gram matrices [K^;Q^] K^T (2 x 128 x 64 x Dk, once per head); in
+    # the sequential pass (once per 64-column value slice, D / 64 slices per
+    # head) K^S^T and Q^S^T (2 x 128 x Dk x 64), T and M times the right-hand
+    # side (2 x 128 x 64 x 64) and the state update (2 x Dk x 64 x 64)
     slices = w.D // 64
-    issued = 3.0 * (2 * 128 * 64 * w.D + slices * (2 * 128 * w.D * 64 + 2 * 128 * 64 * 64 +
-                                                    2 * w.D * 64 * 64)) * n_sub * w.H * B
+    Dk = 128
+    issued = 3.0 * (2 * 128 * 64 * Dk + slices * (2 * 128 * Dk * 64 + 2 * 128 * 64 * 64 +
+                                                   2 * Dk * 64 * 64)) * n_sub * w.H * B
     bytes_per_launch = B * (w.Lc * w.H * w.D * esz * 4 + w.Lc * w.H * 8 + 2 * w.H * w.D * w.D * 4)
     # (the workspace of the prep kernel's per-block output is written and read
     # back, mostly through L2, and is not algorithmic traffic)
@@ -460,17 +461,15 @@ def run_gdn(args, w, rank, world):
         "config": gdn_config_json(w, world, g_scale),
         "ms_per_chunk": ms_step / chunks_per_step,
         "launch_mode": "cuda graph of one step, replayed",
-        "roofline": {"bound": "tensor" if tc else "alu",
-                     "kernel": ("gdn_prep_tc_kernel + gdn_tc_kernel (one call)" if tc else
-                                f"gdn_prep_kernel<{w.D}> + gdn_chunk_kernel<{w.D}> (one call)"),
+        "roofline": {"bound": "tensor",
+                     "kernel": "gdn_prep_tc_kernel + gdn_tc_kernel (one call)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
-                     "peak_source": (f"{pk_src} bf16 burst (the sequential pass issues bf16 "
-                                     f"tensor-core MMAs)" if tc else
-                                     "derived: 148 SMs x 128 fp32 lanes x 2 FLOP (FMA) x 1.965 GHz"),
+                     "peak_source": (f"{pk_src} bf16 burst (both kernels issue bf16 "
+                                     f"tensor-core MMAs)"),
                      "frac_of_fp32_alu_peak": achieved / alu_peak,
-                     "issued_tensor_flops_per_launch": issued if tc else 0.0,
-                     "issued_tensor_tflops": (issued / avg_launch_s / 1e12) if tc else 0.0,
+                     "issued_tensor_flops_per_launch": issued,
+                     "issued_tensor_tflops": issued / avg_launch_s / 1e12,
                      "algorithmic_flops_per_launch": flops_per_launch,
                      "hbm_bytes_per_launch": bytes_per_launch,
                      "hbm_frac": bytes_per_launch / avg_launch_s / 1e9 / hbm,

@@ -460,13 +460,14 @@ typedef struct {
  *          starts after all of them (one that the caller launches as a
  *          programmatic dependent must execute griddepcontrol.wait before it
  *          reads the outputs or the state).
- * Precision. D = 64: fp32 arithmetic on the CUDA cores. D = 128: the
- * sequential pass runs its contractions (K S^T, Q S^T, T and M times the
- * right-hand side, the state update) on the tensor cores as three-term split
- * products of bf16 operands (x = hi + lo, a.b ~ a_hi.b_hi + a_hi.b_lo +
- * a_lo.b_hi, fp32 accumulation: about 2^-16 relative per product, within
- * 1e-4 of the fp64 recurrence on the outputs and the state), with the state
- * in tensor memory for the whole call; everything else is fp32.
+ * Precision. The sequential pass runs its contractions (K S^T, Q S^T, T and
+ * M times the right-hand side, the state update), and the first kernel its
+ * Gram matrices, on the tensor cores as three-term split products of bf16
+ * operands (x = hi + lo, a.b ~ a_hi.b_hi + a_hi.b_lo + a_lo.b_hi, fp32
+ * accumulation: about 2^-16 relative per product, within 1e-4 of the fp64
+ * recurrence on the outputs and the state), with the state in tensor memory
+ * for the whole call; everything else is fp32. D = 64 runs through the same
+ * kernels with the key dims padded to 128 with zeros.
  * active: host array of B flags, NULL = all; an inactive stream's state and
  * out rows are untouched. The state is fp32; outputs are rounded once to
  * cfg->dtype. Asynchronous on `stream`, graph-capturable.

@@ -144,11 +144,11 @@ size_t attend_partials_bytes(int D, int num_sms, int64_t max_units);
 
 // Gated DeltaNet block (gdn.cu): T tokens of each listed stream; q, k, v, out
 // [B][T][H][D], g and beta [B][T][H], state [B][H][D][D] fp32 in place.
-// workspace: a 1 KiB header (device status word of the tensor-core path),
-// then per (listed stream, head, 64-token sub-chunk) the prep kernel's
-// output (D = 128: the bf16 hi/lo operand images of the sequential
-// tensor-core kernel; D = 64: fp32 T and M); gdn_workspace_bytes(n_streams,
-// H, D, T) bytes, 16-byte aligned.
+// workspace: a 1 KiB header (the call's device status word), then per
+// (listed stream, head, 64-token sub-chunk) the prep kernel's output: the
+// bf16 hi/lo operand images of the sequential tensor-core kernel (128 key
+// dims wide for D = 64 too); gdn_workspace_bytes(n_streams, H, D, T) bytes,
+// 16-byte aligned.
 struct GdnParams {
   float* state;
   const void* q;
@@ -170,7 +170,6 @@ struct GdnParams {
   int32_t stream_of[SA_MAX_STREAMS];
 };
 size_t gdn_workspace_bytes(int B, int H, int D, int64_t T);
-size_t gdn_smem_bytes(int D, int dtype);
 cudaError_t launch_gdn(const GdnParams& p, int D, int dtype, cudaStream_t st);
 
 cudaError_t launch_append(const AppendParams& p, int dtype, int num_sms, cudaStream_t st);

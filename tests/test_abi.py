@@ -186,16 +186,16 @@ def test_gdn_chunk_validates_pointers():
         _lib.SA_ERR_INVALID_ARG                      # workspace NULL
     n = ctypes.c_size_t()
     assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
-    # header + B * H * ceil(T / 64) blocks: 96 KiB of operand images for D = 128
-    # (tensor-core pass), 32 KiB of fp32 T and M for D = 64
-    per = 98304 if c.head_dim == 128 else 32768
+    # header + B * H * ceil(T / 64) blocks of 96 KiB of operand images (the
+    # images are 128 key dims wide for D = 64 too)
+    per = 98304
     assert n.value == 1024 + 2 * 3 * 1 * per
     c.tokens = 65
     assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
     assert n.value == 1024 + 2 * 3 * 2 * per
     c.head_dim = 64
     assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
-    assert n.value == 1024 + 2 * 3 * 2 * 32768
+    assert n.value == 1024 + 2 * 3 * 2 * per
     c.head_dim = 128
     assert L.sa_gdn_workspace_size(ctypes.byref(c), ctypes.byref(n)) == _lib.SA_OK
     assert L.sa_gdn_chunk(ctypes.byref(c), p, p, p, p, p, p, p, p, n.value - 16, None,
