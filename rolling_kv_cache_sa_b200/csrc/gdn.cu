@@ -878,7 +878,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
     if (ok) {
       float x[kTcCols];
 #pragma unroll
-      for (int i = 0; i < kTcCols; ++i) x[i] = key_in ? Sg[(size_t)(vcol + cb + i) * DI + r] : 0.f;
+      // (from L2: the state was written by the previous pass piece or call,
+      // whose completion this grid sees through the launch chain)
+      for (int i = 0; i < kTcCols; ++i)
+        x[i] = key_in ? __ldcg(Sg + (size_t)(vcol + cb + i) * DI + r) : 0.f;
       put_row<kTcCols>(smc, L::st, L::st + 16384, r, cb / 8, x);
       const float dec = ptx::ex2(gcum(0, kCt - 1));
 #pragma unroll
