@@ -40,7 +40,7 @@ METRIC = "streamed chunks/s and attention TFLOP/s (% of B200 BF16 peak) per conf
 # DRAM bytes (read + write) per launch of the attention kernel, from the ncu
 # capture summarised in profiles/ (512p, steady chunk with 7168 keys), keyed by
 # a hash of the kernel sources it was taken on: a changed kernel reports null.
-PROFILED_TRAFFIC = {"031578c3b0278178": 137.59e6, "031578c3b0278178/e4m3": 54.17e6}
+PROFILED_TRAFFIC = {"d16678532cbd06c5": 136.73e6, "d16678532cbd06c5/e4m3": 54.07e6}
 
 
 def attend_source_hash() -> str:
