@@ -943,14 +943,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
 #pragma unroll
         for (int i = 0; i < kTcCols; ++i) x[i] *= wt;
         put_row<kTcCols>(smc, L::uu, L::uu + 8192, tr, cb / 8, x);
-      } else if (tok_in) {
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(L::B_U));
+      } else {
+        // query rows: MMA3 reads only the key rows' image, so they arrive
+        // before storing their outputs (the stores then overlap MMA3 instead
+        // of delaying its start; measured 0.1497 against 0.1509 ms per 512p
+        // call)
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(L::B_U));
+        if (tok_in) {
 #pragma unroll
-        for (int i = 0; i < kTcCols; ++i) x[i] += vv[i];
-        store_row<kTcCols>(out + bh0 + (size_t)(t0 + tr) * tok_stride, x);
+          for (int i = 0; i < kTcCols; ++i) x[i] += vv[i];
+          store_row<kTcCols>(out + bh0 + (size_t)(t0 + tr) * tok_stride, x);
+        }
       }
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(L::B_U));
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_D3), par, abort_flag, kTcTimeoutNs))) {
         ok = false;
         break;
