@@ -534,12 +534,15 @@ __global__ void __launch_bounds__(kGdnThreads, kPrepTcCtasPerSm)
 }
 
 // ---------------------------------------------------------------- tensor-core sequential pass
-// D = 64 or 128. One CTA per (stream, head, 64 value dims of the state): 16 warps
-// for the elementwise work (four threads per TMEM lane r, 16 value columns
-// each) and 1 warp that issues the copies and the tcgen05 MMAs. The state slice lives in TMEM, transposed
-// (lane = key dim k, column = value dim v: ST[k][v] = S[v][k]), for the whole
-// call. Per 64-token sub-chunk j, with its operand images from the prep
-// kernel (KQ, TM) arriving by bulk copy one or two sub-chunks ahead:
+// D = 64 or 128. One CTA per (stream, head, 64 value dims of the state): 16
+// warps for the elementwise work (four threads per TMEM lane r, 16 value
+// columns each) and 1 warp that issues the copies and the tcgen05 MMAs. The
+// state slice lives in TMEM, transposed (lane = key dim k, column = value dim
+// v: ST[k][v] = S[v][k]), for the whole launch; a launch walks the sub-chunk
+// range [j_begin, j_end) of the call (a call may run in two pieces, see
+// launch_gdn_t) and loads and stores the state in global memory at its ends.
+// Per 64-token sub-chunk j, with its operand images from the prep kernel (KQ,
+// TM) arriving by bulk copy one or two sub-chunks ahead:
 //   MMA1  D1[t][v]      = sum_k [K^;Q^][t][k] S[v][k]       (K^ S0^T and Q^ S0^T)
 //   (threads) RHS[t][v] = beta_t (v_t[v] - e^{G_t} D1[t][v]); O_in = scale e^{G_t} D1[64+t][v]
 //   MMA2  D2[t][v]      = sum_s [T;M][t][s] RHS[s][v]      (U = T RHS and the intra-chunk outputs)
