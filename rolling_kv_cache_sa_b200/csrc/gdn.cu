@@ -924,14 +924,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) gdn_tc_kernel(const __grid_cons
 #pragma unroll
         for (int i = 0; i < kTcCols; ++i) vv[i] = bt * (vv[i] - eg * x[i]);
         put_row<kTcCols>(smc, L::rhs, L::rhs + 8192, tr, cb / 8, vv);
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(L::B_RHS));
       } else {
+        // query rows: MMA2 reads only the key rows' image, so they arrive first
+        // and form their inter-chunk outputs (registers) while MMA2 runs
+        // (0.1485 against 0.1496 ms per 512p call)
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(L::B_RHS));
         const float sc = p.scale * eg;
 #pragma unroll
         for (int i = 0; i < kTcCols; ++i) vv[i] = sc * x[i];   // (query rows: the inter-chunk output)
       }
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(L::B_RHS));
       // the gates of the next sub-chunk, while MMA2 runs
       if (jl + 1 < nl) gates(jl + 1);
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar(L::B_D2), par, abort_flag, kTcTimeoutNs))) {
